@@ -1,0 +1,170 @@
+"""float64 CPU oracle for RoPE and causal / windowed varlen attention (standard and paired-head).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its
+``cpu_baseline`` leg and ``--impl reference``) may import this package. The product package
+``paired_heads_b200`` never imports it, and it never imports the product package: the two share
+no code. The arithmetic lives in ``oracle.c`` (plain C, float64, explicit loops); this module only
+marshals numpy arrays into it.
+
+Sources: the "modded-nanogpt Paired Head Attention record" page (sections "core idea",
+"interleave semantics under the causal mask", "staggered rotary", "sequence length and window
+handling", "4. interleave index in the Triton kernel"); the "Training an LLM from scratch (part
+2)" page, sections "2. RoPE" and "4. GQA & FlashAttention"; the "ChatGPT" source notes, section
+"SingleHeadAttention"; the "mHC module" page (max-subtracted softmax).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_c = ctypes.c_int
+_l = ctypes.c_int64
+_d = ctypes.c_double
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_rope.argtypes = [_f64p, _i32p, _l, _c, _c, _c, _c, _d]
+        lib.oracle_interleave.argtypes = [_f64p, _f64p, _l, _c, _c]
+        lib.oracle_deinterleave.argtypes = [_f64p, _f64p, _l, _c, _c]
+        lib.oracle_attention.argtypes = [_f64p, _f64p, _f64p, _i64p, _c, _c, _c, _c, _c, _c, _d,
+                                         _f64p, _f64p]
+        lib.oracle_attention_rows.argtypes = [_f64p, _f64p, _f64p, _i64p, _c, _c, _c, _c, _c, _c,
+                                              _d, _i64p, _l, _f64p, _f64p]
+        lib.oracle_attn_fwd.argtypes = [_f64p, _f64p, _f64p, _i32p, _c, _c, _c, _c, _c, _c, _c,
+                                        _d, _f64p, _f64p]
+        for f in ("oracle_rope", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
+                  "oracle_attention_rows", "oracle_attn_fwd"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"{what}: oracle rejected the arguments (rc={rc})")
+
+
+def rope(x, positions, paired: bool = False, stagger: bool = False, base: float = 10000.0):
+    """Rotate x[T][H][hd] (returns a new float64 array). Phase of token t, head h is
+    positions[t] (standard) or 2*positions[t] + (h % 2 if stagger) (paired)."""
+    y = _f64(x).copy()
+    T, H, hd = y.shape
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    assert pos.shape == (T,)
+    _check(_load().oracle_rope(y, pos, T, H, hd, int(paired), int(stagger), float(base)), "rope")
+    return y
+
+
+def interleave(x):
+    """Explicit paired interleave [T][H][d] -> [2T][H/2][d] (copy loop in C)."""
+    x = _f64(x)
+    T, H, d = x.shape
+    y = np.empty((2 * T, H // 2, d), dtype=np.float64)
+    _check(_load().oracle_interleave(x, y, T, H, d), "interleave")
+    return y
+
+
+def deinterleave(y):
+    """Inverse of :func:`interleave`: [2T][H/2][d] -> [T][H][d]."""
+    y = _f64(y)
+    S, Hp, d = y.shape
+    x = np.empty((S // 2, 2 * Hp, d), dtype=np.float64)
+    _check(_load().oracle_deinterleave(y, x, S // 2, 2 * Hp, d), "deinterleave")
+    return x
+
+
+def attention_slots(q, k, v, cu_slots, causal=True, window=0, scale=None):
+    """Attention over slot-major buffers (no pairing): q[S][H][hd], k,v[S][Hkv][hd]; documents
+    are the slot ranges of cu_slots. Returns (o[S][H][hd], lse[S][H])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    S, H, hd = q.shape
+    Hkv = k.shape[1]
+    cu = np.ascontiguousarray(cu_slots, dtype=np.int64)
+    scale = 1.0 / np.sqrt(hd) if scale is None or scale <= 0 else float(scale)
+    o = np.zeros_like(q)
+    lse = np.zeros((S, H), dtype=np.float64)
+    _check(_load().oracle_attention(q, k, v, cu, len(cu) - 1, H, Hkv, hd, int(causal),
+                                    int(window), scale, o, lse), "attention")
+    return o, lse
+
+
+def attn_fwd(q, k, v, cu_seqlens, causal=True, window=0, paired=False, scale=None):
+    """Full forward in token layout: q[T][H][hd], k,v[T][Hkv][hd], cu_seqlens in tokens.
+    Paired: explicit interleave, doubled cu_seqlens, H/2 heads, window unchanged, de-interleave.
+    Returns (o[T][H][hd], lse[T][H])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, H, hd = q.shape
+    Hkv = k.shape[1]
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    scale = 1.0 / np.sqrt(hd) if scale is None or scale <= 0 else float(scale)
+    o = np.zeros_like(q)
+    lse = np.zeros((T, H), dtype=np.float64)
+    _check(_load().oracle_attn_fwd(q, k, v, cu, len(cu) - 1, H, Hkv, hd, int(causal),
+                                   int(window), int(paired), scale, o, lse), "attn_fwd")
+    return o, lse
+
+
+def attn_rows(q, k, v, cu_seqlens, rows, causal=True, window=0, paired=False, scale=None):
+    """Selected output rows of :func:`attn_fwd`, computed one by one.
+
+    ``rows`` index the caller's [T][H] row space as t*H + h. For the paired case the rows are
+    computed on the interleaved sequence addressed as a view of the same buffers -- slot s, head
+    h' lives at flat offset (s*(H/2) + h')*hd, the identity that the tests pin against the
+    explicit interleave bit for bit -- so no 2T copies are made. Returns (o[n][hd], lse[n])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, H, hd = q.shape
+    Hkv = k.shape[1]
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    scale = 1.0 / np.sqrt(hd) if scale is None or scale <= 0 else float(scale)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    if paired:
+        # token t, head h  ->  slot 2t + h//(H/2), head h % (H/2)
+        t, h = rows // H, rows % H
+        Hp = H // 2
+        slot_rows = (2 * t + h // Hp) * Hp + (h % Hp)
+        qs = q.reshape(2 * T, Hp, hd)
+        ks = k.reshape(2 * T, Hkv // 2, hd)
+        vs = v.reshape(2 * T, Hkv // 2, hd)
+        cu_s = np.ascontiguousarray(2 * cu)
+        Hs, Hkvs = Hp, Hkv // 2
+    else:
+        slot_rows, qs, ks, vs, cu_s, Hs, Hkvs = rows, q, k, v, np.ascontiguousarray(cu), H, Hkv
+    slot_rows = np.ascontiguousarray(slot_rows, dtype=np.int64)
+    n = len(slot_rows)
+    o = np.zeros((n, hd), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    _check(_load().oracle_attention_rows(np.ascontiguousarray(qs), np.ascontiguousarray(ks),
+                                         np.ascontiguousarray(vs), cu_s, len(cu_s) - 1, Hs, Hkvs,
+                                         hd, int(causal), int(window), scale, slot_rows, n, o,
+                                         lse), "attn_rows")
+    return o, lse

@@ -1,0 +1,380 @@
+"""Pins for the float64 oracle against things other than itself: closed forms, the pages' worked
+examples (tests/golden), textbook special cases, library routines, invariants and an
+independently written dense formulation. CPU only."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------- rotary
+
+def test_rope_single_pair_is_plane_rotation():
+    # hd = 2: one pair with frequency base^0 = 1, so position p rotates by p radians. For one pair
+    # the half-split form of the "2. RoPE" section (q*cos + rotate_half(q)*sin) and the adjacent-pair
+    # form coincide: (x0, x1) -> (x0 cos p - x1 sin p, x0 sin p + x1 cos p).
+    p = np.array([0, 1, 2, 7, 100, 4097], dtype=np.int32)
+    x = np.zeros((len(p), 2, 2))
+    x[:, 0, 0] = 1.0          # head 0: e0
+    x[:, 1, 1] = 1.0          # head 1: e1
+    y = oracle.rope(x, p)
+    np.testing.assert_allclose(y[:, 0, 0], np.cos(p), atol=1e-15)
+    np.testing.assert_allclose(y[:, 0, 1], np.sin(p), atol=1e-15)
+    np.testing.assert_allclose(y[:, 1, 0], -np.sin(p), atol=1e-15)
+    np.testing.assert_allclose(y[:, 1, 1], np.cos(p), atol=1e-15)
+
+
+def test_rope_frequencies_base_10000_hd8():
+    # inv_freq = 1 / 10000^(2i/8) for i = 0..3 is exactly 1, 1/10, 1/100, 1/1000 and pair i is
+    # (x[2i], x[2i+1]).
+    freqs = [1.0, 0.1, 0.01, 0.001]
+    p = 37
+    for i, f in enumerate(freqs):
+        x = np.zeros((1, 1, 8))
+        x[0, 0, 2 * i] = 1.0
+        y = oracle.rope(x, np.array([p], dtype=np.int32))[0, 0]
+        expect = np.zeros(8)
+        expect[2 * i] = np.cos(p * f)
+        expect[2 * i + 1] = np.sin(p * f)
+        np.testing.assert_allclose(y, expect, atol=1e-13)
+
+
+def test_rope_position_zero_is_identity_and_norm_preserved():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 3, 64))
+    y0 = oracle.rope(x, np.zeros(6, dtype=np.int32))
+    np.testing.assert_array_equal(y0, x)
+    y = oracle.rope(x, rng.integers(0, 70000, 6).astype(np.int32))
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("hd", [16, 64, 128])
+def test_rope_relative_position_invariance(hd):
+    # q_m . k_n depends only on m - n ("2. RoPE" section).
+    rng = np.random.default_rng(hd)
+    q = rng.standard_normal((1, 1, hd))
+    k = rng.standard_normal((1, 1, hd))
+    for m, n in [(5, 3), (100, 0), (2047, 1000)]:
+        ref = None
+        for delta in [0, 1, 17, 4096, 60000]:
+            qm = oracle.rope(q, np.array([m + delta], dtype=np.int32))
+            kn = oracle.rope(k, np.array([n + delta], dtype=np.int32))
+            d = float(np.sum(qm * kn))
+            if ref is None:
+                ref = d
+            assert abs(d - ref) < 1e-10 * max(1.0, abs(ref))
+
+
+def test_paired_staggered_rope_equals_slot_rope_for_one_pair():
+    # H = 2: the paired table gives head h of token t the phase 2t + h, and the interleave puts it
+    # at slot 2t + h. So paired staggered RoPE followed by the interleave equals the interleave
+    # followed by plain RoPE at the slot index.
+    rng = np.random.default_rng(11)
+    T, hd = 9, 32
+    x = rng.standard_normal((T, 2, hd))
+    a = oracle.interleave(oracle.rope(x, np.arange(T, dtype=np.int32), paired=True, stagger=True))
+    b = oracle.rope(oracle.interleave(x), np.arange(2 * T, dtype=np.int32))
+    np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def test_paired_unstaggered_gives_both_heads_phase_2t():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((5, 4, 16))
+    pos = np.arange(5, dtype=np.int32)
+    a = oracle.rope(x, pos, paired=True, stagger=False)
+    b = oracle.rope(x, 2 * pos)
+    np.testing.assert_array_equal(a, b)
+
+
+# ----------------------------------------------------------------------------- interleave
+
+def test_interleave_worked_example():
+    g = _gold("interleave_example.json")
+    T, H = g["T"], g["H"]
+    labels = {}
+    x = np.zeros((T, H, 1))
+    for h in range(H):
+        for t in range(T):
+            code = 100 * (h + 1) + (t + 1)
+            x[t, h, 0] = code
+            labels[code] = g["before"][h][t]
+    y = oracle.interleave(x)  # [2T][H/2][1]
+    got = [labels[int(c)] for c in y.reshape(-1)]
+    assert got == g["after"]
+
+
+def test_interleave_index_map_example():
+    g = _gold("index_map_example.json")
+    T, H = g["T"], g["H"]
+    x = np.zeros((T, H, 1))
+    for t in range(T):
+        for h in range(H):
+            x[t, h, 0] = 10 * t + h
+    y = oracle.interleave(x)
+    for e in g["map"]:
+        assert y[e["slot"], e["head"], 0] == 10 * e["t"] + e["h"]
+
+
+@pytest.mark.parametrize("T,H,d", [(1, 2, 1), (7, 6, 5), (33, 12, 64), (4, 32, 128)])
+def test_interleave_is_a_view(T, H, d):
+    # The explicit copy loop equals reinterpreting [T][H][d] as [2T][H/2][d] (the page's delayed
+    # reshape), bit for bit; de-interleave inverts it.
+    x = np.random.default_rng(T * H + d).standard_normal((T, H, d))
+    y = oracle.interleave(x)
+    np.testing.assert_array_equal(y, x.reshape(2 * T, H // 2, d))
+    np.testing.assert_array_equal(oracle.deinterleave(y), x)
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _dense_attention(q, k, v, cu, causal, window, scale):
+    """Independent dense formulation: per document, a full score matrix, a boolean mask built from
+    a lower-triangular matrix and a band, and a row softmax."""
+    S, H, hd = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    o = np.zeros_like(q)
+    lse = np.zeros((S, H))
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        n = hi - lo
+        if n == 0:
+            continue
+        mask = np.ones((n, n), dtype=bool)
+        if causal:
+            mask &= np.tril(np.ones((n, n), dtype=bool))
+        if window > 0:
+            ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+            mask &= (ii - jj) < window
+        for h in range(H):
+            Q = q[lo:hi, h, :]
+            K = k[lo:hi, h // G, :]
+            V = v[lo:hi, h // G, :]
+            Sm = np.where(mask, (Q @ K.T) * scale, -np.inf)
+            mx = Sm.max(axis=1, keepdims=True)
+            P = np.exp(Sm - mx)
+            den = P.sum(axis=1, keepdims=True)
+            o[lo:hi, h, :] = (P / den) @ V
+            lse[lo:hi, h] = mx[:, 0] + np.log(den[:, 0])
+    return o, lse
+
+
+CASES = [
+    # doc lens, H, Hkv, hd, causal, window
+    ((5,), 1, 1, 4, True, 0),
+    ((16,), 4, 2, 8, True, 0),
+    ((3, 1, 9, 4), 2, 2, 8, True, 3),
+    ((7, 0, 6), 4, 1, 6, True, 1),
+    ((11, 5), 2, 2, 4, False, 0),
+    ((16, 2), 4, 4, 8, True, 100),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("integer_valued", [False, True])
+def test_loops_match_dense_formulation(case, integer_valued):
+    lens, H, Hkv, hd, causal, window = case
+    rng = np.random.default_rng(len(lens) * 100 + H * 10 + hd)
+    S = sum(lens)
+    if integer_valued:
+        q = rng.integers(-3, 4, (S, H, hd)).astype(np.float64)
+        k = rng.integers(-3, 4, (S, Hkv, hd)).astype(np.float64)
+        v = rng.integers(-3, 4, (S, Hkv, hd)).astype(np.float64)
+    else:
+        q, k, v = (rng.standard_normal((S, n, hd)) for n in (H, Hkv, Hkv))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    scale = 1.0 / np.sqrt(hd)
+    o, lse = oracle.attention_slots(q, k, v, cu, causal, window, scale)
+    od, lsed = _dense_attention(q, k, v, cu, causal, window, scale)
+    np.testing.assert_allclose(o, od, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, lsed, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("case", CASES[:4])
+def test_paired_matches_dense_on_reshaped_sequence(case):
+    lens, H, Hkv, hd, causal, window = case
+    H, Hkv = 2 * H, 2 * Hkv
+    rng = np.random.default_rng(7 + H)
+    T = sum(lens)
+    q, k, v = (rng.standard_normal((T, n, hd)) for n in (H, Hkv, Hkv))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    o, lse = oracle.attn_fwd(q, k, v, cu, causal, window, paired=True)
+    od, lsed = _dense_attention(q.reshape(2 * T, H // 2, hd), k.reshape(2 * T, Hkv // 2, hd),
+                                v.reshape(2 * T, Hkv // 2, hd), 2 * cu.astype(np.int64), causal,
+                                window, 1.0 / np.sqrt(hd))
+    np.testing.assert_allclose(o, od.reshape(T, H, hd), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, lsed.reshape(T, H), atol=1e-12, rtol=0)
+
+
+def test_matches_torch_sdpa_float64():
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    rng = np.random.default_rng(3)
+    S, H, hd = 24, 4, 16
+    q, k, v = (rng.standard_normal((S, H, hd)) for _ in range(3))
+    for window in (0, 5):
+        i = np.arange(S)[:, None]
+        j = np.arange(S)[None, :]
+        allowed = (j <= i) & ((i - j < window) if window > 0 else True)
+        tq, tk, tv = (torch.from_numpy(a).permute(1, 0, 2)[None] for a in (q, k, v))
+        ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(allowed))
+        ref = ref[0].permute(1, 0, 2).numpy()
+        o, _ = oracle.attention_slots(q, k, v, np.array([0, S]), True, window)
+        np.testing.assert_allclose(o, ref, atol=1e-12, rtol=0)
+
+
+def test_softmax_rows_sum_to_one():
+    # V = 1 everywhere: each output is the sum of the row's softmax weights.
+    rng = np.random.default_rng(4)
+    S, H, hd = 40, 4, 8
+    q = rng.standard_normal((S, H, hd)) * 3
+    k = rng.standard_normal((S, 2, hd)) * 3
+    v = np.ones((S, 2, hd))
+    for window in (0, 7):
+        o, _ = oracle.attention_slots(q, k, v, np.array([0, 13, 40]), True, window)
+        assert np.max(np.abs(o - 1.0)) < 1e-12
+
+
+def test_lse_is_log_of_visible_count_when_keys_are_zero():
+    S, H, hd = 30, 2, 4
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((S, H, hd))
+    k = np.zeros((S, H, hd))
+    v = rng.standard_normal((S, H, hd))
+    cu = [0, 11, 30]
+    for window in (0, 4):
+        _, lse = oracle.attention_slots(q, k, v, np.array(cu), True, window)
+        for b in range(2):
+            for i in range(cu[b], cu[b + 1]):
+                n = i - cu[b] + 1
+                if window > 0:
+                    n = min(n, window)
+                np.testing.assert_allclose(lse[i], np.log(n), atol=1e-14)
+
+
+def test_tril_examples():
+    # Single head, K = 0 (equal logits), V one-hot by position: the output row is uniform over the
+    # visible keys, so its support is the mask row.
+    g = _gold("tril_examples.json")
+    for n_str, mask in g["masks"].items():
+        n = int(n_str)
+        q = np.random.default_rng(n).standard_normal((n, 1, n))
+        k = np.zeros((n, 1, n))
+        v = np.eye(n).reshape(n, 1, n)
+        o, _ = oracle.attention_slots(q, k, v, np.array([0, n]), True, 0)
+        support = (o[:, 0, :] > 0).astype(int)
+        assert support.tolist() == mask
+        np.testing.assert_allclose(o[:, 0, :].sum(axis=1), 1.0, atol=1e-14)
+
+
+def test_pages_paired_mask_example():
+    # Paired, two heads, K = 0 and V one-hot over (head, position): the query row at position 4 is
+    # uniform over exactly the keys the page says it sees.
+    g = _gold("mask_example.json")
+    T, H = g["T"], g["H"]
+    hd = H * T
+    q = np.random.default_rng(1).standard_normal((T, H, hd))
+    k = np.zeros((T, H, hd))
+    v = np.zeros((T, H, hd))
+    for h in range(H):
+        for t in range(T):
+            v[t, h, h * T + t] = 1.0
+    o, _ = oracle.attn_fwd(q, k, v, np.array([0, T], dtype=np.int32), causal=True, paired=True)
+    t = g["query_position"] - 1
+    for qh in range(H):
+        vis = g["visible"][f"head{qh + 1}"]
+        expect = np.zeros(hd)
+        n = sum(len(p) for p in vis.values())
+        for kh_name, positions in vis.items():
+            kh = int(kh_name[-1]) - 1
+            for p in positions:
+                expect[kh * T + (p - 1)] = 1.0 / n
+        np.testing.assert_allclose(o[t, qh], expect, atol=1e-15)
+
+
+def test_window_covering_everything_equals_no_window():
+    rng = np.random.default_rng(9)
+    q, k, v = (rng.standard_normal((20, 2, 8)) for _ in range(3))
+    cu = np.array([0, 8, 20])
+    a = oracle.attention_slots(q, k, v, cu, True, 0)
+    b = oracle.attention_slots(q, k, v, cu, True, 12)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_window_one_returns_own_value():
+    rng = np.random.default_rng(10)
+    q = rng.standard_normal((12, 4, 8))
+    k = rng.standard_normal((12, 2, 8))
+    v = rng.standard_normal((12, 2, 8))
+    o, lse = oracle.attention_slots(q, k, v, np.array([0, 5, 12]), True, 1)
+    for h in range(4):
+        np.testing.assert_allclose(o[:, h, :], v[:, h // 2, :], atol=1e-15)
+        np.testing.assert_allclose(lse[:, h], np.sum(q[:, h] * k[:, h // 2], axis=-1) / np.sqrt(8),
+                                   atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    # "4. GQA & FlashAttention": K/V heads repeated with repeat_interleave(H/Hkv) give the same
+    # result as grouped sharing.
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((18, 8, 8))
+    k = rng.standard_normal((18, 2, 8))
+    v = rng.standard_normal((18, 2, 8))
+    cu = np.array([0, 6, 18])
+    a = oracle.attention_slots(q, k, v, cu, True, 4)
+    b = oracle.attention_slots(q, np.repeat(k, 4, axis=1), np.repeat(v, 4, axis=1), cu, True, 4)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_global_and_per_document_positions_agree():
+    rng = np.random.default_rng(13)
+    lens = [5, 9, 3]
+    T, H, hd = sum(lens), 4, 16
+    q, k, v = (rng.standard_normal((T, H, hd)) for _ in range(3))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    glob = np.arange(T, dtype=np.int32)
+    local = np.concatenate([np.arange(n) for n in lens]).astype(np.int32)
+    for paired in (False, True):
+        outs = []
+        for pos in (glob, local):
+            qr = oracle.rope(q, pos, paired=paired, stagger=paired)
+            kr = oracle.rope(k, pos, paired=paired, stagger=paired)
+            outs.append(oracle.attn_fwd(qr, kr, v, cu, True, 3, paired=paired))
+        np.testing.assert_allclose(outs[0][0], outs[1][0], atol=1e-10)
+        np.testing.assert_allclose(outs[0][1], outs[1][1], atol=1e-10)
+
+
+@pytest.mark.parametrize("paired", [False, True])
+def test_rows_variant_equals_full(paired):
+    rng = np.random.default_rng(14)
+    lens = [13, 1, 30, 6]
+    T, H, Hkv, hd = sum(lens), 4, 2, 8
+    q = rng.standard_normal((T, H, hd))
+    k = rng.standard_normal((T, Hkv, hd))
+    v = rng.standard_normal((T, Hkv, hd))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    o, lse = oracle.attn_fwd(q, k, v, cu, True, 5, paired=paired)
+    rows = rng.choice(T * H, 40, replace=False)
+    orow, lrow = oracle.attn_rows(q, k, v, cu, rows, True, 5, paired=paired)
+    np.testing.assert_array_equal(orow, o.reshape(T * H, hd)[rows])
+    np.testing.assert_array_equal(lrow, lse.reshape(-1)[rows])
+
+
+def test_oracle_rejects_bad_arguments():
+    q = np.zeros((4, 3, 8))
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, q, q, np.array([0, 4], dtype=np.int32), paired=True)  # odd heads
+    with pytest.raises(ValueError):
+        oracle.attention_slots(q, q, q, np.array([0, 3, 2]))  # decreasing cu
