@@ -1,0 +1,408 @@
+"""Benchmark: one step = RoPE on q and k + varlen (paired-head) attention forward, on synthetic
+inputs resident in HBM. Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--window W]
+                    [--paired 0|1] [--impl reference]
+
+Default workload: the paired-head varlen packed batch (65,536 tokens, documents ~ geometric(512)
+capped at 2048, 6 heads -> 3 pairs, head_dim 128, bf16, causal, window 128 slots, staggered
+rotary). N > 1 runs under torchrun, one process per GPU, each rank with its own documents of the
+same shape (weak scaling; the forward needs no collective, so only the timing reduce crosses
+ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paired_heads_b200 import synth  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (causal-counted) and % of bf16 tensor peak on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- workload algebra
+
+def visible_pairs(w) -> int:
+    """Number of (query slot, head, visible key) triples of the attention (the causal count)."""
+    mult = 2 if w.paired else 1
+    heads = w.n_heads // mult
+    total = 0
+    for n in w.doc_lens:
+        L = n * mult
+        i = np.arange(L, dtype=np.int64)
+        vis = (i + 1) if w.causal else np.full(L, L, dtype=np.int64)
+        if w.window > 0:
+            vis = np.minimum(vis, w.window)
+        total += int(vis.sum())
+    return total * heads
+
+
+def attn_flops(w) -> float:
+    return 4.0 * w.head_dim * visible_pairs(w)
+
+
+def attn_bytes(w) -> float:
+    esz = 2 if w.dtype == "bf16" else 4
+    return float(w.total * w.head_dim * esz * (2 * w.n_heads + 2 * w.n_kv_heads) + 4 * w.total * w.n_heads)
+
+
+def rope_bytes(w, tab_width: int) -> float:
+    esz = 2 if w.dtype == "bf16" else 4
+    return float(2 * w.total * (w.n_heads + w.n_kv_heads) * w.head_dim * esz
+                 + 2 * 4 * w.total * tab_width)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def pick_workload(args):
+    kw = {}
+    if args.window is not None:
+        kw["window"] = args.window
+    if args.paired is not None:
+        kw["paired"] = bool(args.paired)
+        kw["stagger"] = bool(args.paired)
+    return synth.workload(args.workload, **kw)
+
+
+def workload_config(w) -> dict:
+    return {"workload": w.name, "tokens": w.total, "docs": w.batch, "max_doc_len": w.max_len,
+            "n_heads": w.n_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "causal": w.causal, "window": w.window, "paired": w.paired, "stagger": w.stagger,
+            "rope_positions": w.positions}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(w, budget_tokens: int):
+    """The leading documents of the workload, up to ~budget_tokens tokens (at least one)."""
+    lens, acc = [], 0
+    for n in w.doc_lens:
+        if acc and acc + n > budget_tokens:
+            break
+        lens.append(n)
+        acc += n
+    return w.with_(doc_lens=tuple(lens))
+
+
+def time_oracle(w, budget_tokens: int):
+    """Oracle (float64 C) run of one step (RoPE stored in the buffer dtype + attention) on a
+    bounded sample of the workload. Returns (TFLOP/s, seconds, sample workload, threads)."""
+    import oracle
+
+    s = oracle_sample(w, budget_tokens)
+    inp = synth.make_inputs(s)
+    q, k, v = (synth.to_f64(inp[n]) for n in ("q", "k", "v"))
+    pos = inp["positions"].numpy()
+    t0 = time.perf_counter()
+    qr = oracle.rope_stored(q, pos, w.dtype, w.paired, w.stagger, w.rope_base)
+    kr = oracle.rope_stored(k, pos, w.dtype, w.paired, w.stagger, w.rope_base)
+    oracle.attn_fwd(qr, kr, v, inp["cu_seqlens"].numpy(), w.causal, w.window, w.paired, w.scale)
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return attn_flops(s) / dt / 1e12, dt, s, threads
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="paired_varlen", choices=synth.WORKLOADS)
+    ap.add_argument("--window", type=int, default=None)
+    ap.add_argument("--paired", type=int, default=None)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-tokens", type=int, default=16384)
+    args = ap.parse_args()
+    w = pick_workload(args)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    import torch
+
+    from paired_heads_b200.runner import AttentionStep, StepShape
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    inp = synth.make_inputs(w, rank=rank)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    cu, pos = inp["cu_seqlens"].to(dev), inp["positions"].to(dev)
+    tab_rows = int(inp["positions"].max()) + 1
+    step = AttentionStep(StepShape.of(w, tab_rows), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def run_step():
+        step.rope(q, k, pos)
+        step.attn(q, k, v, cu)
+
+    for _ in range(max(args.warmup, 3)):
+        run_step()
+    torch.cuda.synchronize(dev)
+    status, n_items = step.status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.get_device_properties(dev).index if hasattr(
+        torch.cuda.get_device_properties(dev), "index") else local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        step.rope(q, k, pos)
+        ev[s][1].record(stream)
+        step.attn(q, k, v, cu)
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    rope_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    status, _ = step.status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after timing")
+
+    if dist:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+
+    # ---- end to end through the public API with host buffers
+    host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "cu_seqlens", "positions")}
+    o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dcu, dpos = torch.empty_like(cu), torch.empty_like(pos)
+
+    def e2e_step():
+        dq.copy_(host["q"], non_blocking=True)
+        dk.copy_(host["k"], non_blocking=True)
+        dv.copy_(host["v"], non_blocking=True)
+        dcu.copy_(host["cu_seqlens"], non_blocking=True)
+        dpos.copy_(host["positions"], non_blocking=True)
+        step.rope(dq, dk, dpos)
+        o, lse = step.attn(dq, dk, dv, dcu)
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(5, min(args.steps, 20))
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(host[n].numel() * host[n].element_size() for n in host)
+    d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * 4
+
+    flops = attn_flops(w)
+    peaks, peak_src = load_peaks()
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    tab_width = (2 if w.paired else 1) * w.head_dim
+    kernels = {
+        "rope": {"ms": rope_ms, "bytes": rope_bytes(w, tab_width),
+                 "gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9},
+        "attention": {"ms": attn_ms, "flops": flops, "bytes": attn_bytes(w),
+                      "tflops": attn_tflops,
+                      "gbs": attn_bytes(w) / (attn_ms * 1e-3) / 1e9},
+    }
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    attn_bound = "hbm" if flops / attn_bytes(w) < ridge else "tensor"
+    dominant = "attention" if attn_ms >= rope_ms else "rope"
+    if dominant == "rope" or attn_bound == "hbm":
+        kname = dominant
+        achieved = kernels[kname]["gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        kname = "attention"
+        roof = {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"]}
+    roof["kernel"] = kname
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    roof["traffic"] = load_traffic(w, kname)
+    roof["timing"] = ("CUDA events on the launching stream around each library call in the timed "
+                      "region; the attention call includes its scheduler kernel")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) q/k/v; geometric document lengths)",
+        "config": {**workload_config(w), "parallelism": f"dp{world} (independent documents per rank)",
+                   "l2": "inputs larger than L2 (q,k,v + tables > 126 MB); no flush"},
+        "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
+        "attention_only_tflops": attn_tflops,
+        "tokens_per_s": w.total * world / (ms_per_step * 1e-3),
+        "kernels": kernels,
+        "roofline": roof,
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "work_items": n_items,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, secs, s, thr = time_oracle(w, args.oracle_tokens)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                "seconds": secs,
+                                "sample": f"first {s.batch} documents ({s.total} tokens) of the "
+                                          f"workload: float64 RoPE + attention, full rows"}
+    if rank == 0:
+        print(json.dumps(line))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def load_traffic(w, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this workload and
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    key = f"{w.name}:w{w.window}:p{int(w.paired)}:{kernel}"
+    ent = d.get(key)
+    if not ent:
+        return None
+    from paired_heads_b200 import build as b
+
+    if ent.get("sources_sha") != b.sources_sha():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def run_reference(args, w, rank, world):
+    """The oracle, as it stands, timed on the host cores on a bounded sample per step."""
+    if rank != 0:
+        return
+    for _ in range(max(args.warmup, 0)):
+        pass  # the oracle has no warm-up state; each step is timed from cold
+    vals, secs = [], []
+    tokens = max(2048, args.oracle_tokens // 4)
+    s = None
+    thr = 1
+    for _ in range(args.steps):
+        tf, dt, s, thr = time_oracle(w, tokens)
+        vals.append(tf)
+        secs.append(dt)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {**workload_config(w), "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": f"first {s.batch} documents ({s.total} tokens) per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

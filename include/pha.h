@@ -1,0 +1,149 @@
+/*
+ * pha.h -- C ABI of libpha: B200 (sm_100a) forward pass of causal, rotary-embedded, varlen
+ * multi-head attention, including the paired-head variant.
+ *
+ * Method: the "modded-nanogpt Paired Head Attention record" page (hncyxsy.com/news/170276).
+ * In the paired variant the two heads h and h + H/2 of every token are interleaved by position
+ * into a sequence of twice the length with half the heads: token t, head h lands at slot
+ * 2t + h / (H/2), head h % (H/2) (sections "core idea" and "4. interleave index in the Triton
+ * kernel"). For a contiguous [tokens][H][head_dim] buffer this is a pure reinterpretation as
+ * [2*tokens][H/2][head_dim] (section "zero-copy RoPE and delayed reshape"), so no entry point
+ * ever copies data to interleave it. Rotary tables for the paired path pack positions 2p and
+ * 2p+1 side by side in one row; odd heads read the second half ("staggered rotary",
+ * "2. building the paired rotary table"). Sequence lengths and max_len double on the paired
+ * path while the window stays the same ("sequence length and window handling").
+ *
+ * Conventions shared by all entry points:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless stated otherwise.
+ *     The library allocates no memory and keeps no mutable global state; calls on different
+ *     streams may run concurrently as long as they do not share output or workspace buffers.
+ *   - All work is queued on `stream` (a cudaStream_t; NULL = the legacy default stream) and is
+ *     asynchronous: a return of PHA_OK means "arguments accepted and kernels launched".
+ *   - Argument errors are detected before any launch and return a negative pha_status with
+ *     nothing launched and no memory touched. Launch failures return PHA_ERR_CUDA.
+ *   - Tensors are contiguous, row-major. "bf16" is IEEE bfloat16, "f32" IEEE binary32.
+ */
+#ifndef PHA_H
+#define PHA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pha_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    PHA_OK = 0,
+    PHA_ERR_INVALID = -1,     /* bad pointer, size, shape or alignment */
+    PHA_ERR_UNSUPPORTED = -2, /* well-formed but outside what the kernels implement */
+    PHA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than pha_attn_workspace_bytes() */
+    PHA_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
+} pha_status;
+
+typedef enum { PHA_BF16 = 0, PHA_F32 = 1 } pha_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* pha_status_string(pha_status s);
+
+/*
+ * pha_rope_tables -- fill rotary tables on the device.
+ *   Frequencies f_i = base^(-2i/head_dim), i = 0 .. head_dim/2 - 1 (the "Training an LLM from
+ *   scratch (part 2)" page, section "2. RoPE"); angles and their cosines and sines are computed
+ *   in float64 and rounded to float32.
+ *   paired = 0: width = head_dim; cos_tab[p][j] = cos(p * f_{j/2}), sin_tab likewise.
+ *   paired = 1: width = 2*head_dim; columns [0, head_dim) hold angles 2p * f_{j/2}, columns
+ *               [head_dim, 2*head_dim) hold (2p+1) * f_{(j-head_dim)/2} (the paired table of the
+ *               record page, section "2. building the paired rotary table").
+ *   cos_tab, sin_tab: float[rows][width], 16-byte aligned, written.
+ *   Errors: PHA_ERR_INVALID if a pointer is NULL or misaligned, rows < 0, head_dim odd or
+ *   <= 0, base <= 0.
+ */
+pha_status pha_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
+                           double base, pha_stream_t stream);
+
+/*
+ * pha_rope -- in-place rotary embedding of q and k (record page, sections "zero-copy RoPE and
+ * delayed reshape", "staggered rotary", "4. interleave index in the Triton kernel").
+ *   q: [total_tokens][n_heads][head_dim], k: [total_tokens][n_kv_heads][head_dim], dtype
+ *      `dtype`, 16-byte aligned, read and overwritten. k may be NULL when n_kv_heads == 0.
+ *   cos_tab, sin_tab: float[tab_rows][tab_width] as written by pha_rope_tables, 16-byte aligned.
+ *   positions: int32[total_tokens], the table row of each token.
+ *   For token t, head h, pair i (columns 2i, 2i+1) with c = cos_tab[positions[t]][col0 + 2i],
+ *   s = sin_tab[...][col0 + 2i]:  y[2i] = x[2i] c - x[2i+1] s,  y[2i+1] = x[2i] s + x[2i+1] c,
+ *   where col0 = 0, or col0 = stagger_offset for odd h when paired = 1. Arithmetic is float32;
+ *   bf16 results are rounded to nearest even.
+ *   paired = 0: tab_width must equal head_dim and stagger_offset must be 0.
+ *   paired = 1: tab_width must equal 2*head_dim; stagger_offset is head_dim (the page's
+ *               staggered rotary: odd heads take phase 2p+1) or 0 (both heads take 2p).
+ *   A token whose position lies outside [0, tab_rows) is left unchanged; this is not reported.
+ *   Errors: PHA_ERR_INVALID for NULL/misaligned pointers, negative sizes, n_heads <= 0,
+ *   head_dim not a positive multiple of 16 (bf16) or 8 (f32), or table width / stagger_offset
+ *   not as above.
+ */
+pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
+                    int tab_width, const int32_t* positions, int total_tokens, int n_heads,
+                    int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                    int stagger_offset, pha_stream_t stream);
+
+/*
+ * pha_attn_workspace_bytes -- device workspace that pha_attn_fwd needs: the varlen tile work
+ * list for at most batch * ceil(L/128) * H' tiles (L = max_len, doubled when paired; H' =
+ * n_heads, halved when paired) plus a 256-byte header. Returns 0 for invalid arguments.
+ */
+size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired);
+
+/*
+ * pha_attn_fwd -- varlen attention forward: O and the per-row log-sum-exp.
+ *   q: [total_tokens][n_heads][head_dim]; k, v: [total_tokens][n_kv_heads][head_dim]; dtype
+ *      `dtype`; 16-byte aligned; read only.
+ *   cu_seqlens: int32[batch+1], document boundaries in TOKENS (not doubled), non-decreasing,
+ *      cu_seqlens[0] >= 0, cu_seqlens[batch] <= total_tokens; every document at most max_len
+ *      tokens long. When paired = 1 the library itself doubles the boundaries and max_len.
+ *   Sequence seen by the kernels: standard -- slots = tokens, H' = n_heads, Hkv' = n_kv_heads;
+ *      paired -- the same buffers read as [2*total_tokens][n_heads/2][head_dim] (slot 2t+h/(H/2)).
+ *   Query slot i of the document spanning slots [a, b) attends key slot j iff a <= j < b,
+ *      j <= i when causal, and i - j < window when window > 0 (window counts key slots,
+ *      including the query's own; it is NOT doubled on the paired path). Query head h' uses
+ *      kv head h' / (H'/Hkv') (GQA).
+ *   scale: logit multiplier; scale <= 0 selects 1/sqrt(head_dim).
+ *   o: same shape, dtype and layout as q, written (16-byte aligned).
+ *   lse: float[total_tokens][n_heads] (paired: the same bytes as [2*total_tokens][n_heads/2]),
+ *      lse = ln sum_j exp(scale * q.k_j) over visible keys; may be NULL (then not written).
+ *   workspace: device scratch of at least pha_attn_workspace_bytes(...) bytes, 16-byte aligned;
+ *      its contents need not be initialised. The scheduler kernel writes the work list into it
+ *      and records in its first 8 bytes the number of work items and a device-side status
+ *      (see pha_attn_status). May be NULL for PHA_F32, which does not use it.
+ *   Supported: bf16 with head_dim in {64, 128} (tcgen05 tensor-core kernel); f32 with
+ *      1 <= head_dim <= 128 (exact float32 CUDA-core kernel).
+ *   Errors (before launch): PHA_ERR_INVALID for NULL/misaligned pointers, non-positive sizes,
+ *      n_heads % n_kv_heads != 0, paired with odd n_heads or n_kv_heads;
+ *      PHA_ERR_UNSUPPORTED for causal = 0 with window > 0 and for unsupported dtype/head_dim;
+ *      PHA_ERR_WORKSPACE when the workspace is NULL or too small for the bf16 path.
+ *   Errors found on the device (cu_seqlens not as stated): no output row is written and the
+ *      status word in the workspace is set; read it with pha_attn_status.
+ */
+pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                        int batch, int max_len, int total_tokens, int n_heads, int n_kv_heads,
+                        int head_dim, pha_dtype dtype, int causal, int window, int paired,
+                        float scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                        pha_stream_t stream);
+
+/*
+ * pha_attn_status -- synchronise `stream` and read the device-side status that the last
+ * pha_attn_fwd on this workspace recorded: 0 = fine; 1 = cu_seqlens malformed (decreasing,
+ * negative start, beyond total_tokens, or a document longer than max_len); 2 = more work
+ * items than the workspace holds; 3 = a kernel wait exceeded its time limit and the kernel
+ * gave up. *n_items receives the number of scheduled work items (may be NULL).
+ * Host pointers: status, n_items. Errors: PHA_ERR_INVALID for NULL workspace/status,
+ * PHA_ERR_CUDA if the copy fails.
+ */
+pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PHA_H */

@@ -50,6 +50,7 @@ def _load():
     if _lib is None:
         lib = ctypes.CDLL(build())
         lib.oracle_rope.argtypes = [_f64p, _i32p, _l, _c, _c, _c, _c, _d]
+        lib.oracle_round_bf16.argtypes = [_f64p, _l]
         lib.oracle_interleave.argtypes = [_f64p, _f64p, _l, _c, _c]
         lib.oracle_deinterleave.argtypes = [_f64p, _f64p, _l, _c, _c]
         lib.oracle_attention.argtypes = [_f64p, _f64p, _f64p, _i64p, _c, _c, _c, _c, _c, _c, _d,
@@ -58,7 +59,7 @@ def _load():
                                               _d, _i64p, _l, _f64p, _f64p]
         lib.oracle_attn_fwd.argtypes = [_f64p, _f64p, _f64p, _i32p, _c, _c, _c, _c, _c, _c, _c,
                                         _d, _f64p, _f64p]
-        for f in ("oracle_rope", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
+        for f in ("oracle_rope", "oracle_round_bf16", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
                   "oracle_attention_rows", "oracle_attn_fwd"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -83,6 +84,23 @@ def rope(x, positions, paired: bool = False, stagger: bool = False, base: float 
     assert pos.shape == (T,)
     _check(_load().oracle_rope(y, pos, T, H, hd, int(paired), int(stagger), float(base)), "rope")
     return y
+
+
+def round_bf16(x):
+    """Nearest bfloat16 value of every element (ties to even), as float64 (new array)."""
+    y = _f64(x).copy()
+    _check(_load().oracle_round_bf16(y.reshape(-1), y.size), "round_bf16")
+    return y
+
+
+def rope_stored(x, positions, dtype: str, paired: bool = False, stagger: bool = False,
+                base: float = 10000.0):
+    """RoPE as the pipeline stores it: rotated in float64, then rounded to the buffer's dtype
+    ("bf16": nearest bfloat16; "f32": nearest float32)."""
+    y = rope(x, positions, paired, stagger, base)
+    if dtype == "bf16":
+        return round_bf16(y)
+    return y.astype(np.float32).astype(np.float64)
 
 
 def interleave(x):

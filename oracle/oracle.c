@@ -79,6 +79,31 @@ int oracle_rope(double* x, const int32_t* pos, int64_t n_tok, int n_head, int hd
     return ORACLE_OK;
 }
 
+/* Round every element to the nearest bfloat16 value (ties to even), in place. Used where the
+ * pipeline stores a result in a bf16 buffer: RoPE rotates the bf16 q and k tensors in place
+ * ([PHA] "zero-copy RoPE and delayed reshape": the rotated q, k are the tensors attention reads).
+ * bfloat16 keeps 8 significant bits; the smallest normal value is 2^-126. */
+static double round_bf16(double x)
+{
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    double m = frexp(x, &e); /* x = m * 2^e, 0.5 <= |m| < 1 */
+    int bits = 8;
+    if (e < -125) bits -= (-125 - e); /* subnormal range: fewer significant bits */
+    if (bits < 0) return copysign(0.0, x);
+    double r = nearbyint(ldexp(m, bits)); /* default rounding mode: to nearest, ties to even */
+    double y = ldexp(r, e - bits);
+    if (fabs(y) > 0x1.FEp127) return copysign(INFINITY, x); /* beyond the largest bf16 value */
+    return y;
+}
+
+int oracle_round_bf16(double* x, int64_t n)
+{
+    if (!x || n < 0) return ORACLE_EINVAL;
+    for (int64_t i = 0; i < n; ++i) x[i] = round_bf16(x[i]);
+    return ORACLE_OK;
+}
+
 /* Explicit paired interleave ([PHA] "core idea", "4. interleave index"): token t, head h of
  * x[T][H][d] moves to slot 2t + h/(H/2), head h % (H/2) of y[2T][H/2][d]. A copy loop, not a view. */
 int oracle_interleave(const double* x, double* y, int64_t T, int H, int d)

@@ -1,0 +1,66 @@
+// kernels.cuh -- launchers shared between the kernel files and the C-ABI layer (pha_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace pha {
+
+constexpr int kBlockM = 128;  // query slots per tile
+constexpr int kBlockN = 128;  // key slots per tile
+
+// Workspace header (bytes [0, 256)) followed by int4 work items.
+struct WorkspaceHeader {
+    int n_items;
+    int status;
+};
+constexpr size_t kWorkspaceHeaderBytes = 256;
+
+// One work item = one query tile of one head:
+//   x = first query slot, y = (head << 16) | valid query rows, z = first key slot, w = key end.
+// Keys [z, w) are streamed in tiles of kBlockN starting at z.
+
+struct AttnProblem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const int32_t* cu_seqlens;  // tokens, not doubled
+    int batch;
+    int max_len;          // tokens
+    int total_tokens;
+    int slot_mult;        // 2 when paired (slots = 2 * tokens), else 1
+    int heads;            // H' (heads of the slot view)
+    int kv_heads;         // Hkv'
+    int head_dim;
+    int causal;
+    int window;
+    float scale;
+    void* o;
+    float* lse;
+};
+
+cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
+                               double base, cudaStream_t stream);
+
+cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
+                        int tab_width, const int32_t* positions, int total_tokens, int n_heads,
+                        int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
+                        cudaStream_t stream);
+
+cudaError_t launch_attn_f32(const AttnProblem& p, cudaStream_t stream);
+
+// Builds the varlen work list into `items` (capacity entries) and the header.
+cudaError_t launch_schedule(const AttnProblem& p, int capacity, int4* items, WorkspaceHeader* hdr,
+                            cudaStream_t stream);
+
+// tcgen05 attention over a scheduled work list. tm_q / tm_k / tm_v are 2-D bf16 tensor maps
+// over the slot view ([slots][heads * head_dim] and [slots][kv_heads * head_dim]) with a
+// 64 x 128 box and 128-byte swizzle.
+cudaError_t launch_attn_tc(const AttnProblem& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                           const CUtensorMap& tm_v, const int4* items, WorkspaceHeader* hdr,
+                           cudaStream_t stream);
+
+}  // namespace pha

@@ -1,0 +1,179 @@
+// pha_api.cu -- the extern "C" boundary of libpha (declared in include/pha.h).
+//
+// Validates every argument before any launch, builds the TMA tensor maps for the slot view of
+// the caller's buffers, and queues the kernels on the caller's stream. Allocates nothing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/pha.h"
+#include "kernels.cuh"
+
+using namespace pha;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    // Resolved through the runtime so that the library does not link libcuda directly.
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+// 2-D bf16 map over [rows][width] elements, box 64 x 128, 128-byte swizzle, zero fill outside.
+bool encode_slot_map(CUtensorMap* map, const void* base, uint64_t width, uint64_t rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {width, rows};
+    cuuint64_t strides[1] = {width * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int64_t div_up(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t max_work_items(int batch, int max_len, int n_heads, int paired) {
+    const int64_t slots = static_cast<int64_t>(max_len) * (paired ? 2 : 1);
+    const int64_t heads = paired ? n_heads / 2 : n_heads;
+    return static_cast<int64_t>(batch) * div_up(slots, kBlockM) * heads;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pha_status_string(pha_status s) {
+    switch (s) {
+        case PHA_OK: return "ok";
+        case PHA_ERR_INVALID: return "invalid argument";
+        case PHA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PHA_ERR_WORKSPACE: return "workspace missing or too small";
+        case PHA_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+pha_status pha_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
+                           double base, pha_stream_t stream) {
+    if (!cos_tab || !sin_tab || !aligned16(cos_tab) || !aligned16(sin_tab) || rows < 0 ||
+        head_dim <= 0 || (head_dim & 1) || !(base > 0.0) || (paired != 0 && paired != 1))
+        return PHA_ERR_INVALID;
+    return launch_rope_tables(cos_tab, sin_tab, rows, head_dim, paired, base, stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
+pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
+                    int tab_width, const int32_t* positions, int total_tokens, int n_heads,
+                    int n_kv_heads, int head_dim, pha_dtype dtype, int paired, int stagger_offset,
+                    pha_stream_t stream) {
+    if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
+    const int span = dtype == PHA_BF16 ? 16 : 8;
+    if (!q || !aligned16(q) || (n_kv_heads > 0 && (!k || !aligned16(k))) || !cos_tab || !sin_tab ||
+        !aligned16(cos_tab) || !aligned16(sin_tab) || !positions || tab_rows < 0 ||
+        total_tokens < 0 || n_heads <= 0 || n_kv_heads < 0 || head_dim <= 0 ||
+        head_dim % span != 0 || (paired != 0 && paired != 1))
+        return PHA_ERR_INVALID;
+    if (!paired && (tab_width != head_dim || stagger_offset != 0)) return PHA_ERR_INVALID;
+    if (paired && (tab_width != 2 * head_dim ||
+                   (stagger_offset != 0 && stagger_offset != head_dim)))
+        return PHA_ERR_INVALID;
+    if (total_tokens == 0) return PHA_OK;
+    return launch_rope(q, k, cos_tab, sin_tab, tab_rows, tab_width, positions, total_tokens,
+                       n_heads, n_kv_heads, head_dim, dtype == PHA_BF16, paired, stagger_offset,
+                       stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
+size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired) {
+    (void)head_dim;
+    if (batch <= 0 || max_len < 0 || n_heads <= 0 || (paired && (n_heads & 1))) return 0;
+    return kWorkspaceHeaderBytes +
+           static_cast<size_t>(max_work_items(batch, max_len, n_heads, paired)) * sizeof(int4);
+}
+
+pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                        int batch, int max_len, int total_tokens, int n_heads, int n_kv_heads,
+                        int head_dim, pha_dtype dtype, int causal, int window, int paired,
+                        float scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                        pha_stream_t stream) {
+    if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
+    if (!q || !k || !v || !o || !cu_seqlens || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        !aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || batch <= 0 ||
+        max_len < 0 || total_tokens < 0 || total_tokens > (1 << 29) || n_heads <= 0 ||
+        n_kv_heads <= 0 || n_heads > 4096 || n_heads % n_kv_heads != 0 || head_dim <= 0 ||
+        (causal != 0 && causal != 1) || (paired != 0 && paired != 1) || !(scale == scale))
+        return PHA_ERR_INVALID;
+    if (paired && ((n_heads & 1) || (n_kv_heads & 1))) return PHA_ERR_INVALID;
+    if (!causal && window > 0) return PHA_ERR_UNSUPPORTED;
+    if (dtype == PHA_BF16 && head_dim != 64 && head_dim != 128) return PHA_ERR_UNSUPPORTED;
+    if (dtype == PHA_F32 && head_dim > 128) return PHA_ERR_UNSUPPORTED;
+
+    AttnProblem p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.cu_seqlens = cu_seqlens;
+    p.batch = batch;
+    p.max_len = max_len;
+    p.total_tokens = total_tokens;
+    p.slot_mult = paired ? 2 : 1;
+    p.heads = paired ? n_heads / 2 : n_heads;
+    p.kv_heads = paired ? n_kv_heads / 2 : n_kv_heads;
+    p.head_dim = head_dim;
+    p.causal = causal;
+    p.window = window > 0 ? window : 0;
+    p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
+    p.o = o;
+    p.lse = lse;
+
+    if (dtype == PHA_F32) {
+        if (total_tokens == 0) return PHA_OK;
+        return launch_attn_f32(p, stream) == cudaSuccess ? PHA_OK : PHA_ERR_CUDA;
+    }
+
+    const size_t need = pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PHA_ERR_WORKSPACE;
+    const int64_t cap64 = static_cast<int64_t>((workspace_bytes - kWorkspaceHeaderBytes) / sizeof(int4));
+    const int capacity = cap64 > 0x7FFFFFFF ? 0x7FFFFFFF : static_cast<int>(cap64);
+    auto* hdr = static_cast<WorkspaceHeader*>(workspace);
+    auto* items = reinterpret_cast<int4*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
+
+    if (launch_schedule(p, capacity, items, hdr, stream) != cudaSuccess) return PHA_ERR_CUDA;
+    if (total_tokens == 0) return PHA_OK;
+
+    const uint64_t rows = static_cast<uint64_t>(total_tokens) * p.slot_mult;
+    CUtensorMap tq, tk, tv;
+    if (!encode_slot_map(&tq, q, static_cast<uint64_t>(p.heads) * head_dim, rows) ||
+        !encode_slot_map(&tk, k, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
+        !encode_slot_map(&tv, v, static_cast<uint64_t>(p.kv_heads) * head_dim, rows))
+        return PHA_ERR_CUDA;
+    return launch_attn_tc(p, tq, tk, tv, items, hdr, stream) == cudaSuccess ? PHA_OK : PHA_ERR_CUDA;
+}
+
+pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream) {
+    if (!workspace || !status) return PHA_ERR_INVALID;
+    WorkspaceHeader h{};
+    if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return PHA_ERR_CUDA;
+    *status = h.status;
+    if (n_items) *n_items = h.n_items;
+    return PHA_OK;
+}
+
+}  // extern "C"

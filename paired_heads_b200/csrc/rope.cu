@@ -1,0 +1,164 @@
+// rope.cu -- rotary tables and the in-place rotary kernel (standard and paired / staggered).
+//
+// Method: "modded-nanogpt Paired Head Attention record" page, sections "zero-copy RoPE and delayed
+// reshape" (one elementwise pass y = cos * x + sin * x_flip, x_flip swapping the two members of
+// each adjacent pair), "staggered rotary" and "4. interleave index in the Triton kernel" (odd
+// heads read the second half of the 2*head_dim-wide paired row), "2. building the paired rotary
+// table" (row p packs the angles of positions 2p and 2p+1). Frequencies: "Training an LLM from
+// scratch (part 2)", section "2. RoPE".
+//
+// The rotation is HBM-bound: each thread moves one 32-byte span of one (token, head) row with
+// two 16-byte loads and stores; the table row of a token is shared by all of its heads and is
+// served from L1/L2.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.cuh"
+
+namespace pha {
+
+__global__ void rope_tables_kernel(float* __restrict__ cos_tab, float* __restrict__ sin_tab,
+                                   int rows, int head_dim, int paired, double base) {
+    const int width = paired ? 2 * head_dim : head_dim;
+    const int64_t n = static_cast<int64_t>(rows) * width;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t p = idx / width;
+        const int col = static_cast<int>(idx % width);
+        const int half = col / head_dim;  // paired: 0 -> position 2p, 1 -> position 2p+1
+        const int j = col % head_dim;
+        const double pos = paired ? 2.0 * static_cast<double>(p) + half : static_cast<double>(p);
+        const double freq = pow(base, -2.0 * static_cast<double>(j / 2) / head_dim);
+        double s, c;
+        sincos(pos * freq, &s, &c);
+        cos_tab[idx] = static_cast<float>(c);
+        sin_tab[idx] = static_cast<float>(s);
+    }
+}
+
+template <typename T>
+struct Span32;  // 32 bytes of one row: 16 bf16 or 8 f32
+
+template <>
+struct Span32<__nv_bfloat16> {
+    static constexpr int N = 16;
+    __device__ static void load(const __nv_bfloat16* p, float (&x)[N]) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p);
+        const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            x[2 * e] = __uint_as_float(w[e] << 16);
+            x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    }
+    __device__ static void store(__nv_bfloat16* p, const float (&y)[N]) {
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(p + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+};
+
+template <>
+struct Span32<float> {
+    static constexpr int N = 8;
+    __device__ static void load(const float* p, float (&x)[N]) {
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+    __device__ static void store(float* p, const float (&y)[N]) {
+        *reinterpret_cast<float4*>(p) = make_float4(y[0], y[1], y[2], y[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(y[4], y[5], y[6], y[7]);
+    }
+};
+
+// One thread per 32-byte span. Spans are numbered q first, then k; inside a tensor the order is
+// (token, head, span) so that consecutive threads touch consecutive bytes.
+template <typename T>
+__global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restrict__ k,
+                                                   const float* __restrict__ cos_tab,
+                                                   const float* __restrict__ sin_tab,
+                                                   int tab_rows, int tab_width,
+                                                   const int32_t* __restrict__ positions,
+                                                   int64_t n_q_spans, int64_t n_spans, int n_heads,
+                                                   int n_kv_heads, int head_dim, int paired,
+                                                   int stagger_offset) {
+    constexpr int N = Span32<T>::N;
+    const int spans_per_head = head_dim / N;
+    const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+    if (idx >= n_spans) return;
+    const bool is_k = idx >= n_q_spans;
+    const int64_t local = is_k ? idx - n_q_spans : idx;
+    const int H = is_k ? n_kv_heads : n_heads;
+    T* base = is_k ? k : q;
+    const int span = static_cast<int>(local % spans_per_head);
+    const int64_t th = local / spans_per_head;
+    const int h = static_cast<int>(th % H);
+    const int64_t t = th / H;
+    const int pos = __ldg(positions + t);
+    if (pos < 0 || pos >= tab_rows) return;
+    const int col = ((paired && (h & 1)) ? stagger_offset : 0) + span * N;
+    const float* crow = cos_tab + static_cast<int64_t>(pos) * tab_width + col;
+    const float* srow = sin_tab + static_cast<int64_t>(pos) * tab_width + col;
+    T* p = base + local * N;
+
+    float x[N], y[N], c[N], s[N];
+    Span32<T>::load(p, x);
+#pragma unroll
+    for (int e = 0; e < N; e += 4) {
+        const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + e));
+        const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + e));
+        c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
+        s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
+    }
+    // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign is -1 on
+    // the even member and +1 on the odd member, which is a rotation by +angle.
+#pragma unroll
+    for (int e = 0; e < N; e += 2) {
+        y[e] = fmaf(c[e], x[e], -s[e] * x[e + 1]);
+        y[e + 1] = fmaf(c[e + 1], x[e + 1], s[e + 1] * x[e]);
+    }
+    Span32<T>::store(p, y);
+}
+
+cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
+                               double base, cudaStream_t stream) {
+    const int64_t n = static_cast<int64_t>(rows) * (paired ? 2 : 1) * head_dim;
+    if (n == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    const int grid = static_cast<int>(blocks < 148 * 64 ? blocks : 148 * 64);
+    rope_tables_kernel<<<grid, threads, 0, stream>>>(cos_tab, sin_tab, rows, head_dim, paired,
+                                                     base);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
+                        int tab_width, const int32_t* positions, int total_tokens, int n_heads,
+                        int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
+                        cudaStream_t stream) {
+    const int N = is_bf16 ? 16 : 8;
+    const int64_t n_q = static_cast<int64_t>(total_tokens) * n_heads * (head_dim / N);
+    const int64_t n_all = n_q + static_cast<int64_t>(total_tokens) * n_kv_heads * (head_dim / N);
+    if (n_all == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (n_all + threads - 1) / threads;
+    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    if (is_bf16)
+        rope_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), cos_tab, sin_tab,
+            tab_rows, tab_width, positions, n_q, n_all, n_heads, n_kv_heads, head_dim, paired,
+            stagger_offset);
+    else
+        rope_kernel<float><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+            static_cast<float*>(q), static_cast<float*>(k), cos_tab, sin_tab, tab_rows, tab_width,
+            positions, n_q, n_all, n_heads, n_kv_heads, head_dim, paired, stagger_offset);
+    return cudaGetLastError();
+}
+
+}  // namespace pha

@@ -1,0 +1,154 @@
+"""ctypes binding of libpha (include/pha.h). Argument marshalling only: every step runs in the
+library's CUDA kernels. Importing this module loads libpha.so and raises if it is missing -- there
+is no fallback.
+
+Functions keep the C names. Tensor arguments may be torch tensors (their device pointer is
+passed) or plain integers (raw device addresses). ``stream`` defaults to torch's current stream
+on the tensors' device. A negative status raises :class:`PhaError`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpha.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "pha.h")
+
+PHA_BF16 = 0
+PHA_F32 = 1
+STATUS = {0: "PHA_OK", -1: "PHA_ERR_INVALID", -2: "PHA_ERR_UNSUPPORTED", -3: "PHA_ERR_WORKSPACE",
+          -4: "PHA_ERR_CUDA"}
+DEVICE_STATUS = {0: "ok", 1: "malformed cu_seqlens", 2: "work list overflow", 3: "wait timeout"}
+
+
+class PhaError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(code, code)} ({msg})")
+        self.code = code
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libpha.so is not built ({LIB_PATH}); run `python -m paired_heads_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+_lib.pha_status_string.argtypes = [_i]
+_lib.pha_status_string.restype = ctypes.c_char_p
+_lib.pha_rope_tables.argtypes = [_p, _p, _i, _i, _i, ctypes.c_double, _p]
+_lib.pha_rope.argtypes = [_p, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.pha_attn_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+_lib.pha_attn_workspace_bytes.restype = _sz
+_lib.pha_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                              ctypes.c_float, _p, _p, _p, _sz, _p]
+_lib.pha_attn_status.argtypes = [_p, ctypes.POINTER(_i), ctypes.POINTER(_i), _p]
+for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status"):
+    getattr(_lib, _f).restype = _i
+
+
+def exported_symbols() -> list:
+    """Names of the functions include/pha.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(pha_\w+)\s*\(", text, re.M)))
+
+
+def library():
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream, *tensors):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+
+    for t in tensors:
+        if t is not None and not isinstance(t, int) and t.is_cuda:
+            return torch.cuda.current_stream(t.device).cuda_stream
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise PhaError(fn, rc, _lib.pha_status_string(rc).decode())
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return PHA_BF16
+    if t.dtype == torch.float32:
+        return PHA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def pha_status_string(code: int) -> str:
+    return _lib.pha_status_string(code).decode()
+
+
+def pha_rope_tables(cos_tab, sin_tab, rows: int, head_dim: int, paired: bool, base: float = 10000.0,
+                    stream=None):
+    _check("pha_rope_tables", _lib.pha_rope_tables(_ptr(cos_tab), _ptr(sin_tab), rows, head_dim,
+                                                   int(paired), float(base),
+                                                   _stream(stream, cos_tab)))
+
+
+def pha_rope(q, k, cos_tab, sin_tab, positions, paired: bool = False, stagger_offset: int = 0,
+             stream=None, *, tab_rows=None, tab_width=None, total_tokens=None, n_heads=None,
+             n_kv_heads=None, head_dim=None, dtype=None):
+    """In-place RoPE of q [T][H][hd] and k [T][Hkv][hd]. Shapes are taken from the tensors unless
+    given explicitly (needed when raw addresses are passed)."""
+    if total_tokens is None:
+        total_tokens, n_heads, head_dim = q.shape
+        n_kv_heads = 0 if k is None else k.shape[1]
+        tab_rows, tab_width = cos_tab.shape
+        dtype = _dtype_code(q)
+    _check("pha_rope", _lib.pha_rope(_ptr(q), _ptr(k), _ptr(cos_tab), _ptr(sin_tab), tab_rows,
+                                     tab_width, _ptr(positions), total_tokens, n_heads, n_kv_heads,
+                                     head_dim, dtype, int(paired), stagger_offset,
+                                     _stream(stream, q)))
+
+
+def pha_attn_workspace_bytes(batch: int, max_len: int, n_heads: int, head_dim: int,
+                             paired: bool) -> int:
+    return int(_lib.pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, int(paired)))
+
+
+def pha_attn_fwd(q, k, v, cu_seqlens, max_len: int, o, lse, workspace, *, causal: bool = True,
+                 window: int = 0, paired: bool = False, scale: float = 0.0, stream=None,
+                 batch=None, total_tokens=None, n_heads=None, n_kv_heads=None, head_dim=None,
+                 dtype=None, workspace_bytes=None):
+    """Varlen attention forward into o (like q) and lse [T][H] float32 (or None)."""
+    if total_tokens is None:
+        total_tokens, n_heads, head_dim = q.shape
+        n_kv_heads = k.shape[1]
+        batch = cu_seqlens.shape[0] - 1
+        dtype = _dtype_code(q)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pha_attn_fwd", _lib.pha_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch,
+                                             max_len, total_tokens, n_heads, n_kv_heads, head_dim,
+                                             dtype, int(causal), int(window), int(paired),
+                                             float(scale), _ptr(o), _ptr(lse), _ptr(workspace),
+                                             workspace_bytes, _stream(stream, q)))
+
+
+def pha_attn_status(workspace, stream=None):
+    """(device status, scheduled work items) recorded in the workspace; synchronises."""
+    st, n = _i(0), _i(0)
+    _check("pha_attn_status", _lib.pha_attn_status(_ptr(workspace), ctypes.byref(st),
+                                                   ctypes.byref(n), _stream(stream, workspace)))
+    return st.value, n.value

@@ -1,0 +1,74 @@
+"""One forward step -- RoPE on q and k, then varlen attention -- over a fixed problem shape.
+
+``AttentionStep`` owns the device buffers the C ABI expects the caller to provide (rotary tables,
+workspace, O and LSE), allocated once through torch, and issues the two library calls. It is
+plumbing only: all arithmetic runs in libpha's kernels.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import pha
+
+
+@dataclasses.dataclass
+class StepShape:
+    n_heads: int
+    n_kv_heads: int
+    head_dim: int
+    dtype: str                 # "bf16" | "f32"
+    batch: int
+    max_len: int
+    total_tokens: int
+    tab_rows: int              # rows of the rotary tables (max position + 1)
+    paired: bool = False
+    stagger: bool = False
+    causal: bool = True
+    window: int = 0
+    scale: float = 0.0
+    rope_base: float = 10000.0
+
+    @classmethod
+    def of(cls, w, tab_rows: int) -> "StepShape":
+        """Shape of a synth.Workload."""
+        return cls(w.n_heads, w.n_kv_heads, w.head_dim, w.dtype, w.batch, w.max_len, w.total,
+                   tab_rows, w.paired, w.stagger, w.causal, w.window, w.scale, w.rope_base)
+
+
+class AttentionStep:
+    def __init__(self, shape: StepShape, device="cuda"):
+        self.s = shape
+        dev = torch.device(device)
+        width = (2 if shape.paired else 1) * shape.head_dim
+        self.cos_tab = torch.empty(max(shape.tab_rows, 1), width, device=dev)
+        self.sin_tab = torch.empty_like(self.cos_tab)
+        pha.pha_rope_tables(self.cos_tab, self.sin_tab, shape.tab_rows, shape.head_dim,
+                            shape.paired, shape.rope_base)
+        dt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+        self.o = torch.empty(shape.total_tokens, shape.n_heads, shape.head_dim, dtype=dt, device=dev)
+        self.lse = torch.empty(shape.total_tokens, shape.n_heads, dtype=torch.float32, device=dev)
+        nbytes = pha.pha_attn_workspace_bytes(shape.batch, shape.max_len, shape.n_heads,
+                                              shape.head_dim, shape.paired)
+        self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        self.stagger_offset = shape.head_dim if (shape.paired and shape.stagger) else 0
+
+    def rope(self, q, k, positions, stream=None):
+        pha.pha_rope(q, k, self.cos_tab, self.sin_tab, positions, paired=self.s.paired,
+                     stagger_offset=self.stagger_offset, stream=stream)
+
+    def attn(self, q, k, v, cu_seqlens, stream=None):
+        pha.pha_attn_fwd(q, k, v, cu_seqlens, self.s.max_len, self.o, self.lse, self.workspace,
+                         causal=self.s.causal, window=self.s.window, paired=self.s.paired,
+                         scale=self.s.scale, stream=stream)
+        return self.o, self.lse
+
+    def __call__(self, q, k, v, cu_seqlens, positions, stream=None):
+        """RoPE q and k in place, then attention. Returns (o, lse) (buffers owned by the step)."""
+        self.rope(q, k, positions, stream)
+        return self.attn(q, k, v, cu_seqlens, stream)
+
+    def status(self):
+        """(device status, scheduled work items) of the last attention call; synchronises."""
+        return pha.pha_attn_status(self.workspace)

@@ -1,0 +1,140 @@
+"""The C-ABI library loads, exports every entry point include/pha.h declares, and rejects bad
+arguments before touching the GPU (these calls never reach a CUDA call, so they run on CPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from paired_heads_b200 import build as pha_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pha():
+    pha_build.build()
+    from paired_heads_b200 import pha as mod
+
+    return mod
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "pha.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pha_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    assert _declared() == ["pha_attn_fwd", "pha_attn_status", "pha_attn_workspace_bytes",
+                           "pha_rope", "pha_rope_tables", "pha_status_string"]
+
+
+def test_library_exports_every_declared_symbol(pha):
+    lib = ctypes.CDLL(pha.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", pha.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(_declared()) <= exported
+
+
+def test_status_strings(pha):
+    assert pha.pha_status_string(0) == "ok"
+    assert pha.pha_status_string(-3).startswith("workspace")
+    assert pha.pha_status_string(7) == "unknown status"
+
+
+def test_workspace_bytes_closed_form(pha):
+    # 256-byte header + 16 bytes per (query tile of 128 slots, head) work item
+    assert pha.pha_attn_workspace_bytes(8, 1024, 12, 64, False) == 256 + 16 * 8 * 8 * 12
+    assert pha.pha_attn_workspace_bytes(113, 2048, 6, 128, True) == 256 + 16 * 113 * 32 * 3
+    assert pha.pha_attn_workspace_bytes(1, 1, 2, 64, True) == 256 + 16 * 1 * 1 * 1
+    assert pha.pha_attn_workspace_bytes(0, 10, 2, 64, False) == 0
+    assert pha.pha_attn_workspace_bytes(1, 10, 3, 64, True) == 0   # odd heads cannot pair
+
+
+A = 0x10000          # an aligned fake device address (never dereferenced: calls fail first)
+MIS = 0x10004        # misaligned
+
+
+def _attn(pha, **kw):
+    args = dict(q=A, k=A, v=A, cu=A, batch=1, max_len=128, total=128, H=4, Hkv=4, hd=64,
+                dtype=pha.PHA_BF16, causal=1, window=0, paired=0, scale=0.0, o=A, lse=A, ws=A,
+                ws_bytes=1 << 20)
+    args.update(kw)
+    lib = pha.library()
+    return lib.pha_attn_fwd(args["q"], args["k"], args["v"], args["cu"], args["batch"],
+                            args["max_len"], args["total"], args["H"], args["Hkv"], args["hd"],
+                            args["dtype"], args["causal"], args["window"], args["paired"],
+                            ctypes.c_float(args["scale"]), args["o"], args["lse"], args["ws"],
+                            args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=6, Hkv=4), -1),                    # heads not a multiple of kv heads
+    (dict(H=6, Hkv=6, paired=1), 0),           # (valid shape; see below)
+    (dict(H=6, Hkv=3, paired=1), -1),          # odd kv heads cannot pair
+    (dict(H=5, Hkv=5, paired=1), -1),          # odd heads cannot pair
+    (dict(causal=0, window=16), -2),           # windowed non-causal attention
+    (dict(hd=96), -2),                         # bf16 tensor-core path: head_dim 64 / 128 only
+    (dict(dtype=1, hd=160), -2),               # f32 path: head_dim <= 128
+    (dict(q=MIS), -1),
+    (dict(o=MIS), -1),
+    (dict(lse=A + 2), -1),
+    (dict(q=None), -1),
+    (dict(batch=0), -1),
+    (dict(total=-1), -1),
+    (dict(dtype=7), -1),
+    (dict(ws=None), -3),
+    (dict(ws_bytes=100), -3),
+    (dict(ws=MIS), -3),
+])
+def test_attn_argument_errors(pha, kw, code):
+    if code == 0:
+        # a valid problem would launch; only check that the workspace bound is what gates it
+        assert _attn(pha, ws_bytes=10, **kw) == -3
+        return
+    assert _attn(pha, **kw) == code
+
+
+def _rope(pha, **kw):
+    args = dict(q=A, k=A, cos=A, sin=A, rows=16, width=64, pos=A, total=4, H=2, Hkv=2, hd=64,
+                dtype=pha.PHA_BF16, paired=0, stagger=0)
+    args.update(kw)
+    return pha.library().pha_rope(args["q"], args["k"], args["cos"], args["sin"], args["rows"],
+                                  args["width"], args["pos"], args["total"], args["H"],
+                                  args["Hkv"], args["hd"], args["dtype"], args["paired"],
+                                  args["stagger"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(width=128),                           # standard table must be head_dim wide
+    dict(stagger=64),                          # stagger only on the paired path
+    dict(paired=1, width=64),                  # paired table must be 2*head_dim wide
+    dict(paired=1, width=128, stagger=32),     # stagger offset 0 or head_dim
+    dict(hd=40, width=40),                     # bf16 spans of 16 elements
+    dict(dtype=1, hd=12, width=12),            # f32 spans of 8 elements
+    dict(q=MIS),
+    dict(cos=MIS),
+    dict(k=None),
+    dict(H=0),
+    dict(total=-2),
+])
+def test_rope_argument_errors(pha, kw):
+    assert _rope(pha, **kw) == -1
+
+
+def test_rope_empty_is_a_no_op(pha):
+    assert _rope(pha, total=0) == 0
+    assert _rope(pha, total=0, paired=1, width=128, stagger=64) == 0
+
+
+def test_rope_tables_argument_errors(pha):
+    lib = pha.library()
+    assert lib.pha_rope_tables(MIS, A, 4, 64, 0, ctypes.c_double(1e4), None) == -1
+    assert lib.pha_rope_tables(A, A, 4, 63, 0, ctypes.c_double(1e4), None) == -1
+    assert lib.pha_rope_tables(A, A, 4, 64, 0, ctypes.c_double(0.0), None) == -1
+    assert lib.pha_rope_tables(A, A, -1, 64, 1, ctypes.c_double(1e4), None) == -1

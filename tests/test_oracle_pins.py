@@ -378,3 +378,27 @@ def test_oracle_rejects_bad_arguments():
         oracle.attn_fwd(q, q, q, np.array([0, 4], dtype=np.int32), paired=True)  # odd heads
     with pytest.raises(ValueError):
         oracle.attention_slots(q, q, q, np.array([0, 3, 2]))  # decreasing cu
+
+
+# ----------------------------------------------------------------------------- bf16 storage
+
+def test_round_bf16_ties_and_neighbours():
+    # bfloat16 keeps 8 significant bits: the neighbours of 1 are 1 - 2^-8 and 1 + 2^-7.
+    cases = [
+        (1.0, 1.0),
+        (1 + 2.0 ** -8, 1.0),                      # tie -> even (1.0)
+        (1 + 3 * 2.0 ** -8, 1 + 2.0 ** -6),        # tie -> even (mantissa ...10)
+        (1 + 2.0 ** -8 + 2.0 ** -30, 1 + 2.0 ** -7),
+        (-(1 + 2.0 ** -8 + 2.0 ** -30), -(1 + 2.0 ** -7)),
+        (3.4e38, np.inf),                          # past the midpoint above the largest bf16
+        (0.0, 0.0),
+    ]
+    got = oracle.round_bf16(np.array([c[0] for c in cases]))
+    assert got.tolist() == [c[1] for c in cases]
+
+
+def test_round_bf16_matches_torch_on_float32_values():
+    torch = pytest.importorskip("torch")
+    x = np.random.default_rng(21).standard_normal(100000).astype(np.float32) * 10.0
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x.astype(np.float64)), ref)
