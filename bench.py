@@ -173,8 +173,8 @@ def time_oracle(w, budget_tokens: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="paired_varlen", choices=synth.WORKLOADS)
     ap.add_argument("--window", type=int, default=None)
     ap.add_argument("--paired", type=int, default=None)

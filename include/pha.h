@@ -73,12 +73,14 @@ pha_status pha_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_di
  *   positions: int32[total_tokens], the table row of each token.
  *   For token t, head h, pair i (columns 2i, 2i+1) with c = cos_tab[positions[t]][col0 + 2i],
  *   s = sin_tab[...][col0 + 2i]:  y[2i] = x[2i] c - x[2i+1] s,  y[2i+1] = x[2i] s + x[2i+1] c,
- *   where col0 = 0, or col0 = stagger_offset for odd h when paired = 1. Arithmetic is float32;
- *   bf16 results are rounded to nearest even.
+ *   where col0 = 0, or col0 = stagger_offset for odd h when paired = 1.
  *   paired = 0: tab_width must equal head_dim and stagger_offset must be 0.
  *   paired = 1: tab_width must equal 2*head_dim; stagger_offset is head_dim (the page's
  *               staggered rotary: odd heads take phase 2p+1) or 0 (both heads take 2p).
  *   A token whose position lies outside [0, tab_rows) is left unchanged; this is not reported.
+ *   The rotation is computed in float64 (exact products) and rounded once to the dtype, so the
+ *   result is the correctly rounded rotation with the tables' float32 values.
+ *   total_tokens = 0 is a no-op and then q, k, the tables and positions may be NULL.
  *   Errors: PHA_ERR_INVALID for NULL/misaligned pointers, negative sizes, n_heads <= 0,
  *   head_dim not a positive multiple of 16 (bf16) or 8 (f32), or table width / stagger_offset
  *   not as above.
@@ -116,6 +118,8 @@ size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_di
  *      its contents need not be initialised. The scheduler kernel writes the work list into it
  *      and records in its first 8 bytes the number of work items and a device-side status
  *      (see pha_attn_status). May be NULL for PHA_F32, which does not use it.
+ *   total_tokens = 0: q, k, v, o, lse may be NULL; the scheduler still records 0 work items.
+ *   Slots that lie outside every document (cu_seqlens[batch] < total_tokens) are not written.
  *   Supported: bf16 with head_dim in {64, 128} (tcgen05 tensor-core kernel); f32 with
  *      1 <= head_dim <= 128 (exact float32 CUDA-core kernel).
  *   Errors (before launch): PHA_ERR_INVALID for NULL/misaligned pointers, non-positive sizes,

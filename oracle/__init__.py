@@ -49,7 +49,7 @@ def _load():
     global _lib
     if _lib is None:
         lib = ctypes.CDLL(build())
-        lib.oracle_rope.argtypes = [_f64p, _i32p, _l, _c, _c, _c, _c, _d]
+        lib.oracle_rope.argtypes = [_f64p, _i32p, _l, _c, _c, _c, _c, _d, _c]
         lib.oracle_round_bf16.argtypes = [_f64p, _l]
         lib.oracle_interleave.argtypes = [_f64p, _f64p, _l, _c, _c]
         lib.oracle_deinterleave.argtypes = [_f64p, _f64p, _l, _c, _c]
@@ -75,14 +75,17 @@ def _check(rc: int, what: str) -> None:
         raise ValueError(f"{what}: oracle rejected the arguments (rc={rc})")
 
 
-def rope(x, positions, paired: bool = False, stagger: bool = False, base: float = 10000.0):
+def rope(x, positions, paired: bool = False, stagger: bool = False, base: float = 10000.0,
+         table_f32: bool = False):
     """Rotate x[T][H][hd] (returns a new float64 array). Phase of token t, head h is
-    positions[t] (standard) or 2*positions[t] + (h % 2 if stagger) (paired)."""
+    positions[t] (standard) or 2*positions[t] + (h % 2 if stagger) (paired). table_f32 rounds
+    the cosines and sines to float32 first (the values a float32 rotary table holds)."""
     y = _f64(x).copy()
     T, H, hd = y.shape
     pos = np.ascontiguousarray(positions, dtype=np.int32)
     assert pos.shape == (T,)
-    _check(_load().oracle_rope(y, pos, T, H, hd, int(paired), int(stagger), float(base)), "rope")
+    _check(_load().oracle_rope(y, pos, T, H, hd, int(paired), int(stagger), float(base),
+                               int(table_f32)), "rope")
     return y
 
 
@@ -95,9 +98,10 @@ def round_bf16(x):
 
 def rope_stored(x, positions, dtype: str, paired: bool = False, stagger: bool = False,
                 base: float = 10000.0):
-    """RoPE as the pipeline stores it: rotated in float64, then rounded to the buffer's dtype
-    ("bf16": nearest bfloat16; "f32": nearest float32)."""
-    y = rope(x, positions, paired, stagger, base)
+    """RoPE as the pipeline stores it: cosines and sines taken from float32 tables, rotation in
+    float64, result rounded to the buffer's dtype ("bf16": nearest bfloat16; "f32": nearest
+    float32)."""
+    y = rope(x, positions, paired, stagger, base, table_f32=True)
     if dtype == "bf16":
         return round_bf16(y)
     return y.astype(np.float32).astype(np.float64)

@@ -57,9 +57,12 @@ static double rope_phase(int32_t pos, int h, int paired, int stagger)
     return 2.0 * (double)pos + ((stagger && (h % 2)) ? 1.0 : 0.0);
 }
 
-/* In-place RoPE on x[n_tok][n_head][hd] (float64). */
+/* In-place RoPE on x[n_tok][n_head][hd] (float64). table_f32 != 0 rounds each cosine and sine to
+ * float32 before use, as the pipeline does when it keeps them in float32 tables ([PHA] "2. building
+ * the paired rotary table": factor1 / factor2 are precomputed, stored tables); the rotation itself
+ * stays float64. */
 int oracle_rope(double* x, const int32_t* pos, int64_t n_tok, int n_head, int hd,
-                int paired, int stagger, double base)
+                int paired, int stagger, double base, int table_f32)
 {
     if (!x || !pos || n_tok < 0 || n_head <= 0 || hd <= 0 || (hd % 2) != 0) return ORACLE_EINVAL;
 #pragma omp parallel for schedule(static)
@@ -70,6 +73,10 @@ int oracle_rope(double* x, const int32_t* pos, int64_t n_tok, int n_head, int hd
             for (int i = 0; i < hd / 2; ++i) {
                 double theta = phase * rope_freq(i, hd, base);
                 double c = cos(theta), s = sin(theta);
+                if (table_f32) {
+                    c = (double)(float)c;
+                    s = (double)(float)s;
+                }
                 double a = row[2 * i], b = row[2 * i + 1];
                 row[2 * i] = a * c - b * s;
                 row[2 * i + 1] = a * s + b * c;

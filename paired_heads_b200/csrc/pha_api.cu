@@ -82,10 +82,13 @@ pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab
                     pha_stream_t stream) {
     if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
     const int span = dtype == PHA_BF16 ? 16 : 8;
-    if (!q || !aligned16(q) || (n_kv_heads > 0 && (!k || !aligned16(k))) || !cos_tab || !sin_tab ||
-        !aligned16(cos_tab) || !aligned16(sin_tab) || !positions || tab_rows < 0 ||
-        total_tokens < 0 || n_heads <= 0 || n_kv_heads < 0 || head_dim <= 0 ||
+    if (tab_rows < 0 || total_tokens < 0 || n_heads <= 0 || n_kv_heads < 0 || head_dim <= 0 ||
         head_dim % span != 0 || (paired != 0 && paired != 1))
+        return PHA_ERR_INVALID;
+    // With no tokens there is nothing to read or write; the buffers may be empty (NULL).
+    if (total_tokens > 0 &&
+        (!q || !aligned16(q) || (n_kv_heads > 0 && (!k || !aligned16(k))) || !cos_tab ||
+         !sin_tab || !aligned16(cos_tab) || !aligned16(sin_tab) || !positions))
         return PHA_ERR_INVALID;
     if (!paired && (tab_width != head_dim || stagger_offset != 0)) return PHA_ERR_INVALID;
     if (paired && (tab_width != 2 * head_dim ||
@@ -112,8 +115,11 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
                         float scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
                         pha_stream_t stream) {
     if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
-    if (!q || !k || !v || !o || !cu_seqlens || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
-        !aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || batch <= 0 ||
+    // With no tokens the q / k / v / o / lse buffers may be empty (NULL); cu_seqlens is still read.
+    const bool have = total_tokens > 0;
+    if ((have && (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+                  !aligned16(o))) ||
+        !cu_seqlens || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || batch <= 0 ||
         max_len < 0 || total_tokens < 0 || total_tokens > (1 << 29) || n_heads <= 0 ||
         n_kv_heads <= 0 || n_heads > 4096 || n_heads % n_kv_heads != 0 || head_dim <= 0 ||
         (causal != 0 && causal != 1) || (paired != 0 && paired != 1) || !(scale == scale))

@@ -9,7 +9,10 @@
 //
 // The rotation is HBM-bound: each thread moves one 32-byte span of one (token, head) row with
 // two 16-byte loads and stores; the table row of a token is shared by all of its heads and is
-// served from L1/L2.
+// served from L1/L2. The arithmetic is float64: a bf16 or f32 element times a float32 table value
+// is exact in double, so y = c*x0 - s*x1 is rounded exactly once there and once more to the
+// output dtype (round to nearest even) -- the correctly rounded value of the rotation with the
+// tables' float32 cosines and sines.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -37,13 +40,32 @@ __global__ void rope_tables_kernel(float* __restrict__ cos_tab, float* __restric
     }
 }
 
+// Nearest bfloat16 (ties to even) of a double, as its 16-bit pattern; one rounding step.
+__device__ __forceinline__ uint32_t bf16_bits_rne(double y) {
+    const uint64_t b = static_cast<uint64_t>(__double_as_longlong(y));
+    const uint32_t sign = static_cast<uint32_t>(b >> 48) & 0x8000u;
+    const int e = static_cast<int>((b >> 52) & 0x7FF);
+    const uint64_t man = b & 0xFFFFFFFFFFFFFull;
+    if (e == 0x7FF) return sign | 0x7F80u | (man ? 0x40u : 0u);  // inf, nan
+    const int eb = e - 1023 + 127;                                // bf16 biased exponent
+    if (eb >= 255) return sign | 0x7F80u;                        // overflow
+    if (eb <= 0)  // bf16 subnormal range: count units of 2^-133 (rint rounds half to even;
+                  // 128 units carry into the smallest normal's bit pattern)
+        return sign | static_cast<uint32_t>(rint(fabs(y) * 0x1p133));
+    const uint32_t keep = static_cast<uint32_t>(man >> 45);      // 7 mantissa bits kept
+    const uint64_t rem = man & ((1ull << 45) - 1), half = 1ull << 44;
+    uint32_t bits = (static_cast<uint32_t>(eb) << 7) | keep;
+    if (rem > half || (rem == half && (keep & 1u))) ++bits;      // may carry into the exponent
+    return sign | bits;
+}
+
 template <typename T>
 struct Span32;  // 32 bytes of one row: 16 bf16 or 8 f32
 
 template <>
 struct Span32<__nv_bfloat16> {
     static constexpr int N = 16;
-    __device__ static void load(const __nv_bfloat16* p, float (&x)[N]) {
+    __device__ static void load(const __nv_bfloat16* p, double (&x)[N]) {
         const uint4 a = *reinterpret_cast<const uint4*>(p);
         const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -53,10 +75,10 @@ struct Span32<__nv_bfloat16> {
             x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
         }
     }
-    __device__ static void store(__nv_bfloat16* p, const float (&y)[N]) {
+    __device__ static void store(__nv_bfloat16* p, const double (&y)[N]) {
         uint32_t w[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+        for (int e = 0; e < 8; ++e) w[e] = bf16_bits_rne(y[2 * e]) | (bf16_bits_rne(y[2 * e + 1]) << 16);
         *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(p + 8) = make_uint4(w[4], w[5], w[6], w[7]);
     }
@@ -65,15 +87,18 @@ struct Span32<__nv_bfloat16> {
 template <>
 struct Span32<float> {
     static constexpr int N = 8;
-    __device__ static void load(const float* p, float (&x)[N]) {
+    __device__ static void load(const float* p, double (&x)[N]) {
         const float4 a = *reinterpret_cast<const float4*>(p);
         const float4 b = *reinterpret_cast<const float4*>(p + 4);
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
         x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
     }
-    __device__ static void store(float* p, const float (&y)[N]) {
-        *reinterpret_cast<float4*>(p) = make_float4(y[0], y[1], y[2], y[3]);
-        *reinterpret_cast<float4*>(p + 4) = make_float4(y[4], y[5], y[6], y[7]);
+    __device__ static void store(float* p, const double (&y)[N]) {
+        float f[N];
+#pragma unroll
+        for (int e = 0; e < N; ++e) f[e] = __double2float_rn(y[e]);
+        *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
     }
 };
 
@@ -107,7 +132,8 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
     const float* srow = sin_tab + static_cast<int64_t>(pos) * tab_width + col;
     T* p = base + local * N;
 
-    float x[N], y[N], c[N], s[N];
+    double x[N], y[N];
+    float c[N], s[N];
     Span32<T>::load(p, x);
 #pragma unroll
     for (int e = 0; e < N; e += 4) {
@@ -117,11 +143,12 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
         s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
     }
     // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign is -1 on
-    // the even member and +1 on the odd member, which is a rotation by +angle.
+    // the even member and +1 on the odd member, which is a rotation by +angle. Both products are
+    // exact in double, so the fma rounds once.
 #pragma unroll
     for (int e = 0; e < N; e += 2) {
-        y[e] = fmaf(c[e], x[e], -s[e] * x[e + 1]);
-        y[e + 1] = fmaf(c[e + 1], x[e + 1], s[e + 1] * x[e]);
+        y[e] = fma(static_cast<double>(c[e]), x[e], -(static_cast<double>(s[e]) * x[e + 1]));
+        y[e + 1] = fma(static_cast<double>(c[e + 1]), x[e + 1], static_cast<double>(s[e + 1]) * x[e]);
     }
     Span32<T>::store(p, y);
 }

@@ -84,12 +84,14 @@ def test_rope_parity(case):
         ref = oracle.rope_stored(x, pos_ok, dt, paired, stagger)
         ref[3], ref[7] = x[3], x[7]
         g = got.to(torch.float64).cpu().numpy()
-        if dt == "bf16":
-            diff = np.abs(g - ref)
-            assert np.all(diff <= _ulp_bf16(ref) * 1.0001), float((diff / _ulp_bf16(ref)).max())
-            assert np.mean(diff == 0) > 0.99
-        else:
-            np.testing.assert_allclose(g, ref, rtol=2e-6, atol=2e-6)
+        # Both sides round the float64 rotation of the float32 table values once to the dtype,
+        # so they agree bit for bit except where the two float32 tables differ in a last bit
+        # (CUDA's and the C library's float64 sin / cos / pow), which may move a result by one
+        # unit in the last place.
+        diff = np.abs(g - ref)
+        ulp = _ulp_bf16(ref) if dt == "bf16" else np.spacing(np.abs(ref).astype(np.float32))
+        assert np.all(diff <= ulp * 1.0001), float((diff / ulp).max())
+        assert np.mean(diff == 0) > 0.9999, float(np.mean(diff == 0))
 
 
 # ------------------------------------------------------------------------------------ fp32 path

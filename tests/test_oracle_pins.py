@@ -402,3 +402,17 @@ def test_round_bf16_matches_torch_on_float32_values():
     x = np.random.default_rng(21).standard_normal(100000).astype(np.float32) * 10.0
     ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(oracle.round_bf16(x.astype(np.float64)), ref)
+
+
+def test_float32_tables_only_perturb_by_float32_rounding():
+    # Rounding cos / sin to float32 changes each rotated element by at most
+    # 2^-24 (|x_2i| + |x_2i+1|) (one float32 half-ulp on each factor of magnitude <= 1).
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((200, 4, 64))
+    pos = rng.integers(0, 70000, 200).astype(np.int32)
+    for paired in (False, True):
+        a = oracle.rope(x, pos, paired, paired)
+        b = oracle.rope(x, pos, paired, paired, table_f32=True)
+        pair = np.abs(x.reshape(200, 4, 32, 2)).sum(-1).repeat(2, axis=-1)
+        assert np.all(np.abs(a - b) <= 2.0 ** -24 * pair * 1.0001)
+        assert np.any(a != b)
