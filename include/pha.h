@@ -91,9 +91,10 @@ pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab
                     int stagger_offset, pha_stream_t stream);
 
 /*
- * pha_attn_workspace_bytes -- device workspace that pha_attn_fwd needs: the varlen tile work
- * list for at most batch * ceil(L/128) * H' tiles (L = max_len, doubled when paired; H' =
- * n_heads, halved when paired) plus a 256-byte header. Returns 0 for invalid arguments.
+ * pha_attn_workspace_bytes -- device workspace that pha_attn_fwd needs: a 256-byte header,
+ * int32[batch + 1] of per-document scratch (padded to 16 bytes) and the varlen work list, 16
+ * bytes for each of at most batch * ceil(L/256) * H' (query block, head) items (L = max_len,
+ * doubled when paired; H' = n_heads, halved when paired). Returns 0 for invalid arguments.
  */
 size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired);
 

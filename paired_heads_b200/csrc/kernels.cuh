@@ -9,17 +9,24 @@
 
 namespace pha {
 
-constexpr int kBlockM = 128;  // query slots per tile
-constexpr int kBlockN = 128;  // key slots per tile
+constexpr int kBlockM = 128;         // query rows per sub-tile (one softmax warpgroup)
+constexpr int kBlockN = 128;         // key slots per tile
+constexpr int kItemRows = 2 * kBlockM;  // query slots per work item
+constexpr int kMaxCostBuckets = 4096;   // scheduler cost classes (longest-first ordering)
 
-// Workspace header (bytes [0, 256)) followed by int4 work items.
+// Workspace: header (bytes [0, 256)), per-document block offsets (int32[batch + 1], padded to 16
+// bytes), then int4 work items.
 struct WorkspaceHeader {
     int n_items;
     int status;
 };
 constexpr size_t kWorkspaceHeaderBytes = 256;
 
-// One work item = one query tile of one head:
+inline size_t workspace_doc_bytes(int batch) {
+    return (static_cast<size_t>(batch + 1) * sizeof(int) + 15) & ~static_cast<size_t>(15);
+}
+
+// One work item = one block of up to kItemRows query slots of one head:
 //   x = first query slot, y = (head << 16) | valid query rows, z = first key slot, w = key end.
 // Keys [z, w) are streamed in tiles of kBlockN starting at z.
 
@@ -52,9 +59,10 @@ cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin
 
 cudaError_t launch_attn_f32(const AttnProblem& p, cudaStream_t stream);
 
-// Builds the varlen work list into `items` (capacity entries) and the header.
-cudaError_t launch_schedule(const AttnProblem& p, int capacity, int4* items, WorkspaceHeader* hdr,
-                            cudaStream_t stream);
+// Builds the varlen work list into `items` (capacity entries) and the header; doc_blocks is
+// int32[batch + 1] scratch.
+cudaError_t launch_schedule(const AttnProblem& p, int capacity, int* doc_blocks, int4* items,
+                            WorkspaceHeader* hdr, cudaStream_t stream);
 
 // tcgen05 attention over a scheduled work list. tm_q / tm_k / tm_v are 2-D bf16 tensor maps
 // over the slot view ([slots][heads * head_dim] and [slots][kv_heads * head_dim]) with a

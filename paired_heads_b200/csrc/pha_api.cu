@@ -48,7 +48,7 @@ int64_t div_up(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t max_work_items(int batch, int max_len, int n_heads, int paired) {
     const int64_t slots = static_cast<int64_t>(max_len) * (paired ? 2 : 1);
     const int64_t heads = paired ? n_heads / 2 : n_heads;
-    return static_cast<int64_t>(batch) * div_up(slots, kBlockM) * heads;
+    return static_cast<int64_t>(batch) * div_up(slots, kItemRows) * heads;
 }
 
 }  // namespace
@@ -105,7 +105,7 @@ pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab
 size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired) {
     (void)head_dim;
     if (batch <= 0 || max_len < 0 || n_heads <= 0 || (paired && (n_heads & 1))) return 0;
-    return kWorkspaceHeaderBytes +
+    return kWorkspaceHeaderBytes + workspace_doc_bytes(batch) +
            static_cast<size_t>(max_work_items(batch, max_len, n_heads, paired)) * sizeof(int4);
 }
 
@@ -154,12 +154,16 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
 
     const size_t need = pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired);
     if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PHA_ERR_WORKSPACE;
-    const int64_t cap64 = static_cast<int64_t>((workspace_bytes - kWorkspaceHeaderBytes) / sizeof(int4));
+    const size_t fixed = kWorkspaceHeaderBytes + workspace_doc_bytes(batch);
+    const int64_t cap64 = static_cast<int64_t>((workspace_bytes - fixed) / sizeof(int4));
     const int capacity = cap64 > 0x7FFFFFFF ? 0x7FFFFFFF : static_cast<int>(cap64);
-    auto* hdr = static_cast<WorkspaceHeader*>(workspace);
-    auto* items = reinterpret_cast<int4*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
+    auto* base = static_cast<uint8_t*>(workspace);
+    auto* hdr = reinterpret_cast<WorkspaceHeader*>(base);
+    auto* doc_blocks = reinterpret_cast<int*>(base + kWorkspaceHeaderBytes);
+    auto* items = reinterpret_cast<int4*>(base + fixed);
 
-    if (launch_schedule(p, capacity, items, hdr, stream) != cudaSuccess) return PHA_ERR_CUDA;
+    if (launch_schedule(p, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+        return PHA_ERR_CUDA;
     if (total_tokens == 0) return PHA_OK;
 
     const uint64_t rows = static_cast<uint64_t>(total_tokens) * p.slot_mult;

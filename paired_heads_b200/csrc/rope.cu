@@ -9,10 +9,13 @@
 //
 // The rotation is HBM-bound: each thread moves one 32-byte span of one (token, head) row with
 // two 16-byte loads and stores; the table row of a token is shared by all of its heads and is
-// served from L1/L2. The arithmetic is float64: a bf16 or f32 element times a float32 table value
-// is exact in double, so y = c*x0 - s*x1 is rounded exactly once there and once more to the
-// output dtype (round to nearest even) -- the correctly rounded value of the rotation with the
-// tables' float32 cosines and sines.
+// served from L1/L2. Every output is the correctly rounded (nearest even) value of the rotation
+// with the tables' float32 cosines and sines:
+//   bf16: y = fma(c, a, s*b) in float32 differs from the exact value by at most
+//         ulp(y)/2 + ulp(s*b)/2; when y lies farther than that from the nearest bf16 rounding
+//         midpoint, rounding y gives the same bf16 as rounding the exact value. The rare rest is
+//         recomputed in float64, where bf16 x float32 products are exact, and rounded from there.
+//   f32:  always float64 (exact products, one rounding), then rounded to float32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -41,7 +44,7 @@ __global__ void rope_tables_kernel(float* __restrict__ cos_tab, float* __restric
 }
 
 // Nearest bfloat16 (ties to even) of a double, as its 16-bit pattern; one rounding step.
-__device__ __forceinline__ uint32_t bf16_bits_rne(double y) {
+__device__ __noinline__ uint32_t bf16_bits_rne(double y) {
     const uint64_t b = static_cast<uint64_t>(__double_as_longlong(y));
     const uint32_t sign = static_cast<uint32_t>(b >> 48) & 0x8000u;
     const int e = static_cast<int>((b >> 52) & 0x7FF);
@@ -59,46 +62,65 @@ __device__ __forceinline__ uint32_t bf16_bits_rne(double y) {
     return sign | bits;
 }
 
+// One rotated element y = c*a + sb*b (sb = -s for the even member of a pair, +s for the odd one),
+// as the 16-bit pattern of the nearest bf16 of the exact value.
+__device__ __forceinline__ uint32_t rot_bf16(float a, float c, float b, float sb) {
+    const float t = sb * b;
+    const float y = fmaf(c, a, t);  // c*a enters the fma unrounded
+    const uint32_t bits = __float_as_uint(y);
+    // float32 ulps of y to the bf16 rounding midpoint of its binade (pattern ...8000)
+    const int dist = abs(static_cast<int>(bits & 0xFFFFu) - 0x8000);
+    // |y - exact| <= ulp(y)/2 + |t| 2^-24 < (1/2 + |t|/|y|) ulp(y); keep 1.5 ulp of margin
+    if (fabsf(t) <= fabsf(y) * static_cast<float>(dist - 2)) {
+        uint32_t r;
+        asm("{\n\t.reg .b16 h;\n\tcvt.rn.bf16.f32 h, %1;\n\tmov.b32 %0, {h, h};\n\t}" : "=r"(r) : "f"(y));
+        return r & 0xFFFFu;
+    }
+    return bf16_bits_rne(fma(static_cast<double>(c), static_cast<double>(a),
+                             static_cast<double>(sb) * static_cast<double>(b)));
+}
+
 template <typename T>
 struct Span32;  // 32 bytes of one row: 16 bf16 or 8 f32
 
 template <>
 struct Span32<__nv_bfloat16> {
     static constexpr int N = 16;
-    __device__ static void load(const __nv_bfloat16* p, double (&x)[N]) {
+    __device__ static void rotate(__nv_bfloat16* p, const float (&c)[N], const float (&s)[N]) {
         const uint4 a = *reinterpret_cast<const uint4*>(p);
         const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t o[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            x[2 * e] = __uint_as_float(w[e] << 16);
-            x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+            const float x0 = __uint_as_float(w[e] << 16);
+            const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+            o[e] = rot_bf16(x0, c[2 * e], x1, -s[2 * e]) |
+                   (rot_bf16(x1, c[2 * e + 1], x0, s[2 * e + 1]) << 16);
         }
-    }
-    __device__ static void store(__nv_bfloat16* p, const double (&y)[N]) {
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = bf16_bits_rne(y[2 * e]) | (bf16_bits_rne(y[2 * e + 1]) << 16);
-        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(p + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+        *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(p + 8) = make_uint4(o[4], o[5], o[6], o[7]);
     }
 };
 
 template <>
 struct Span32<float> {
     static constexpr int N = 8;
-    __device__ static void load(const float* p, double (&x)[N]) {
+    __device__ static void rotate(float* p, const float (&c)[N], const float (&s)[N]) {
         const float4 a = *reinterpret_cast<const float4*>(p);
         const float4 b = *reinterpret_cast<const float4*>(p + 4);
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-    }
-    __device__ static void store(float* p, const double (&y)[N]) {
-        float f[N];
+        const float x[N] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float y[N];
 #pragma unroll
-        for (int e = 0; e < N; ++e) f[e] = __double2float_rn(y[e]);
-        *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
-        *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+        for (int e = 0; e < N; e += 2) {
+            // products of float32 values are exact in double: one rounding in the fma, one to f32
+            y[e] = __double2float_rn(fma(static_cast<double>(c[e]), static_cast<double>(x[e]),
+                                         -static_cast<double>(s[e]) * static_cast<double>(x[e + 1])));
+            y[e + 1] = __double2float_rn(fma(static_cast<double>(c[e + 1]), static_cast<double>(x[e + 1]),
+                                             static_cast<double>(s[e + 1]) * static_cast<double>(x[e])));
+        }
+        *reinterpret_cast<float4*>(p) = make_float4(y[0], y[1], y[2], y[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(y[4], y[5], y[6], y[7]);
     }
 };
 
@@ -132,9 +154,7 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
     const float* srow = sin_tab + static_cast<int64_t>(pos) * tab_width + col;
     T* p = base + local * N;
 
-    double x[N], y[N];
     float c[N], s[N];
-    Span32<T>::load(p, x);
 #pragma unroll
     for (int e = 0; e < N; e += 4) {
         const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + e));
@@ -143,14 +163,8 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
         s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
     }
     // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign is -1 on
-    // the even member and +1 on the odd member, which is a rotation by +angle. Both products are
-    // exact in double, so the fma rounds once.
-#pragma unroll
-    for (int e = 0; e < N; e += 2) {
-        y[e] = fma(static_cast<double>(c[e]), x[e], -(static_cast<double>(s[e]) * x[e + 1]));
-        y[e + 1] = fma(static_cast<double>(c[e + 1]), x[e + 1], static_cast<double>(s[e + 1]) * x[e]);
-    }
-    Span32<T>::store(p, y);
+    // the even member and +1 on the odd member, which is a rotation by +angle.
+    Span32<T>::rotate(p, c, s);
 }
 
 cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,

@@ -1,17 +1,22 @@
-// schedule.cu -- varlen tile scheduler: cu_seqlens -> list of (query tile, head) work items.
+// schedule.cu -- varlen tile scheduler: cu_seqlens -> list of (query block, head) work items.
 //
 // Paired path: document boundaries and max_len are doubled ("modded-nanogpt Paired Head
 // Attention record" page, section "sequence length and window handling") while the window stays
-// as given. For each query tile of 128 slots [q0, q0+n) of a document [a, b) the key range is
+// as given. A work item is a block of up to kItemRows = 256 query slots [q0, q0+n) of one
+// document [a, b) and one head; its key range is
 //   causal:      [max(a, q0 - window + 1), q0 + n)   (window <= 0: from a)
 //   non-causal:  [a, b)
-// so key tiles that the causal mask or the window hide entirely are never scheduled. Key tiles
-// start at the range's first slot (not at a multiple of 128): with a window of w the range of a
-// full query tile is 127 + w slots wide, i.e. ceil((127 + w) / 128) key tiles.
+// so key tiles that the causal mask or the window hide from the whole block are never scheduled
+// (the attention kernel further skips, per 128-row half of the block, the tiles that half cannot
+// see). Key tiles start at the range's first slot, not at a multiple of 128.
 //
 // Items are ordered longest first (counting sort on the number of key tiles) so that a static
-// round-robin over persistent CTAs balances; the heads of one query tile are adjacent so that
-// CTAs sharing a kv head (GQA) run close together in time and share K/V through L2.
+// round-robin over persistent CTAs balances; the heads of one block are adjacent so that CTAs
+// sharing a kv head (GQA) run close together in time and share K/V through L2.
+//
+// One CTA of 1024 threads: (1) per-document validation and block counts, (2) an exclusive scan
+// over documents, (3) a cost histogram over all blocks, (4) a scan of the histogram in descending
+// cost order, (5) emission, one thread per block.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,47 +25,83 @@
 namespace pha {
 
 constexpr int kSchedThreads = 1024;
-constexpr int kSchedBuckets = 4096;  // cost classes; costs above the last share one class
 
-__device__ __forceinline__ void tile_range(const AttnProblem& p, int64_t a, int64_t b, int64_t q0,
-                                           int64_t& n_q, int64_t& kv_lo, int64_t& kv_hi) {
-    n_q = b - q0 < kBlockM ? b - q0 : kBlockM;
-    if (p.causal) {
-        kv_hi = q0 + n_q;
-        kv_lo = a;
-        if (p.window > 0 && q0 - p.window + 1 > a) kv_lo = q0 - p.window + 1;
-    } else {
-        kv_lo = a;
-        kv_hi = b;
+// Exclusive scan of one value per thread across the CTA; returns the thread's prefix and writes
+// the total to *total. Needs kSchedThreads / 32 ints of shared scratch.
+__device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
     }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < kSchedThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        warp_sums[lane] = s;  // inclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int before = warp > 0 ? warp_sums[warp - 1] : 0;
+    const int t = warp_sums[kSchedThreads / 32 - 1];
+    __syncthreads();  // warp_sums may be reused by the caller's next scan
+    *total = t;
+    return before + x - v;
+}
+
+struct BlockRange {
+    int q0, n_q, kv_lo, kv_hi, cost;
+};
+
+__device__ __forceinline__ BlockRange block_range(const AttnProblem& p, int64_t a, int64_t b,
+                                                  int blk, int n_buckets) {
+    BlockRange r;
+    const int64_t q0 = a + static_cast<int64_t>(blk) * kItemRows;
+    const int64_t n_q = b - q0 < kItemRows ? b - q0 : kItemRows;
+    int64_t lo = a, hi = b;
+    if (p.causal) {
+        hi = q0 + n_q;
+        if (p.window > 0 && q0 - p.window + 1 > a) lo = q0 - p.window + 1;
+    }
+    int64_t cost = (hi - lo + kBlockN - 1) / kBlockN;
+    if (cost >= n_buckets) cost = n_buckets - 1;
+    r.q0 = static_cast<int>(q0);
+    r.n_q = static_cast<int>(n_q);
+    r.kv_lo = static_cast<int>(lo);
+    r.kv_hi = static_cast<int>(hi);
+    r.cost = static_cast<int>(cost);
+    return r;
 }
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, int capacity,
+                                                                 int n_buckets,
+                                                                 int* __restrict__ doc_blocks,
                                                                  int4* __restrict__ items,
                                                                  WorkspaceHeader* hdr) {
-    __shared__ int hist[kSchedBuckets];
+    __shared__ int hist[kMaxCostBuckets];
+    __shared__ int warp_sums[kSchedThreads / 32];
     __shared__ int bad;
     const int tid = threadIdx.x;
-    for (int c = tid; c < kSchedBuckets; c += kSchedThreads) hist[c] = 0;
+    const int64_t mult = p.slot_mult;
+    for (int c = tid; c < n_buckets; c += kSchedThreads) hist[c] = 0;
     if (tid == 0) bad = 0;
     __syncthreads();
 
-    const int64_t mult = p.slot_mult;
-    // validation + histogram of per-tile costs
+    // (1) validation and blocks per document
     for (int d = tid; d < p.batch; d += kSchedThreads) {
         const int64_t a0 = p.cu_seqlens[d], b0 = p.cu_seqlens[d + 1];
-        if (a0 < 0 || b0 < a0 || b0 > p.total_tokens || b0 - a0 > p.max_len) {
+        int nb = 0;
+        if (a0 < 0 || b0 < a0 || b0 > p.total_tokens || b0 - a0 > p.max_len)
             atomicOr(&bad, 1);
-            continue;
-        }
-        const int64_t a = a0 * mult, b = b0 * mult;
-        for (int64_t q0 = a; q0 < b; q0 += kBlockM) {
-            int64_t n_q, lo, hi;
-            tile_range(p, a, b, q0, n_q, lo, hi);
-            int64_t cost = (hi - lo + kBlockN - 1) / kBlockN;
-            if (cost >= kSchedBuckets) cost = kSchedBuckets - 1;
-            atomicAdd(&hist[cost], 1);
-        }
+        else
+            nb = static_cast<int>(((b0 - a0) * mult + kItemRows - 1) / kItemRows);
+        doc_blocks[d] = nb;
     }
     __syncthreads();
     if (bad) {
@@ -70,19 +111,21 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
         }
         return;
     }
-    // exclusive scan in descending cost order (one thread; 4096 entries)
-    __shared__ int total_tiles;
-    if (tid == 0) {
-        int acc = 0;
-        for (int c = kSchedBuckets - 1; c >= 0; --c) {
-            const int n = hist[c];
-            hist[c] = acc;
-            acc += n;
-        }
-        total_tiles = acc;
+    // (2) exclusive scan over documents (in place, chunks of kSchedThreads)
+    int carry = 0;
+    for (int base = 0; base < p.batch; base += kSchedThreads) {
+        const int d = base + tid;
+        const int v = d < p.batch ? doc_blocks[d] : 0;
+        int total;
+        const int ex = block_exclusive_scan(v, warp_sums, &total);
+        if (d < p.batch) doc_blocks[d] = carry + ex;
+        carry += total;
+        __syncthreads();
     }
+    const int n_blocks = carry;
+    if (tid == 0) doc_blocks[p.batch] = n_blocks;
     __syncthreads();
-    const int64_t n_items = static_cast<int64_t>(total_tiles) * p.heads;
+    const int64_t n_items = static_cast<int64_t>(n_blocks) * p.heads;
     if (n_items > capacity) {
         if (tid == 0) {
             hdr->n_items = 0;
@@ -90,20 +133,43 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
         }
         return;
     }
-    for (int d = tid; d < p.batch; d += kSchedThreads) {
-        const int64_t a = static_cast<int64_t>(p.cu_seqlens[d]) * mult;
-        const int64_t b = static_cast<int64_t>(p.cu_seqlens[d + 1]) * mult;
-        for (int64_t q0 = a; q0 < b; q0 += kBlockM) {
-            int64_t n_q, lo, hi;
-            tile_range(p, a, b, q0, n_q, lo, hi);
-            int64_t cost = (hi - lo + kBlockN - 1) / kBlockN;
-            if (cost >= kSchedBuckets) cost = kSchedBuckets - 1;
-            const int slot = atomicAdd(&hist[cost], 1);
-            for (int h = 0; h < p.heads; ++h)
-                items[static_cast<int64_t>(slot) * p.heads + h] =
-                    make_int4(static_cast<int>(q0), (h << 16) | static_cast<int>(n_q),
-                              static_cast<int>(lo), static_cast<int>(hi));
+
+    auto doc_of = [&](int g) {  // last d with doc_blocks[d] <= g (skips empty documents)
+        int lo = 0, hi = p.batch;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (doc_blocks[mid] <= g) lo = mid; else hi = mid;
         }
+        return lo;
+    };
+    // (3) cost histogram
+    for (int g = tid; g < n_blocks; g += kSchedThreads) {
+        const int d = doc_of(g);
+        const BlockRange r = block_range(p, p.cu_seqlens[d] * mult, p.cu_seqlens[d + 1] * mult,
+                                         g - doc_blocks[d], n_buckets);
+        atomicAdd(&hist[r.cost], 1);
+    }
+    __syncthreads();
+    // (4) exclusive scan in descending cost order: bucket c starts after all costlier buckets
+    carry = 0;
+    for (int base = 0; base < n_buckets; base += kSchedThreads) {
+        const int c = n_buckets - 1 - (base + tid);
+        const int v = c >= 0 ? hist[c] : 0;
+        int total;
+        const int ex = block_exclusive_scan(v, warp_sums, &total);
+        if (c >= 0) hist[c] = carry + ex;
+        carry += total;
+        __syncthreads();
+    }
+    // (5) emission
+    for (int g = tid; g < n_blocks; g += kSchedThreads) {
+        const int d = doc_of(g);
+        const BlockRange r = block_range(p, p.cu_seqlens[d] * mult, p.cu_seqlens[d + 1] * mult,
+                                         g - doc_blocks[d], n_buckets);
+        const int slot = atomicAdd(&hist[r.cost], 1);
+        int4* dst = items + static_cast<int64_t>(slot) * p.heads;
+        for (int h = 0; h < p.heads; ++h)
+            dst[h] = make_int4(r.q0, (h << 16) | r.n_q, r.kv_lo, r.kv_hi);
     }
     if (tid == 0) {
         hdr->n_items = static_cast<int>(n_items);
@@ -111,9 +177,16 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     }
 }
 
-cudaError_t launch_schedule(const AttnProblem& p, int capacity, int4* items, WorkspaceHeader* hdr,
-                            cudaStream_t stream) {
-    schedule_kernel<<<1, kSchedThreads, 0, stream>>>(p, capacity, items, hdr);
+int schedule_buckets(const AttnProblem& p) {
+    const int64_t slots = static_cast<int64_t>(p.max_len) * p.slot_mult;
+    const int64_t nb = (slots + kItemRows) / kBlockN + 2;
+    return static_cast<int>(nb < kMaxCostBuckets ? nb : kMaxCostBuckets);
+}
+
+cudaError_t launch_schedule(const AttnProblem& p, int capacity, int* doc_blocks, int4* items,
+                            WorkspaceHeader* hdr, cudaStream_t stream) {
+    schedule_kernel<<<1, kSchedThreads, 0, stream>>>(p, capacity, schedule_buckets(p), doc_blocks,
+                                                     items, hdr);
     return cudaGetLastError();
 }
 

@@ -48,10 +48,13 @@ def test_status_strings(pha):
 
 
 def test_workspace_bytes_closed_form(pha):
-    # 256-byte header + 16 bytes per (query tile of 128 slots, head) work item
-    assert pha.pha_attn_workspace_bytes(8, 1024, 12, 64, False) == 256 + 16 * 8 * 8 * 12
-    assert pha.pha_attn_workspace_bytes(113, 2048, 6, 128, True) == 256 + 16 * 113 * 32 * 3
-    assert pha.pha_attn_workspace_bytes(1, 1, 2, 64, True) == 256 + 16 * 1 * 1 * 1
+    # 256-byte header + int32[batch+1] padded to 16 bytes + 16 bytes per (block of 256 query
+    # slots, head) work item
+    def pad(n):
+        return (4 * (n + 1) + 15) // 16 * 16
+    assert pha.pha_attn_workspace_bytes(8, 1024, 12, 64, False) == 256 + pad(8) + 16 * 8 * 4 * 12
+    assert pha.pha_attn_workspace_bytes(113, 2048, 6, 128, True) == 256 + pad(113) + 16 * 113 * 16 * 3
+    assert pha.pha_attn_workspace_bytes(1, 1, 2, 64, True) == 256 + pad(1) + 16 * 1 * 1 * 1
     assert pha.pha_attn_workspace_bytes(0, 10, 2, 64, False) == 0
     assert pha.pha_attn_workspace_bytes(1, 10, 3, 64, True) == 0   # odd heads cannot pair
 
