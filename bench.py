@@ -184,9 +184,9 @@ def main():
     args = ap.parse_args()
     w = pick_workload(args)
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from paired_heads_b200 import dist as pdist
+
+    rank, world, local_rank = pdist.env()
 
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
@@ -197,14 +197,7 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    dist = pdist.init("nccl", device=dev)
 
     inp = synth.make_inputs(w, rank=rank)
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
@@ -229,8 +222,7 @@ def main():
         torch.cuda.get_device_properties(dev), "index") else local_rank)
     clocks.start()
     time.sleep(0.3)
-    if dist:
-        dist.barrier()
+    pdist.barrier(dist)
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -243,8 +235,7 @@ def main():
         ev[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
-    if dist:
-        dist.barrier()
+    pdist.barrier(dist)
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
     rope_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
@@ -253,10 +244,7 @@ def main():
     if status != 0:
         raise SystemExit(f"device status {status} after timing")
 
-    if dist:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = pdist.max_over_ranks(dist, elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
 
     # ---- end to end through the public API with host buffers
@@ -281,19 +269,14 @@ def main():
         e2e_step()
     torch.cuda.synchronize(dev)
     e_steps = max(5, min(args.steps, 20))
-    if dist:
-        dist.barrier()
+    pdist.barrier(dist)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(e_steps):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = a.elapsed_time(b) / e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = pdist.max_over_ranks(dist, a.elapsed_time(b) / e_steps, dev)
     h2d = sum(host[n].numel() * host[n].element_size() for n in host)
     d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * 4
 
@@ -353,9 +336,7 @@ def main():
                                           f"workload: float64 RoPE + attention, full rows"}
     if rank == 0:
         print(json.dumps(line))
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
+    pdist.finalize(dist)
 
 
 def load_traffic(w, kernel: str):
