@@ -147,6 +147,34 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
  */
 pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream);
 
+/*
+ * pha_attn_fwd_noalloc -- pha_attn_fwd without a caller-provided workspace.
+ *   The pages describe nothing like it: it exists for callers that cannot allocate device
+ *   memory, such as a plug-in that receives only its input and output buffers from a host
+ *   framework that owns all device memory, or latency-critical code that must not call
+ *   cudaMalloc because it can synchronise the whole device.
+ *   Arguments and results are those of pha_attn_fwd, minus workspace / workspace_bytes. The
+ *   scratch is a 1 MiB array inside the library, one per GPU, held by every GPU that loads the
+ *   library until the process exits. The call itself allocates nothing.
+ *   Limit: problems whose pha_attn_workspace_bytes(...) exceeds 1 MiB are rejected with
+ *   PHA_ERR_WORKSPACE before any launch (PHA_F32 uses no scratch and has no such limit).
+ *   Set-up: the first call on a device looks up the array's device address, with the calling
+ *   thread's current device; that device must be the one `stream` belongs to. Make that first
+ *   call before any stream capture.
+ *   Sharing: every call uses the same array, which keeps the last call's contents. Nothing in it
+ *   needs to start at zero (each call rewrites what it reads). Calls whose kernels can run at the
+ *   same time on one GPU (unordered streams, several host threads) race on the array; order them
+ *   on one stream or with events. The device-side status that pha_attn_status reports lives in
+ *   this array and cannot be read through this entry point.
+ *   Errors: as pha_attn_fwd; PHA_ERR_UNSUPPORTED for a device index >= 64; PHA_ERR_CUDA if the
+ *   address lookup fails.
+ */
+pha_status pha_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens, int batch, int max_len,
+                                int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                                pha_dtype dtype, int causal, int window, int paired, float scale,
+                                void* o, float* lse, pha_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

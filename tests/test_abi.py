@@ -27,8 +27,9 @@ def _declared():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["pha_attn_fwd", "pha_attn_status", "pha_attn_workspace_bytes",
-                           "pha_rope", "pha_rope_tables", "pha_status_string"]
+    assert _declared() == ["pha_attn_fwd", "pha_attn_fwd_noalloc", "pha_attn_status",
+                           "pha_attn_workspace_bytes", "pha_rope", "pha_rope_tables",
+                           "pha_status_string"]
 
 
 def test_library_exports_every_declared_symbol(pha):

@@ -1,0 +1,68 @@
+"""pha_attn_fwd_noalloc: the attention forward for callers that cannot allocate device memory
+(for example a plug-in that only receives its input and output buffers, or code that must not
+call cudaMalloc because it can synchronise the device). It uses a 1 MiB scratch array built into
+the library instead of a caller workspace. Checked through the C ABI against pha_attn_fwd on two
+different problems in a row, so stale contents of the shared array cannot leak into the second
+call. Collected last so that a failure here never hides the other tests."""
+import pytest
+import torch
+
+from paired_heads_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+LSE_ABS = 1e-3
+
+
+def _problems():
+    return [
+        synth.workload("paired_varlen", doc_lens=synth.geometric_doc_lengths(6000, 512.0, 2048, 1)),
+        synth.workload("gpt2", doc_lens=(1024, 700, 333)),
+    ]
+
+
+def _run(w, use_noalloc):
+    from paired_heads_b200 import pha
+
+    inp = {n: t.cuda() for n, t in synth.make_inputs(w).items()}
+    o = torch.full_like(inp["q"], float("nan"))
+    lse = torch.full((w.total, w.n_heads), float("nan"), device="cuda")
+    kw = dict(causal=w.causal, window=w.window, paired=w.paired, scale=w.scale)
+    if use_noalloc:
+        pha.pha_attn_fwd_noalloc(inp["q"], inp["k"], inp["v"], inp["cu_seqlens"], w.max_len, o,
+                                 lse, **kw)
+    else:
+        ws = torch.empty(pha.pha_attn_workspace_bytes(w.batch, w.max_len, w.n_heads, w.head_dim,
+                                                      w.paired), dtype=torch.uint8, device="cuda")
+        pha.pha_attn_fwd(inp["q"], inp["k"], inp["v"], inp["cu_seqlens"], w.max_len, o, lse, ws,
+                         **kw)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
+    from paired_heads_b200 import build
+
+    build.build()
+    for w in _problems():
+        o_ref, lse_ref = _run(w, use_noalloc=False)
+        o, lse = _run(w, use_noalloc=True)
+        err = (o.float() - o_ref.float()).abs()
+        assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+        assert err.max().item() <= BF16_MAX_ABS and err.mean().item() <= BF16_MEAN_ABS
+        assert (lse - lse_ref).abs().max().item() <= LSE_ABS
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    from paired_heads_b200 import pha
+
+    q = torch.zeros(16, 2, 64, dtype=torch.bfloat16, device="cuda")
+    cu = torch.tensor([0, 16], dtype=torch.int32, device="cuda")
+    # 70,000 documents of up to 2048 tokens need far more than 1 MiB of work list
+    with pytest.raises(pha.PhaError) as e:
+        pha.pha_attn_fwd_noalloc(q, q, q, cu, 2048, torch.empty_like(q), None, batch=70000,
+                                 total_tokens=16, n_heads=2, n_kv_heads=2, head_dim=64,
+                                 dtype=pha.PHA_BF16)
+    assert e.value.code == -3
