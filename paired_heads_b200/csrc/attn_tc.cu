@@ -12,13 +12,15 @@
 // share one stream of 128-key K / V tiles. CTA = 10 warps, persistent (one CTA per SM, static
 // round-robin over the longest-first work list):
 //   warps 0-3   softmax of sub-tile 0      warps 4-7   softmax of sub-tile 1
-//               thread = query row = TMEM lane. Two passes over the S row in TMEM (row max, then
-//               exponentials), masking only tiles that straddle a causal / window / document
-//               edge; P (bf16) is written back into the first 64 columns of its own S buffer;
-//               O is rescaled in TMEM only when the running max grew by more than 2^8. At the end
-//               the row is normalised and O and the LSE are stored.
-//   warp 8      TMA producer: Q of both sub-tiles, then K and V tiles into kKStages / kVStages
-//               rings (64-column x 128-row boxes, 128-byte swizzle).
+//               thread = query row = TMEM lane. Two passes over the S row in TMEM (row max with
+//               three-input max, then exponentials with packed f32x2 arithmetic). Masks are
+//               applied only on tiles that straddle a causal / window / document edge, and only
+//               the bound(s) that tile needs. P (bf16) goes back into the first 64 columns of its
+//               own S buffer; O is rescaled in TMEM only when the running max grew by more than
+//               2^8. At the end the row is normalised and O and the LSE are stored.
+//   warp 8      TMA producer: Q sub-tiles into a ring of 3 slots (so the next item's Q arrives
+//               while the current item computes), K and V tiles into their rings (64-column x
+//               128-row boxes, 128-byte swizzle).
 //   warp 9      MMA issuer (one thread) and TMEM owner (512 columns):
 //               S_r = Q_r K^T   tcgen05.mma kind::f16, A and B from shared memory, M=128 N=128
 //               O_r += P_r V    tcgen05.mma kind::f16, A (P) from TMEM, B (V) from shared memory
@@ -48,10 +50,11 @@ struct TcLayout {
     static constexpr int kChunk = 128 * 128;  // one [128 rows][64 bf16] swizzled chunk (bytes)
     static constexpr int kQSub = kBlockM * HD * 2;
     static constexpr int kKV = kBlockN * HD * 2;
-    static constexpr int kKStages = HD == 128 ? 3 : 4;
+    static constexpr int kQSlots = 3;
+    static constexpr int kKStages = HD == 128 ? 2 : 4;
     static constexpr int kVStages = HD == 128 ? 2 : 4;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + 2 * kQSub;
+    static constexpr int kOffK = kOffQ + kQSlots * kQSub;
     static constexpr int kOffV = kOffK + kKStages * kKV;
     static constexpr int kOffBar = kOffV + kVStages * kKV;
     static constexpr int kBarBytes = 512;
@@ -62,7 +65,7 @@ struct TcLayout {
 };
 
 struct TcBars {
-    uint64_t q_full, q_empty;
+    uint64_t q_full[3], q_empty[3];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2], pv_done[2], o_ready[2];
     uint64_t drain;
@@ -92,8 +95,8 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int kk) {
 
 // A decoded work item and the per-sub-tile key ranges (identical in every role).
 struct Item {
-    int q0, n_q, head, kv_lo, kv_hi, n_kv;
-    int nr[2];               // valid rows of sub-tile r (0 = sub-tile absent)
+    int q0, n_q, head, kv_lo, kv_hi, n_kv, n_sub;
+    int nr[2];                  // valid rows of sub-tile r (0 = sub-tile absent)
     int t_first[2], t_last[2];  // key tiles sub-tile r needs
 };
 
@@ -105,6 +108,7 @@ __device__ __forceinline__ Item decode_item(int4 w, const AttnProblem& p) {
     it.kv_lo = w.z;
     it.kv_hi = w.w;
     it.n_kv = (w.w - w.z + kBlockN - 1) / kBlockN;
+    it.n_sub = it.n_q > kBlockM ? 2 : 1;
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int qr0 = it.q0 + kBlockM * r;
@@ -120,6 +124,48 @@ __device__ __forceinline__ Item decode_item(int4 w, const AttnProblem& p) {
         it.t_last[r] = nr > 0 ? (hi - 1 - it.kv_lo) / kBlockN : -1;
     }
     return it;
+}
+
+// Mask modes of one (sub-tile, key tile): which column bounds some row of the tile needs.
+enum : int { kMaskNone = 0, kMaskLo = 1, kMaskHi = 2, kMaskBoth = 3 };
+
+template <int MODE>
+__device__ __forceinline__ float mask_col(float s, int c, int c_lo, int c_hi) {
+    if (MODE & kMaskLo) s = c < c_lo ? -INFINITY : s;
+    if (MODE & kMaskHi) s = c > c_hi ? -INFINITY : s;
+    return s;
+}
+
+// Pass 1 over 64 columns starting at `base`: running max of the visible scores.
+template <int MODE>
+__device__ __forceinline__ float row_max64(const uint32_t* v, int base, int c_lo, int c_hi,
+                                           float mx) {
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
+        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
+        mx = fmax3(mx, a, b);
+    }
+    return mx;
+}
+
+// Pass 2 over 64 columns: p = 2^(s * scale_log2 - m) for the visible scores (0 elsewhere),
+// packed into 32 bf16 pairs; returns the (two-lane) partial row sum.
+template <int MODE>
+__device__ __forceinline__ uint64_t row_exp64(const uint32_t* v, int base, int c_lo, int c_hi,
+                                              uint64_t scale2, uint64_t negm2, uint64_t sum2,
+                                              uint32_t* pk) {
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
+        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
+        float xa, xb;
+        f32x2_split(fma_f32x2(f32x2(a, b), scale2, negm2), xa, xb);
+        const float pa = ex2(xa), pb = ex2(xb);
+        sum2 = add_f32x2(sum2, f32x2(pa, pb));
+        pk[e >> 1] = pack_bf16x2(pa, pb);
+    }
+    return sum2;
 }
 
 template <int HD>
@@ -140,8 +186,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int lane = threadIdx.x & 31;
 
     if (warp == 8 && lane == 0) {
-        mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+        }
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
@@ -177,23 +225,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t it_cnt = 0, kc = 0, vc = 0;
+            uint32_t qc = 0, kc = 0, vc = 0;
             bool ok = true;
+            int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
             for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
-                const Item it = decode_item(__ldg(items + idx), p);
+                const Item it = decode_item(next, p);
+                if (idx + gridDim.x < n_items) next = __ldg(items + idx + gridDim.x);  // prefetch
                 const int g = it.head / G;
-                if (!mbar_wait(&bars->q_empty, (it_cnt & 1) ^ 1, abort_flag, dev_status)) {
-                    ok = false;
-                    break;
-                }
-                const int n_sub = it.nr[1] > 0 ? 2 : 1;
-                mbar_arrive_expect_tx(&bars->q_full, n_sub * L::kQSub);
-                for (int r = 0; r < n_sub; ++r)
+                for (int r = 0; r < it.n_sub; ++r) {
+                    const uint32_t sq = qc % L::kQSlots;
+                    if (!mbar_wait(&bars->q_empty[sq], ((qc / L::kQSlots) & 1) ^ 1, abort_flag,
+                                   dev_status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars->q_full[sq], L::kQSub);
                     for (int c = 0; c < HD / 64; ++c)
-                        tma_load_2d(smem + L::kOffQ + r * L::kQSub + c * L::kChunk, &tm_q,
-                                    it.head * HD + 64 * c, it.q0 + kBlockM * r, &bars->q_full);
-                ++it_cnt;
-                for (int t = 0; t < it.n_kv; ++t) {
+                        tma_load_2d(smem + L::kOffQ + sq * L::kQSub + c * L::kChunk, &tm_q,
+                                    it.head * HD + 64 * c, it.q0 + kBlockM * r, &bars->q_full[sq]);
+                    ++qc;
+                }
+                for (int t = 0; ok && t < it.n_kv; ++t) {
                     const int row = it.kv_lo + t * kBlockN;
                     const uint32_t sk = kc % L::kKStages;
                     if (!mbar_wait(&bars->k_empty[sk], ((kc / L::kKStages) & 1) ^ 1, abort_flag,
@@ -221,7 +273,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (!ok) {
                 // Wait (bounded) for the copies this thread issued last into every buffer.
-                if (it_cnt > 0) drain_wait(&bars->q_full, (it_cnt - 1) & 1);
+                for (uint32_t n = qc > L::kQSlots ? qc - L::kQSlots : 0; n < qc; ++n)
+                    drain_wait(&bars->q_full[n % L::kQSlots], (n / L::kQSlots) & 1);
                 for (uint32_t n = kc > L::kKStages ? kc - L::kKStages : 0; n < kc; ++n)
                     drain_wait(&bars->k_full[n % L::kKStages], (n / L::kKStages) & 1);
                 for (uint32_t n = vc > L::kVStages ? vc - L::kVStages : 0; n < vc; ++n)
@@ -234,16 +287,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, HD, 0, 1);
-            uint32_t it_cnt = 0, kc = 0, vc = 0;
+            uint32_t qc = 0, kc = 0, vc = 0;
             uint32_t p_cnt[2] = {0, 0};
             bool ok = true;
+            int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
             for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
-                const Item it = decode_item(__ldg(items + idx), p);
-                if (!mbar_wait(&bars->q_full, it_cnt & 1, abort_flag, dev_status)) {
-                    ok = false;
-                    break;
+                const Item it = decode_item(next, p);
+                if (idx + gridDim.x < n_items) next = __ldg(items + idx + gridDim.x);  // prefetch
+                uint32_t q_slot[2], q_par[2];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    q_slot[r] = (qc + r) % L::kQSlots;
+                    q_par[r] = ((qc + r) / L::kQSlots) & 1;
                 }
-                tc_fence_after();
                 for (int t = 0; t < it.n_kv && ok; ++t) {
                     const uint32_t sk = kc % L::kKStages;
                     if (!mbar_wait(&bars->k_full[sk], (kc / L::kKStages) & 1, abort_flag, dev_status)) {
@@ -255,23 +311,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         if (t < it.t_first[r] || t > it.t_last[r]) continue;
-                        // S_r reuses the columns of P_r: the last P_r . V must have finished
-                        if (p_cnt[r] > 0 && !mbar_wait(&bars->pv_done[r], (p_cnt[r] - 1) & 1,
-                                                       abort_flag, dev_status)) {
+                        // Q_r must have landed (first tile of the sub-tile), and S_r reuses the
+                        // columns of P_r: the last P_r . V must have finished.
+                        if ((t == it.t_first[r] &&
+                             !mbar_wait(&bars->q_full[q_slot[r]], q_par[r], abort_flag, dev_status)) ||
+                            (p_cnt[r] > 0 && !mbar_wait(&bars->pv_done[r], (p_cnt[r] - 1) & 1,
+                                                        abort_flag, dev_status))) {
                             ok = false;
                             break;
                         }
-                        const uint32_t q_tile = sbase + L::kOffQ + r * L::kQSub;
+                        tc_fence_after();
+                        const uint32_t q_tile = sbase + L::kOffQ + q_slot[r] * L::kQSub;
 #pragma unroll
                         for (int kk = 0; kk < HD / 16; ++kk)
                             umma_f16_ss(tmem + 128 * r, desc_kmajor(q_tile, kk), desc_kmajor(k_tile, kk),
                                         idesc_qk, kk == 0 ? 0u : 1u);
                         umma_commit(&bars->s_full[r]);
+                        if (t == it.t_last[r]) umma_commit(&bars->q_empty[q_slot[r]]);
                     }
                     if (!ok) break;
                     umma_commit(&bars->k_empty[sk]);
                     ++kc;
-                    if (t == it.n_kv - 1) umma_commit(&bars->q_empty);
                     const uint32_t sv = vc % L::kVStages;
                     if (!mbar_wait(&bars->v_full[sv], (vc / L::kVStages) & 1, abort_flag, dev_status)) {
                         ok = false;
@@ -300,7 +360,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     umma_commit(&bars->v_empty[sv]);
                     ++vc;
                 }
-                ++it_cnt;
+                qc += it.n_sub;
             }
             // Wait (bounded) until every MMA this thread issued has finished.
             umma_commit(&bars->drain);
@@ -315,11 +375,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t tm_s = tm_lane + 128 * r;
         const uint32_t tm_o = tm_lane + L::kTmO + HD * r;
         const float scale_log2 = p.scale * kLog2e;
+        const uint64_t scale2 = f32x2(scale_log2, scale_log2);
         const int window = p.window;
         uint32_t s_cnt = 0, o_cnt = 0;
         bool ok = true;
+        int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
-            const Item it = decode_item(__ldg(items + idx), p);
+            const Item it = decode_item(next, p);
+            if (idx + gridDim.x < n_items) next = __ldg(items + idx + gridDim.x);  // prefetch
             // per-sub-tile fields by select (r is not a compile-time index here)
             const int nr = r ? it.nr[1] : it.nr[0];
             const int t_first = r ? it.t_first[1] : it.t_first[0];
@@ -330,6 +393,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // visible key slots of this row: [j_min, j_max]
             const int j_max = p.causal ? min(i, it.kv_hi - 1) : it.kv_hi - 1;
             const int j_min = window > 0 ? i - window + 1 : INT32_MIN / 2;
+            // a tile needs the lower / upper bound iff some valid row of the sub-tile does:
+            // the largest j_min belongs to the last valid row, the smallest j_max to the first
+            const int tile_jmin = window > 0 ? qr0 + nr - window : INT32_MIN / 2;
+            const int tile_jmax = p.causal ? min(qr0, it.kv_hi - 1) : it.kv_hi - 1;
             float m = -INFINITY, l = 0.f;
             for (int t = t_first; t <= t_last; ++t) {
                 const int kv0 = it.kv_lo + t * kBlockN;
@@ -338,11 +405,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ok) break;
                 ++s_cnt;
                 tc_fence_after();
-                const bool full_tile = (kv0 + kBlockN - 1 < it.kv_hi) &&
-                                       (!p.causal || kv0 + kBlockN - 1 <= qr0) &&
-                                       (window <= 0 || (qr0 + nr - 1) - kv0 < window);
-                const int c_lo = full_tile ? 0 : j_min - kv0;
-                const int c_hi = full_tile ? kBlockN - 1 : j_max - kv0;
+                const int mode = (tile_jmin > kv0 ? kMaskLo : 0) |
+                                 (kv0 + kBlockN - 1 > tile_jmax ? kMaskHi : 0);
+                const int c_lo = j_min - kv0, c_hi = j_max - kv0;
                 // pass 1: row max over the visible columns
                 float mx = -INFINITY;
 #pragma unroll 1
@@ -351,11 +416,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld32(tm_s + 64 * hlf, v);
                     tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const int c = 64 * hlf + e;
-                        const float s = (c < c_lo || c > c_hi) ? -INFINITY : __uint_as_float(v[e]);
-                        mx = fmaxf(mx, s);
+                    switch (mode) {
+                        case kMaskNone: mx = row_max64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, mx); break;
+                        case kMaskLo: mx = row_max64<kMaskLo>(v, 64 * hlf, c_lo, c_hi, mx); break;
+                        case kMaskHi: mx = row_max64<kMaskHi>(v, 64 * hlf, c_lo, c_hi, mx); break;
+                        default: mx = row_max64<kMaskBoth>(v, 64 * hlf, c_lo, c_hi, mx); break;
                     }
                 }
                 const float m_new = fmaxf(m, mx * scale_log2);
@@ -364,9 +429,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const bool rescale = m_new > m + 8.0f;
                 const float alpha = rescale ? ex2(m - m_new) : 1.0f;
                 if (rescale) m = m_new;
-                const float m_safe = (m == -INFINITY) ? 0.f : m;
-                // pass 2: P = exp2(s * scale * log2e - m) as bf16 into the first half of S
-                float sum = 0.f;
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                const uint64_t negm2 = f32x2(neg_m, neg_m);
+                // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first half of S
+                uint64_t sum2 = f32x2(0.f, 0.f);
 #pragma unroll 1
                 for (int hlf = 0; hlf < 2; ++hlf) {
                     uint32_t v[64];
@@ -374,20 +440,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
                     tmem_wait_ld();
                     uint32_t pk[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = 64 * hlf + 2 * e;
-                        const float s0 = (c < c_lo || c > c_hi) ? -INFINITY : __uint_as_float(v[2 * e]);
-                        const float s1 = (c + 1 < c_lo || c + 1 > c_hi) ? -INFINITY
-                                                                          : __uint_as_float(v[2 * e + 1]);
-                        const float p0 = ex2(fmaf(s0, scale_log2, -m_safe));
-                        const float p1 = ex2(fmaf(s1, scale_log2, -m_safe));
-                        sum += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
+                    switch (mode) {
+                        case kMaskNone: sum2 = row_exp64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                        case kMaskLo: sum2 = row_exp64<kMaskLo>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                        case kMaskHi: sum2 = row_exp64<kMaskHi>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                        default: sum2 = row_exp64<kMaskBoth>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
                     }
                     tmem_st32(tm_s + 32 * hlf, pk);
                 }
-                l = l * alpha + sum;
+                float s_lo, s_hi;
+                f32x2_split(sum2, s_lo, s_hi);
+                l = l * alpha + (s_lo + s_hi);
                 if (t > t_first && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {

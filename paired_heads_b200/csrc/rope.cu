@@ -7,9 +7,9 @@
 // table" (row p packs the angles of positions 2p and 2p+1). Frequencies: "Training an LLM from
 // scratch (part 2)", section "2. RoPE".
 //
-// The rotation is HBM-bound: each thread moves one 32-byte span of one (token, head) row with
-// two 16-byte loads and stores; the table row of a token is shared by all of its heads and is
-// served from L1/L2. Every output is the correctly rounded (nearest even) value of the rotation
+// The rotation is HBM-bound: one warp per token moves the token's q and k rows in 16-byte chunks
+// (coalesced 512-byte warp accesses, several chunks in flight per lane); the table row of a token
+// is shared by all of its heads and is served from L1/L2. Every output is the correctly rounded (nearest even) value of the rotation
 // with the tables' float32 cosines and sines:
 //   bf16: y = fma(c, a, s*b) in float32 differs from the exact value by at most
 //         ulp(y)/2 + ulp(s*b)/2; when y lies farther than that from the nearest bf16 rounding
@@ -80,91 +80,108 @@ __device__ __forceinline__ uint32_t rot_bf16(float a, float c, float b, float sb
                              static_cast<double>(sb) * static_cast<double>(b)));
 }
 
+// 16-byte chunks of a row: 8 bf16 (4 pairs) or 4 f32 (2 pairs), rotated with the chunk's table
+// values c[j], s[j] (j = element within the chunk).
 template <typename T>
-struct Span32;  // 32 bytes of one row: 16 bf16 or 8 f32
+struct Chunk16;
 
 template <>
-struct Span32<__nv_bfloat16> {
-    static constexpr int N = 16;
-    __device__ static void rotate(__nv_bfloat16* p, const float (&c)[N], const float (&s)[N]) {
-        const uint4 a = *reinterpret_cast<const uint4*>(p);
-        const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        uint32_t o[8];
+struct Chunk16<__nv_bfloat16> {
+    static constexpr int E = 8;
+    __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
             const float x0 = __uint_as_float(w[e] << 16);
             const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
             o[e] = rot_bf16(x0, c[2 * e], x1, -s[2 * e]) |
                    (rot_bf16(x1, c[2 * e + 1], x0, s[2 * e + 1]) << 16);
         }
-        *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(p + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+        return make_uint4(o[0], o[1], o[2], o[3]);
     }
 };
 
 template <>
-struct Span32<float> {
-    static constexpr int N = 8;
-    __device__ static void rotate(float* p, const float (&c)[N], const float (&s)[N]) {
-        const float4 a = *reinterpret_cast<const float4*>(p);
-        const float4 b = *reinterpret_cast<const float4*>(p + 4);
-        const float x[N] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        float y[N];
+struct Chunk16<float> {
+    static constexpr int E = 4;
+    __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
+        const float x[E] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z),
+                            __uint_as_float(a.w)};
+        float y[E];
 #pragma unroll
-        for (int e = 0; e < N; e += 2) {
+        for (int e = 0; e < E; e += 2) {
             // products of float32 values are exact in double: one rounding in the fma, one to f32
             y[e] = __double2float_rn(fma(static_cast<double>(c[e]), static_cast<double>(x[e]),
                                          -static_cast<double>(s[e]) * static_cast<double>(x[e + 1])));
             y[e + 1] = __double2float_rn(fma(static_cast<double>(c[e + 1]), static_cast<double>(x[e + 1]),
                                              static_cast<double>(s[e + 1]) * static_cast<double>(x[e])));
         }
-        *reinterpret_cast<float4*>(p) = make_float4(y[0], y[1], y[2], y[3]);
-        *reinterpret_cast<float4*>(p + 4) = make_float4(y[4], y[5], y[6], y[7]);
+        return make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                          __float_as_uint(y[3]));
     }
 };
 
-// One thread per 32-byte span. Spans are numbered q first, then k; inside a tensor the order is
-// (token, head, span) so that consecutive threads touch consecutive bytes.
+// One warp per token. The token's q row (n_heads * head_dim contiguous elements) followed by its
+// k row is cut into 16-byte chunks; lane l takes chunks l, l + 32, ... in batches of kBatch, so
+// every load instruction of the warp reads 512 contiguous bytes and each lane keeps kBatch x 16
+// bytes of HBM reads in flight. All heads of the token share its table row, which is read from
+// HBM once and then served from L1.
+constexpr int kRopeBatch = 8;
+
 template <typename T>
 __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restrict__ k,
                                                    const float* __restrict__ cos_tab,
                                                    const float* __restrict__ sin_tab,
                                                    int tab_rows, int tab_width,
                                                    const int32_t* __restrict__ positions,
-                                                   int64_t n_q_spans, int64_t n_spans, int n_heads,
+                                                   int64_t total_tokens, int n_heads,
                                                    int n_kv_heads, int head_dim, int paired,
                                                    int stagger_offset) {
-    constexpr int N = Span32<T>::N;
-    const int spans_per_head = head_dim / N;
-    const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    if (idx >= n_spans) return;
-    const bool is_k = idx >= n_q_spans;
-    const int64_t local = is_k ? idx - n_q_spans : idx;
-    const int H = is_k ? n_kv_heads : n_heads;
-    T* base = is_k ? k : q;
-    const int span = static_cast<int>(local % spans_per_head);
-    const int64_t th = local / spans_per_head;
-    const int h = static_cast<int>(th % H);
-    const int64_t t = th / H;
-    const int pos = __ldg(positions + t);
-    if (pos < 0 || pos >= tab_rows) return;
-    const int col = ((paired && (h & 1)) ? stagger_offset : 0) + span * N;
-    const float* crow = cos_tab + static_cast<int64_t>(pos) * tab_width + col;
-    const float* srow = sin_tab + static_cast<int64_t>(pos) * tab_width + col;
-    T* p = base + local * N;
-
-    float c[N], s[N];
+    constexpr int E = Chunk16<T>::E;
+    const int cph = head_dim / E;                  // chunks per head row
+    const int q_chunks = n_heads * cph;
+    const int n_chunks = q_chunks + n_kv_heads * cph;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t t = warp0; t < total_tokens; t += n_warps) {
+        const int pos = __ldg(positions + t);
+        const bool in_range = pos >= 0 && pos < tab_rows;
+        uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
+        uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
+        const float* crow = cos_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
+        const float* srow = sin_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
+        for (int base = 0; base < n_chunks; base += 32 * kRopeBatch) {
+            uint4 raw[kRopeBatch];
 #pragma unroll
-    for (int e = 0; e < N; e += 4) {
-        const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + e));
-        const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + e));
-        c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
-        s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
+            for (int j = 0; j < kRopeBatch; ++j) {
+                const int i = base + 32 * j + lane;
+                if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
+            }
+            if (!in_range) continue;  // positions outside the table: leave the token unchanged
+#pragma unroll
+            for (int j = 0; j < kRopeBatch; ++j) {
+                const int i = base + 32 * j + lane;
+                if (i >= n_chunks) break;
+                const int ih = i < q_chunks ? i : i - q_chunks;  // chunk index within q or k row
+                const int h = ih / cph;
+                const int col = ((paired && (h & 1)) ? stagger_offset : 0) + (ih - h * cph) * E;
+                float c[E], s[E];
+#pragma unroll
+                for (int e = 0; e < E; e += 4) {
+                    const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col + e));
+                    const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col + e));
+                    c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
+                    s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
+                }
+                // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign
+                // is -1 on the even member and +1 on the odd member (a rotation by +angle).
+                const uint4 y = Chunk16<T>::rotate(raw[j], c, s);
+                if (i < q_chunks) qrow[i] = y; else krow[i - q_chunks] = y;
+            }
+        }
     }
-    // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign is -1 on
-    // the even member and +1 on the odd member, which is a rotation by +angle.
-    Span32<T>::rotate(p, c, s);
 }
 
 cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
@@ -183,22 +200,19 @@ cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin
                         int tab_width, const int32_t* positions, int total_tokens, int n_heads,
                         int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
                         cudaStream_t stream) {
-    const int N = is_bf16 ? 16 : 8;
-    const int64_t n_q = static_cast<int64_t>(total_tokens) * n_heads * (head_dim / N);
-    const int64_t n_all = n_q + static_cast<int64_t>(total_tokens) * n_kv_heads * (head_dim / N);
-    if (n_all == 0) return cudaSuccess;
-    const int threads = 256;
-    const int64_t blocks = (n_all + threads - 1) / threads;
-    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    if (total_tokens == 0) return cudaSuccess;
+    const int threads = 256;  // 8 warps = 8 tokens per block
+    const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
+    const unsigned blocks = static_cast<unsigned>(blocks64 < (1 << 30) ? blocks64 : (1 << 30));
     if (is_bf16)
-        rope_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        rope_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
             static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), cos_tab, sin_tab,
-            tab_rows, tab_width, positions, n_q, n_all, n_heads, n_kv_heads, head_dim, paired,
+            tab_rows, tab_width, positions, total_tokens, n_heads, n_kv_heads, head_dim, paired,
             stagger_offset);
     else
-        rope_kernel<float><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        rope_kernel<float><<<blocks, threads, 0, stream>>>(
             static_cast<float*>(q), static_cast<float*>(k), cos_tab, sin_tab, tab_rows, tab_width,
-            positions, n_q, n_all, n_heads, n_kv_heads, head_dim, paired, stagger_offset);
+            positions, total_tokens, n_heads, n_kv_heads, head_dim, paired, stagger_offset);
     return cudaGetLastError();
 }
 
