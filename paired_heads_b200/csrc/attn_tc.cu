@@ -416,6 +416,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld32(tm_s + 64 * hlf, v);
                     tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
                     tmem_wait_ld();
+                    regs_after_wait(v);
+                    regs_after_wait(v + 32);
                     switch (mode) {
                         case kMaskNone: mx = row_max64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, mx); break;
                         case kMaskLo: mx = row_max64<kMaskLo>(v, 64 * hlf, c_lo, c_hi, mx); break;
@@ -439,6 +441,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld32(tm_s + 64 * hlf, v);
                     tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
                     tmem_wait_ld();
+                    regs_after_wait(v);
+                    regs_after_wait(v + 32);
                     uint32_t pk[32];
                     switch (mode) {
                         case kMaskNone: sum2 = row_exp64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
@@ -457,6 +461,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         uint32_t v[32];
                         tmem_ld32(tm_o + 32 * c, v);
                         tmem_wait_ld();
+                        regs_after_wait(v);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
                         tmem_st32(tm_o + 32 * c, v);
@@ -482,6 +487,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint32_t v[32];
                 tmem_ld32(tm_o + 32 * c, v);
                 tmem_wait_ld();
+                regs_after_wait(v);
                 if (valid) {
                     uint32_t pk[16];
 #pragma unroll

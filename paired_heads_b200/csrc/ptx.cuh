@@ -57,6 +57,19 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase of `bar` with the given parity. Returns false (and raises the
 // CTA-wide abort flag and the device status) when the limit passes or another thread of the
 // CTA has already aborted. Never spins forever.
@@ -210,6 +223,44 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// tcgen05.ld fills its destination registers asynchronously; these waits list the registers as
+// read-write operands so that the compiler cannot move a use of them above the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+          "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+          "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+          "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+          "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+          "+r"(r[31])
+        :
+        : "memory");
+}
+
+// No instruction: marks 32 registers as written at this point, after a tcgen05.wait::ld, so that
+// the compiler keeps every use of them below the wait.
+__device__ __forceinline__ void regs_after_wait(uint32_t* r) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31]));
+}
+
+// 16 consecutive 32-bit columns for the warp's 32 lanes.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -248,6 +299,28 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
+}
+
+// Two base-2 exponentials on the FMA pipe (no special-function unit): x = n + f with
+// n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low mantissa bits), f in [-0.5, 0.5];
+// 2^f from a degree-3 polynomial fitted to 2^f on [-0.5, 0.5] in relative error (coefficients from
+// exp2_poly_fit.py; max relative error 7.5e-5), and n added to the exponent field. Inputs below
+// -126 (including -inf) are clamped there, giving a value < 2^-125 in place of 0.
+__device__ __forceinline__ void ex2_poly2(float xa, float xb, float& ya, float& yb) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    const uint64_t x2 = f32x2(fmaxf(xa, -126.0f), fmaxf(xb, -126.0f));
+    const uint64_t j2 = add_f32x2(x2, f32x2(kShift, kShift));
+    const uint64_t n2 = add_f32x2(j2, f32x2(-kShift, -kShift));
+    const uint64_t f2 = fma_f32x2(n2, f32x2(-1.0f, -1.0f), x2);
+    uint64_t p2 = fma_f32x2(f2, f32x2(0.055170975625514984f, 0.055170975625514984f),
+                            f32x2(0.24260970950126648f, 0.24260970950126648f));
+    p2 = fma_f32x2(p2, f2, f32x2(0.6932609677314758f, 0.6932609677314758f));
+    p2 = fma_f32x2(p2, f2, f32x2(0.9999281764030457f, 0.9999281764030457f));
+    float ja, jb, pa, pb;
+    f32x2_split(j2, ja, jb);
+    f32x2_split(p2, pa, pb);
+    ya = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ja) << 23));
+    yb = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(jb) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
