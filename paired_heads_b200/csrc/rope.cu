@@ -62,22 +62,35 @@ __device__ __noinline__ uint32_t bf16_bits_rne(double y) {
     return sign | bits;
 }
 
-// One rotated element y = c*a + sb*b (sb = -s for the even member of a pair, +s for the odd one),
-// as the 16-bit pattern of the nearest bf16 of the exact value.
-__device__ __forceinline__ uint32_t rot_bf16(float a, float c, float b, float sb) {
-    const float t = sb * b;
-    const float y = fmaf(c, a, t);  // c*a enters the fma unrounded
-    const uint32_t bits = __float_as_uint(y);
-    // float32 ulps of y to the bf16 rounding midpoint of its binade (pattern ...8000)
-    const int dist = abs(static_cast<int>(bits & 0xFFFFu) - 0x8000);
-    // |y - exact| <= ulp(y)/2 + |t| 2^-24 < (1/2 + |t|/|y|) ulp(y); keep 1.5 ulp of margin
-    if (fabsf(t) <= fabsf(y) * static_cast<float>(dist - 2)) {
-        uint32_t r;
-        asm("{\n\t.reg .b16 h;\n\tcvt.rn.bf16.f32 h, %1;\n\tmov.b32 %0, {h, h};\n\t}" : "=r"(r) : "f"(y));
-        return r & 0xFFFFu;
-    }
-    return bf16_bits_rne(fma(static_cast<double>(c), static_cast<double>(a),
-                             static_cast<double>(sb) * static_cast<double>(b)));
+// float32 ulps from y to the bf16 rounding midpoint of y's binade (bit pattern ...8000), as a
+// float: the low 16 bits OR-ed into 2^23 give 2^23 + low16 exactly.
+__device__ __forceinline__ float ulps_to_midpoint(float y) {
+    return __uint_as_float((__float_as_uint(y) & 0xFFFFu) | 0x4B000000u) - 8421376.0f;  // 2^23 + 2^15
+}
+
+// y = fma(c, a, t) with t = rounded s*b is within ulp(y)/2 + |t| 2^-24 < (1/2 + |t|/|y|) ulp(y)
+// of the exact c*a + s*b; when y lies more than that (plus 1.5 ulp of margin) from the bf16
+// rounding midpoint, rounding y gives the bf16 of the exact value.
+__device__ __forceinline__ bool rounds_like_exact(float y, float t) {
+    return fabsf(t) <= fabsf(y) * (fabsf(ulps_to_midpoint(y)) - 2.0f);
+}
+
+// One rotated pair (x0, x1) with the pair's table values c, s:
+//   y0 = c x0 - s x1,  y1 = c x1 + s x0   (packed f32x2 arithmetic)
+// as two bf16 of the exact values (16-bit patterns, y0 in the low half).
+__device__ __forceinline__ uint32_t rot_pair_bf16(float x0, float x1, float c, float s) {
+    const uint64_t t2 = mul_f32x2(f32x2(-s, s), f32x2(x1, x0));
+    const uint64_t y2 = fma_f32x2(f32x2(c, c), f32x2(x0, x1), t2);
+    float y0, y1, t0, t1;
+    f32x2_split(y2, y0, y1);
+    f32x2_split(t2, t0, t1);
+    if (rounds_like_exact(y0, t0) && rounds_like_exact(y1, t1)) return pack_bf16x2(y0, y1);
+    // rare: recompute in float64, where bf16 x float32 products are exact
+    const double e0 = fma(static_cast<double>(c), static_cast<double>(x0),
+                          -static_cast<double>(s) * static_cast<double>(x1));
+    const double e1 = fma(static_cast<double>(c), static_cast<double>(x1),
+                          static_cast<double>(s) * static_cast<double>(x0));
+    return bf16_bits_rne(e0) | (bf16_bits_rne(e1) << 16);
 }
 
 // 16-byte chunks of a row: 8 bf16 (4 pairs) or 4 f32 (2 pairs), rotated with the chunk's table
@@ -92,12 +105,9 @@ struct Chunk16<__nv_bfloat16> {
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
         uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float x0 = __uint_as_float(w[e] << 16);
-            const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
-            o[e] = rot_bf16(x0, c[2 * e], x1, -s[2 * e]) |
-                   (rot_bf16(x1, c[2 * e + 1], x0, s[2 * e + 1]) << 16);
-        }
+        for (int e = 0; e < 4; ++e)  // both members of a pair share one angle: c[2e] == c[2e+1]
+            o[e] = rot_pair_bf16(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u),
+                                 c[2 * e], s[2 * e]);
         return make_uint4(o[0], o[1], o[2], o[3]);
     }
 };
@@ -152,6 +162,21 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
         uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
         const float* crow = cos_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
         const float* srow = sin_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
+        // When cph divides 32 (and, paired, 32/cph is even so the head parity is fixed too), every
+        // chunk of this lane sits at the same table columns: load them once per token.
+        const bool uniform_cols = (32 % cph == 0) && (!paired || ((32 / cph) % 2 == 0));
+        float cu[E], su[E];
+        if (uniform_cols && in_range) {
+            const int h0 = (lane % n_chunks) / cph;  // any chunk of this lane gives the columns
+            const int col0 = ((paired && (h0 & 1)) ? stagger_offset : 0) + (lane % cph) * E;
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+                const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col0 + e));
+                const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col0 + e));
+                cu[e] = cv.x; cu[e + 1] = cv.y; cu[e + 2] = cv.z; cu[e + 3] = cv.w;
+                su[e] = sv.x; su[e + 1] = sv.y; su[e + 2] = sv.z; su[e + 3] = sv.w;
+            }
+        }
         for (int base = 0; base < n_chunks; base += 32 * kRopeBatch) {
             uint4 raw[kRopeBatch];
 #pragma unroll
@@ -164,16 +189,24 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
             for (int j = 0; j < kRopeBatch; ++j) {
                 const int i = base + 32 * j + lane;
                 if (i >= n_chunks) break;
-                const int ih = i < q_chunks ? i : i - q_chunks;  // chunk index within q or k row
-                const int h = ih / cph;
-                const int col = ((paired && (h & 1)) ? stagger_offset : 0) + (ih - h * cph) * E;
                 float c[E], s[E];
+                if (uniform_cols) {
 #pragma unroll
-                for (int e = 0; e < E; e += 4) {
-                    const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col + e));
-                    const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col + e));
-                    c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
-                    s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
+                    for (int e = 0; e < E; ++e) {
+                        c[e] = cu[e];
+                        s[e] = su[e];
+                    }
+                } else {
+                    const int ih = i < q_chunks ? i : i - q_chunks;  // chunk index within q or k row
+                    const int h = ih / cph;
+                    const int col = ((paired && (h & 1)) ? stagger_offset : 0) + (ih - h * cph) * E;
+#pragma unroll
+                    for (int e = 0; e < E; e += 4) {
+                        const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col + e));
+                        const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col + e));
+                        c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
+                        s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
+                    }
                 }
                 // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign
                 // is -1 on the even member and +1 on the odd member (a rotation by +angle).
