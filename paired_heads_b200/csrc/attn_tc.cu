@@ -136,6 +136,36 @@ __device__ __forceinline__ float mask_col(float s, int c, int c_lo, int c_hi) {
     return s;
 }
 
+// Pass 1 over 32 columns starting at `base`: running max of the visible scores.
+template <int MODE>
+__device__ __forceinline__ float row_max32(const uint32_t* v, int base, int c_lo, int c_hi, float mx) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
+        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
+        mx = fmax3(mx, a, b);
+    }
+    return mx;
+}
+
+// Pass 2 over 32 columns: 16 packed bf16 pairs of p = 2^(s * scale_log2 - m), 0 where masked.
+template <int MODE>
+__device__ __forceinline__ uint64_t row_exp32(const uint32_t* v, int base, int c_lo, int c_hi,
+                                              uint64_t scale2, uint64_t negm2, uint64_t sum2,
+                                              uint32_t* pk) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
+        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
+        float xa, xb;
+        f32x2_split(fma_f32x2(f32x2(a, b), scale2, negm2), xa, xb);
+        const float pa = ex2(xa), pb = ex2(xb);
+        sum2 = add_f32x2(sum2, f32x2(pa, pb));
+        pk[e >> 1] = pack_bf16x2(pa, pb);
+    }
+    return sum2;
+}
+
 // Pass 1 over 64 columns starting at `base`: running max of the visible scores.
 template <int MODE>
 __device__ __forceinline__ float row_max64(const uint32_t* v, int base, int c_lo, int c_hi,
@@ -405,24 +435,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ok) break;
                 ++s_cnt;
                 tc_fence_after();
-                const int mode = (tile_jmin > kv0 ? kMaskLo : 0) |
-                                 (kv0 + kBlockN - 1 > tile_jmax ? kMaskHi : 0);
                 const int c_lo = j_min - kv0, c_hi = j_max - kv0;
+                // Masked tiles are processed in 32-column chunks classed uniformly over this
+                // warp's 32 rows [r0, r0 + 31]: the row bounds c_lo(row), c_hi(row) grow with the
+                // row, so a chunk is skipped when it lies below the first row's c_lo or above the
+                // last row's c_hi, needs no lower (upper) mask when it lies wholly at or above the
+                // last row's c_lo (at or below the first row's c_hi), and is masked on the needed
+                // side(s) otherwise. Skipped chunks cost no loads, no exponentials, and P = 0.
+                const bool full_tile = (tile_jmin <= kv0) && (kv0 + kBlockN - 1 <= tile_jmax);
+                const int r0 = (warp & 3) * 32;
+                const int lo_first = window > 0 ? qr0 + r0 - window + 1 - kv0 : INT32_MIN / 2;
+                const int lo_last = window > 0 ? lo_first + 31 : INT32_MIN / 2;
+                const int hi_first = (p.causal ? min(qr0 + r0, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
+                const int hi_last = (p.causal ? min(qr0 + r0 + 31, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
+                auto chunk_class = [&](int c) -> int {  // 4 = skip, else mask mode bits
+                    const int lo = 32 * c, hi = lo + 31;
+                    if (hi < lo_first || lo > hi_last) return 4;
+                    return (lo < lo_last ? kMaskLo : 0) | (hi > hi_first ? kMaskHi : 0);
+                };
                 // pass 1: row max over the visible columns
                 float mx = -INFINITY;
+                if (full_tile) {
+                    // unmasked tile: two 64-column halves, one wait each
 #pragma unroll 1
-                for (int hlf = 0; hlf < 2; ++hlf) {
-                    uint32_t v[64];
-                    tmem_ld32(tm_s + 64 * hlf, v);
-                    tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
-                    tmem_wait_ld();
-                    regs_after_wait(v);
-                    regs_after_wait(v + 32);
-                    switch (mode) {
-                        case kMaskNone: mx = row_max64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, mx); break;
-                        case kMaskLo: mx = row_max64<kMaskLo>(v, 64 * hlf, c_lo, c_hi, mx); break;
-                        case kMaskHi: mx = row_max64<kMaskHi>(v, 64 * hlf, c_lo, c_hi, mx); break;
-                        default: mx = row_max64<kMaskBoth>(v, 64 * hlf, c_lo, c_hi, mx); break;
+                    for (int hlf = 0; hlf < 2; ++hlf) {
+                        uint32_t v[64];
+                        tmem_ld32(tm_s + 64 * hlf, v);
+                        tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
+                        tmem_wait_ld();
+                        regs_after_wait(v);
+                        regs_after_wait(v + 32);
+                        mx = row_max64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, mx);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        const int cls = chunk_class(c);
+                        if (cls == 4) continue;
+                        uint32_t v[32];
+                        tmem_ld32(tm_s + 32 * c, v);
+                        tmem_wait_ld();
+                        regs_after_wait(v);
+                        switch (cls) {
+                            case kMaskNone: mx = row_max32<kMaskNone>(v, 32 * c, c_lo, c_hi, mx); break;
+                            case kMaskLo: mx = row_max32<kMaskLo>(v, 32 * c, c_lo, c_hi, mx); break;
+                            case kMaskHi: mx = row_max32<kMaskHi>(v, 32 * c, c_lo, c_hi, mx); break;
+                            default: mx = row_max32<kMaskBoth>(v, 32 * c, c_lo, c_hi, mx); break;
+                        }
                     }
                 }
                 const float m_new = fmaxf(m, mx * scale_log2);
@@ -433,24 +492,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (rescale) m = m_new;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const uint64_t negm2 = f32x2(neg_m, neg_m);
-                // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first half of S
+                // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first half of S (packed
+                // words of 32 columns go to 16 columns, all of them already read in this pass)
                 uint64_t sum2 = f32x2(0.f, 0.f);
+                if (full_tile) {
 #pragma unroll 1
-                for (int hlf = 0; hlf < 2; ++hlf) {
-                    uint32_t v[64];
-                    tmem_ld32(tm_s + 64 * hlf, v);
-                    tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
-                    tmem_wait_ld();
-                    regs_after_wait(v);
-                    regs_after_wait(v + 32);
-                    uint32_t pk[32];
-                    switch (mode) {
-                        case kMaskNone: sum2 = row_exp64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                        case kMaskLo: sum2 = row_exp64<kMaskLo>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                        case kMaskHi: sum2 = row_exp64<kMaskHi>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                        default: sum2 = row_exp64<kMaskBoth>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                    for (int hlf = 0; hlf < 2; ++hlf) {
+                        uint32_t v[64];
+                        tmem_ld32(tm_s + 64 * hlf, v);
+                        tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
+                        tmem_wait_ld();
+                        regs_after_wait(v);
+                        regs_after_wait(v + 32);
+                        uint32_t pk[32];
+                        sum2 = row_exp64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk);
+                        tmem_st32(tm_s + 32 * hlf, pk);
                     }
-                    tmem_st32(tm_s + 32 * hlf, pk);
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        const int cls = chunk_class(c);
+                        uint32_t pk[16];
+                        if (cls == 4) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                        } else {
+                            uint32_t v[32];
+                            tmem_ld32(tm_s + 32 * c, v);
+                            tmem_wait_ld();
+                            regs_after_wait(v);
+                            switch (cls) {
+                                case kMaskNone: sum2 = row_exp32<kMaskNone>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                                case kMaskLo: sum2 = row_exp32<kMaskLo>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                                case kMaskHi: sum2 = row_exp32<kMaskHi>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                                default: sum2 = row_exp32<kMaskBoth>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
+                            }
+                        }
+                        tmem_st16(tm_s + 16 * c, pk);
+                    }
                 }
                 float s_lo, s_hi;
                 f32x2_split(sum2, s_lo, s_hi);
