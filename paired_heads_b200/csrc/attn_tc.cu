@@ -218,7 +218,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 8 && lane == 0) {
         for (int s = 0; s < 3; ++s) {
             mbar_init(&bars->q_full[s], 1);
-            mbar_init(&bars->q_empty[s], 1);
+            // freed by the MMA thread's commit after the sub-tile's last S and by the 4 warps of
+            // its softmax warpgroup after the epilogue has staged O through the slot
+            mbar_init(&bars->q_empty[s], 5);
         }
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars->k_full[s], 1);
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint64_t scale2 = f32x2(scale_log2, scale_log2);
         const int window = p.window;
         uint32_t s_cnt = 0, o_cnt = 0;
+        uint32_t q_seq = 0;  // index of the current item's first Q sub-tile in this CTA's stream
         bool ok = true;
         int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
@@ -417,6 +420,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int nr = r ? it.nr[1] : it.nr[0];
             const int t_first = r ? it.t_first[1] : it.t_first[0];
             const int t_last = r ? it.t_last[1] : it.t_last[0];
+            const uint32_t my_q = q_seq + r;
+            q_seq += it.n_sub;
             if (nr == 0) continue;
             const int qr0 = it.q0 + kBlockM * r;
             const int i = qr0 + row;
@@ -559,27 +564,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const bool valid = row < nr;
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
-                                  (static_cast<int64_t>(i) * H + it.head) * HD;
+            // O / l -> bf16, staged through this sub-tile's Q slot (its last S has completed):
+            // each warp writes its 32 rows with an XOR swizzle of the 16-byte chunks, then copies
+            // them out two rows per instruction, so every global store of the warp covers 512
+            // contiguous bytes. Rows past the end of the document are not written.
+            constexpr int kChunks = HD / 8;  // 16-byte chunks per row
+            uint8_t* stage = smem + L::kOffQ + (my_q % L::kQSlots) * L::kQSub + (warp & 3) * 32 * (HD * 2);
+            const int wrow = row & 31;
 #pragma unroll 1
             for (int c = 0; c < HD / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tm_o + 32 * c, v);
                 tmem_wait_ld();
                 regs_after_wait(v);
-                if (valid) {
-                    uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv_l,
-                                            __uint_as_float(v[2 * e + 1]) * inv_l);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-                    dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint4 w4 = make_uint4(
+                        pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv_l, __uint_as_float(v[8 * q4 + 1]) * inv_l),
+                        pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv_l, __uint_as_float(v[8 * q4 + 3]) * inv_l),
+                        pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv_l, __uint_as_float(v[8 * q4 + 5]) * inv_l),
+                        pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv_l, __uint_as_float(v[8 * q4 + 7]) * inv_l));
+                    const int chunk = 4 * c + q4;
+                    *reinterpret_cast<uint4*>(stage + wrow * (HD * 2) + ((chunk ^ (wrow & (kChunks - 1))) << 4)) = w4;
                 }
             }
+            __syncwarp();
+            {
+                const int row0 = qr0 + (warp & 3) * 32;  // first slot of this warp's rows
+                constexpr int kRowsPerIter = 32 / kChunks;
+#pragma unroll 4
+                for (int j = 0; j < 32 / kRowsPerIter; ++j) {
+                    const int rl = j * kRowsPerIter + lane / kChunks;
+                    const int chunk = lane % kChunks;
+                    if ((warp & 3) * 32 + rl < nr) {
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(
+                            stage + rl * (HD * 2) + ((chunk ^ (rl & (kChunks - 1))) << 4));
+                        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) +
+                                             (static_cast<int64_t>(row0 + rl) * H + it.head) * HD + chunk * 8;
+                        *reinterpret_cast<uint4*>(dst) = w4;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->q_empty[my_q % L::kQSlots]);
             tc_fence_before();
             if (valid && p.lse) p.lse[static_cast<int64_t>(i) * H + it.head] = (m + log2f(l)) * kLn2;
         }
