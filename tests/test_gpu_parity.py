@@ -149,6 +149,14 @@ ATTN_CASES = [
     ((250, 130), 4, 2, 128, False, 0, True),
     ((2000,), 2, 2, 128, True, 300, True),
     ((0, 77, 0, 0, 190), 2, 1, 64, True, 0, False),
+    # windows around the 32-column chunk boundaries of the masked-tile path
+    ((600, 257), 4, 4, 128, True, 31, False),
+    ((600, 257), 4, 4, 64, True, 33, True),
+    ((500, 3), 2, 2, 128, True, 63, True),
+    ((500, 3), 2, 2, 64, True, 65, False),
+    ((900,), 4, 2, 128, True, 96, True),
+    ((900,), 4, 2, 64, True, 129, False),
+    ((1100, 130), 6, 6, 128, True, 257, True),
 ]
 
 
