@@ -137,7 +137,7 @@ struct Chunk16<float> {
 // every load instruction of the warp reads 512 contiguous bytes and each lane keeps kBatch x 16
 // bytes of HBM reads in flight. All heads of the token share its table row, which is read from
 // HBM once and then served from L1.
-constexpr int kRopeBatch = 8;
+constexpr int kRopeBatch = 4;
 
 template <typename T>
 __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restrict__ k,
