@@ -41,57 +41,10 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "attn_common.cuh"
 #include "kernels.cuh"
 
 namespace pha {
-
-template <int HD>
-struct TcLayout {
-    static constexpr int kChunk = 128 * 128;  // one [128 rows][64 bf16] swizzled chunk (bytes)
-    static constexpr int kQSub = kBlockM * HD * 2;
-    static constexpr int kKV = kBlockN * HD * 2;
-    static constexpr int kQSlots = 3;
-    static constexpr int kKStages = HD == 128 ? 2 : 4;
-    static constexpr int kVStages = HD == 128 ? 2 : 4;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQSlots * kQSub;
-    static constexpr int kOffV = kOffK + kKStages * kKV;
-    static constexpr int kOffBar = kOffV + kVStages * kKV;
-    static constexpr int kBarBytes = 512;
-    static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + slack to align to 1024
-    static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kTmO = 256;
-    static_assert(kSmemBytes <= 232448, "shared memory budget");
-};
-
-struct TcBars {
-    uint64_t q_full[3], q_empty[3];
-    uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-    uint64_t s_full[2], p_full[2], pv_done[2], o_ready[2];
-    uint64_t drain;
-    uint32_t tmem_base;
-    int abort;
-};
-
-constexpr int kTcThreads = 320;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-
-// Drain wait used on the exit path: bounded, ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_test(bar, parity))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
-
-// K-major 128-row tile (Q or K): k-step kk covers 16 bf16 of the contraction dimension.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
-    return smem_desc_sw128(tile + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-}
-// MN-major V tile ([keys][hd] in 64-column chunks): k-step kk covers 16 keys.
-__device__ __forceinline__ uint64_t desc_v(uint32_t tile, int kk) {
-    return smem_desc_sw128(tile + kk * 2048, 16384, 1024);
-}
 
 // A decoded work item and the per-sub-tile key ranges (identical in every role).
 struct Item {
@@ -124,78 +77,6 @@ __device__ __forceinline__ Item decode_item(int4 w, const AttnProblem& p) {
         it.t_last[r] = nr > 0 ? (hi - 1 - it.kv_lo) / kBlockN : -1;
     }
     return it;
-}
-
-// Mask modes of one (sub-tile, key tile): which column bounds some row of the tile needs.
-enum : int { kMaskNone = 0, kMaskLo = 1, kMaskHi = 2, kMaskBoth = 3 };
-
-template <int MODE>
-__device__ __forceinline__ float mask_col(float s, int c, int c_lo, int c_hi) {
-    if (MODE & kMaskLo) s = c < c_lo ? -INFINITY : s;
-    if (MODE & kMaskHi) s = c > c_hi ? -INFINITY : s;
-    return s;
-}
-
-// Pass 1 over 32 columns starting at `base`: running max of the visible scores.
-template <int MODE>
-__device__ __forceinline__ float row_max32(const uint32_t* v, int base, int c_lo, int c_hi, float mx) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
-        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
-        mx = fmax3(mx, a, b);
-    }
-    return mx;
-}
-
-// Pass 2 over 32 columns: 16 packed bf16 pairs of p = 2^(s * scale_log2 - m), 0 where masked.
-template <int MODE>
-__device__ __forceinline__ uint64_t row_exp32(const uint32_t* v, int base, int c_lo, int c_hi,
-                                              uint64_t scale2, uint64_t negm2, uint64_t sum2,
-                                              uint32_t* pk) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
-        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
-        float xa, xb;
-        f32x2_split(fma_f32x2(f32x2(a, b), scale2, negm2), xa, xb);
-        const float pa = ex2(xa), pb = ex2(xb);
-        sum2 = add_f32x2(sum2, f32x2(pa, pb));
-        pk[e >> 1] = pack_bf16x2(pa, pb);
-    }
-    return sum2;
-}
-
-// Pass 1 over 64 columns starting at `base`: running max of the visible scores.
-template <int MODE>
-__device__ __forceinline__ float row_max64(const uint32_t* v, int base, int c_lo, int c_hi,
-                                           float mx) {
-#pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
-        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
-        mx = fmax3(mx, a, b);
-    }
-    return mx;
-}
-
-// Pass 2 over 64 columns: p = 2^(s * scale_log2 - m) for the visible scores (0 elsewhere),
-// packed into 32 bf16 pairs; returns the (two-lane) partial row sum.
-template <int MODE>
-__device__ __forceinline__ uint64_t row_exp64(const uint32_t* v, int base, int c_lo, int c_hi,
-                                              uint64_t scale2, uint64_t negm2, uint64_t sum2,
-                                              uint32_t* pk) {
-#pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-        const float a = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
-        const float b = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
-        float xa, xb;
-        f32x2_split(fma_f32x2(f32x2(a, b), scale2, negm2), xa, xb);
-        const float pa = ex2(xa), pb = ex2(xb);
-        sum2 = add_f32x2(sum2, f32x2(pa, pb));
-        pk[e >> 1] = pack_bf16x2(pa, pb);
-    }
-    return sum2;
 }
 
 template <int HD>
