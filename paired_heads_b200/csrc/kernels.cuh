@@ -11,7 +11,10 @@ namespace pha {
 
 constexpr int kBlockM = 128;         // query rows per sub-tile (one softmax warpgroup)
 constexpr int kBlockN = 128;         // key slots per tile
-constexpr int kItemRows = 2 * kBlockM;  // query slots per work item
+constexpr int kItemRows = 2 * kBlockM;  // query slots per block work item (attn_tc)
+constexpr int kBandTiles = 8;            // query tiles per band work item (attn_band)
+constexpr int kBandRows = kBandTiles * kBlockM;
+static_assert(kBandRows >= kItemRows, "band items must not outnumber block items");
 constexpr int kMaxCostBuckets = 4096;   // scheduler cost classes (longest-first ordering)
 
 // Workspace: header (bytes [0, 256)), per-document block offsets (int32[batch + 1], padded to 16
@@ -26,9 +29,12 @@ inline size_t workspace_doc_bytes(int batch) {
     return (static_cast<size_t>(batch + 1) * sizeof(int) + 15) & ~static_cast<size_t>(15);
 }
 
-// One work item = one block of up to kItemRows query slots of one head:
+// Block work item (attn_tc) = one block of up to kItemRows query slots of one head:
 //   x = first query slot, y = (head << 16) | valid query rows, z = first key slot, w = key end.
 // Keys [z, w) are streamed in tiles of kBlockN starting at z.
+// Band work item (attn_band) = a run of up to kBandTiles query tiles of one head:
+//   x = first query slot q0, y = (head << 16) | (has_prev << 15) | query tiles, z = document end.
+// Key tiles start at q0 - kBlockN (has_prev) or q0, one per step.
 
 struct AttnProblem {
     const void* q;
@@ -59,10 +65,10 @@ cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin
 
 cudaError_t launch_attn_f32(const AttnProblem& p, cudaStream_t stream);
 
-// Builds the varlen work list into `items` (capacity entries) and the header; doc_blocks is
-// int32[batch + 1] scratch.
-cudaError_t launch_schedule(const AttnProblem& p, int capacity, int* doc_blocks, int4* items,
-                            WorkspaceHeader* hdr, cudaStream_t stream);
+// Builds the varlen work list (band items when `band`, else block items) into `items` (capacity
+// entries) and the header; doc_blocks is int32[batch + 1] scratch.
+cudaError_t launch_schedule(const AttnProblem& p, bool band, int capacity, int* doc_blocks,
+                            int4* items, WorkspaceHeader* hdr, cudaStream_t stream);
 
 // tcgen05 attention over a scheduled work list. tm_q / tm_k / tm_v are 2-D bf16 tensor maps
 // over the slot view ([slots][heads * head_dim] and [slots][kv_heads * head_dim]) with a
@@ -70,5 +76,15 @@ cudaError_t launch_schedule(const AttnProblem& p, int capacity, int* doc_blocks,
 cudaError_t launch_attn_tc(const AttnProblem& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const int4* items, WorkspaceHeader* hdr,
                            cudaStream_t stream);
+
+// True when the band kernel covers the problem: causal, 1 <= window <= kBlockN.
+inline bool band_applies(const AttnProblem& p) {
+    return p.causal && p.window >= 1 && p.window <= kBlockN;
+}
+
+// tcgen05 attention over a band work list (same tensor maps as launch_attn_tc).
+cudaError_t launch_attn_band(const AttnProblem& p, const CUtensorMap& tm_q,
+                             const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int4* items,
+                             WorkspaceHeader* hdr, cudaStream_t stream);
 
 }  // namespace pha

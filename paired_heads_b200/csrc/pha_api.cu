@@ -162,7 +162,10 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
     auto* doc_blocks = reinterpret_cast<int*>(base + kWorkspaceHeaderBytes);
     auto* items = reinterpret_cast<int4*>(base + fixed);
 
-    if (launch_schedule(p, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+    // Causal windows of at most one key tile run on the band kernel, everything else on the block
+    // kernel; the scheduler emits the matching item shape.
+    const bool band = band_applies(p);
+    if (launch_schedule(p, band, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
         return PHA_ERR_CUDA;
     if (total_tokens == 0) return PHA_OK;
 
@@ -172,7 +175,9 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
         !encode_slot_map(&tk, k, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
         !encode_slot_map(&tv, v, static_cast<uint64_t>(p.kv_heads) * head_dim, rows))
         return PHA_ERR_CUDA;
-    return launch_attn_tc(p, tq, tk, tv, items, hdr, stream) == cudaSuccess ? PHA_OK : PHA_ERR_CUDA;
+    const cudaError_t e = band ? launch_attn_band(p, tq, tk, tv, items, hdr, stream)
+                               : launch_attn_tc(p, tq, tk, tv, items, hdr, stream);
+    return e == cudaSuccess ? PHA_OK : PHA_ERR_CUDA;
 }
 
 pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream) {

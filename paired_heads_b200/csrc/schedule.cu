@@ -2,13 +2,21 @@
 //
 // Paired path: document boundaries and max_len are doubled ("modded-nanogpt Paired Head
 // Attention record" page, section "sequence length and window handling") while the window stays
-// as given. A work item is a block of up to kItemRows = 256 query slots [q0, q0+n) of one
+// as given. Two item shapes, one per attention kernel:
+//
+// Block items (attn_tc.cu): a block of up to kItemRows = 256 query slots [q0, q0+n) of one
 // document [a, b) and one head; its key range is
 //   causal:      [max(a, q0 - window + 1), q0 + n)   (window <= 0: from a)
 //   non-causal:  [a, b)
 // so key tiles that the causal mask or the window hide from the whole block are never scheduled
 // (the attention kernel further skips, per 128-row half of the block, the tiles that half cannot
 // see). Key tiles start at the range's first slot, not at a multiple of 128.
+//
+// Band items (attn_band.cu, causal with 1 <= window <= 128): a run of up to kBandTiles query
+// tiles of 128 slots, tile u = [q0 + 128u, q0 + 128u + 128) of one document and one head, tiles
+// counted from the document start. Such a query tile sees at most the key tile at its own start
+// and the one before it, so the run streams key tiles from q0 - 128 (q0 - 128 >= a, "has
+// previous") or q0, one per step, each shared by two consecutive query tiles.
 //
 // Items are ordered longest first (counting sort on the number of key tiles) so that a static
 // round-robin over persistent CTAs balances; the heads of one block are adjacent so that CTAs
@@ -56,31 +64,38 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
 }
 
 struct BlockRange {
-    int q0, n_q, kv_lo, kv_hi, cost;
+    int4 item;  // the encoded work item (head field left 0)
+    int cost;   // key tiles streamed, clamped to the last bucket
 };
 
 __device__ __forceinline__ BlockRange block_range(const AttnProblem& p, int64_t a, int64_t b,
-                                                  int blk, int n_buckets) {
+                                                  int blk, int n_buckets, bool band) {
     BlockRange r;
-    const int64_t q0 = a + static_cast<int64_t>(blk) * kItemRows;
-    const int64_t n_q = b - q0 < kItemRows ? b - q0 : kItemRows;
-    int64_t lo = a, hi = b;
-    if (p.causal) {
-        hi = q0 + n_q;
-        if (p.window > 0 && q0 - p.window + 1 > a) lo = q0 - p.window + 1;
+    const int rows = band ? kBandRows : kItemRows;
+    const int64_t q0 = a + static_cast<int64_t>(blk) * rows;
+    const int64_t n_q = b - q0 < rows ? b - q0 : rows;
+    int64_t cost;
+    if (band) {
+        const int n_qt = static_cast<int>((n_q + kBlockM - 1) / kBlockM);
+        const int hp = blk > 0 ? 1 : 0;
+        cost = n_qt + hp;
+        r.item = make_int4(static_cast<int>(q0), (hp << 15) | n_qt, static_cast<int>(b), 0);
+    } else {
+        int64_t lo = a, hi = b;
+        if (p.causal) {
+            hi = q0 + n_q;
+            if (p.window > 0 && q0 - p.window + 1 > a) lo = q0 - p.window + 1;
+        }
+        cost = (hi - lo + kBlockN - 1) / kBlockN;
+        r.item = make_int4(static_cast<int>(q0), static_cast<int>(n_q), static_cast<int>(lo),
+                           static_cast<int>(hi));
     }
-    int64_t cost = (hi - lo + kBlockN - 1) / kBlockN;
-    if (cost >= n_buckets) cost = n_buckets - 1;
-    r.q0 = static_cast<int>(q0);
-    r.n_q = static_cast<int>(n_q);
-    r.kv_lo = static_cast<int>(lo);
-    r.kv_hi = static_cast<int>(hi);
-    r.cost = static_cast<int>(cost);
+    r.cost = static_cast<int>(cost >= n_buckets ? n_buckets - 1 : cost);
     return r;
 }
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, int capacity,
-                                                                 int n_buckets,
+                                                                 int n_buckets, int band,
                                                                  int* __restrict__ doc_blocks,
                                                                  int4* __restrict__ items,
                                                                  WorkspaceHeader* hdr) {
@@ -89,6 +104,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     __shared__ int bad;
     const int tid = threadIdx.x;
     const int64_t mult = p.slot_mult;
+    const int rows = band ? kBandRows : kItemRows;
     for (int c = tid; c < n_buckets; c += kSchedThreads) hist[c] = 0;
     if (tid == 0) bad = 0;
     __syncthreads();
@@ -100,7 +116,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
         if (a0 < 0 || b0 < a0 || b0 > p.total_tokens || b0 - a0 > p.max_len)
             atomicOr(&bad, 1);
         else
-            nb = static_cast<int>(((b0 - a0) * mult + kItemRows - 1) / kItemRows);
+            nb = static_cast<int>(((b0 - a0) * mult + rows - 1) / rows);
         doc_blocks[d] = nb;
     }
     __syncthreads();
@@ -146,7 +162,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     for (int g = tid; g < n_blocks; g += kSchedThreads) {
         const int d = doc_of(g);
         const BlockRange r = block_range(p, p.cu_seqlens[d] * mult, p.cu_seqlens[d + 1] * mult,
-                                         g - doc_blocks[d], n_buckets);
+                                         g - doc_blocks[d], n_buckets, band);
         atomicAdd(&hist[r.cost], 1);
     }
     __syncthreads();
@@ -165,11 +181,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     for (int g = tid; g < n_blocks; g += kSchedThreads) {
         const int d = doc_of(g);
         const BlockRange r = block_range(p, p.cu_seqlens[d] * mult, p.cu_seqlens[d + 1] * mult,
-                                         g - doc_blocks[d], n_buckets);
+                                         g - doc_blocks[d], n_buckets, band);
         const int slot = atomicAdd(&hist[r.cost], 1);
         int4* dst = items + static_cast<int64_t>(slot) * p.heads;
         for (int h = 0; h < p.heads; ++h)
-            dst[h] = make_int4(r.q0, (h << 16) | r.n_q, r.kv_lo, r.kv_hi);
+            dst[h] = make_int4(r.item.x, (h << 16) | r.item.y, r.item.z, r.item.w);
     }
     if (tid == 0) {
         hdr->n_items = static_cast<int>(n_items);
@@ -177,16 +193,17 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     }
 }
 
-int schedule_buckets(const AttnProblem& p) {
+int schedule_buckets(const AttnProblem& p, bool band) {
+    if (band) return kBandTiles + 2;
     const int64_t slots = static_cast<int64_t>(p.max_len) * p.slot_mult;
     const int64_t nb = (slots + kItemRows) / kBlockN + 2;
     return static_cast<int>(nb < kMaxCostBuckets ? nb : kMaxCostBuckets);
 }
 
-cudaError_t launch_schedule(const AttnProblem& p, int capacity, int* doc_blocks, int4* items,
-                            WorkspaceHeader* hdr, cudaStream_t stream) {
-    schedule_kernel<<<1, kSchedThreads, 0, stream>>>(p, capacity, schedule_buckets(p), doc_blocks,
-                                                     items, hdr);
+cudaError_t launch_schedule(const AttnProblem& p, bool band, int capacity, int* doc_blocks,
+                            int4* items, WorkspaceHeader* hdr, cudaStream_t stream) {
+    schedule_kernel<<<1, kSchedThreads, 0, stream>>>(p, capacity, schedule_buckets(p, band),
+                                                     band ? 1 : 0, doc_blocks, items, hdr);
     return cudaGetLastError();
 }
 

@@ -157,6 +157,12 @@ ATTN_CASES = [
     ((900,), 4, 2, 128, True, 96, True),
     ((900,), 4, 2, 64, True, 129, False),
     ((1100, 130), 6, 6, 128, True, 257, True),
+    # band kernel (causal, window <= 128): runs of 8 query tiles (1024 slots) with exact and
+    # one-row-over chunk boundaries, single-tile documents, the smallest windows, GQA
+    ((512, 513, 64, 1, 2049), 4, 2, 128, True, 128, True),
+    ((1024, 1025, 127, 129, 1), 2, 2, 64, True, 2, False),
+    ((3000, 7), 8, 2, 128, True, 100, False),
+    ((128, 256, 2176), 2, 2, 128, True, 128, False),
 ]
 
 
