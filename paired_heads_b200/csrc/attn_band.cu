@@ -376,6 +376,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     // Keep the reference max until the row max grows by more than 8 (a factor
                     // 256): O / l and the lse are exact for any reference value.
                     const bool rescale = m_new > m + 8.0f;
+                    const bool o_nonzero = m != -INFINITY;  // some key seen: O may be nonzero
                     const float alpha = rescale ? ex2(m - m_new) : 1.0f;
                     if (rescale) m = m_new;
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
@@ -406,7 +407,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     float s_lo, s_hi;
                     f32x2_split(sum2, s_lo, s_hi);
                     l = l * alpha + (s_lo + s_hi);
-                    if (t > 0 && __any_sync(0xffffffffu, rescale)) {
+                    if (t > 0 && __any_sync(0xffffffffu, rescale && o_nonzero)) {
 #pragma unroll 1
                         for (int c = 0; c < HD / 32; ++c) {
                             uint32_t v[32];
