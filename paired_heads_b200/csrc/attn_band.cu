@@ -475,6 +475,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     }
                 }
                 __syncwarp();
+                fence_proxy_async_smem();  // the slot's next fill is written by the async proxy (TMA)
                 if (lane == 0) mbar_arrive(&bars->q_empty[n % L::kQSlots]);
                 tc_fence_before();
                 if (row < nr && p.lse)

@@ -487,6 +487,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             __syncwarp();
+            fence_proxy_async_smem();  // the slot's next fill is written by the async proxy (TMA)
             if (lane == 0) mbar_arrive(&bars->q_empty[my_q % L::kQSlots]);
             tc_fence_before();
             if (valid && p.lse) p.lse[static_cast<int64_t>(i) * H + it.head] = (m + log2f(l)) * kLn2;
