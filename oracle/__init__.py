@@ -59,7 +59,8 @@ def _load():
                                               _d, _i64p, _l, _f64p, _f64p]
         lib.oracle_attn_fwd.argtypes = [_f64p, _f64p, _f64p, _i32p, _c, _c, _c, _c, _c, _c, _c,
                                         _d, _f64p, _f64p]
-        for f in ("oracle_rope", "oracle_round_bf16", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
+        lib.oracle_rms_norm.argtypes = [_f64p, _l, _c, ctypes.c_void_p, _d]
+        for f in ("oracle_rms_norm", "oracle_rope", "oracle_round_bf16", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
                   "oracle_attention_rows", "oracle_attn_fwd"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -102,6 +103,35 @@ def rope_stored(x, positions, dtype: str, paired: bool = False, stagger: bool = 
     float64, result rounded to the buffer's dtype ("bf16": nearest bfloat16; "f32": nearest
     float32)."""
     y = rope(x, positions, paired, stagger, base, table_f32=True)
+    if dtype == "bf16":
+        return round_bf16(y)
+    return y.astype(np.float32).astype(np.float64)
+
+
+def rms_norm(x, gamma=None, eps: float = 1e-6):
+    """RMS normalisation over the last axis of x (returns a new float64 array); gamma: per-element
+    weights of that axis, or None for ones ("Training an LLM from scratch (part 2)", section
+    "1. RMSNorm")."""
+    y = _f64(x).copy()
+    d = y.shape[-1]
+    g = None if gamma is None else _f64(gamma).reshape(d).copy()
+    _check(_load().oracle_rms_norm(y.reshape(-1), y.size // d, d,
+                                   None if g is None else g.ctypes.data, float(eps)), "rms_norm")
+    return y
+
+
+def norm_rope_stored(x, positions, dtype: str, paired: bool = False, stagger: bool = False,
+                     base: float = 10000.0, gamma=None, eps: float = 1e-6, tab_rows=None):
+    """QK RMS-norm of each head row, then RoPE with float32 table values, rounded once to the
+    buffer's dtype. Tokens whose position lies outside [0, tab_rows) are normalised but not
+    rotated."""
+    n = rms_norm(x, gamma, eps)
+    pos = np.ascontiguousarray(positions, dtype=np.int64)
+    safe = np.clip(pos, 0, None).astype(np.int32)
+    y = rope(n, safe, paired, stagger, base, table_f32=True)
+    if tab_rows is not None:
+        out = (pos < 0) | (pos >= tab_rows)
+        y[out] = n[out]
     if dtype == "bf16":
         return round_bf16(y)
     return y.astype(np.float32).astype(np.float64)

@@ -20,6 +20,9 @@
  *   [MASK] "ChatGPT" source notes (ranhao.site), section "SingleHeadAttention": lower-triangular
  *          causal mask, logits divided by sqrt(head_size), softmax over keys, weights times V.
  *   [SOFT] "mHC module" (lshu.cn/news/67890): softmax stabilised by subtracting the row max.
+ *   [RMS]  "Training an LLM from scratch (part 2)", section "1. RMSNorm": y = x / sqrt(E[x^2] + eps)
+ *          * gamma over the last dimension; [PHA] "4. interleave index in the Triton kernel": the
+ *          rotary kernel also applies the QK RMS-norm (to each head row of q and k).
  *
  * Readings where the pages are silent or ambiguous (each is listed in the design notes):
  *   - rotation acts on adjacent pairs (x[2i], x[2i+1]) -- the [PHA] flip of a (..., D/2, 2) view;
@@ -82,6 +85,23 @@ int oracle_rope(double* x, const int32_t* pos, int64_t n_tok, int n_head, int hd
                 row[2 * i + 1] = a * s + b * c;
             }
         }
+    }
+    return ORACLE_OK;
+}
+
+/* RMS normalisation of each of the n_rows rows of x[n_rows][d] (in place), [RMS]:
+ * y_j = x_j / sqrt((1/d) sum_k x_k^2 + eps) * gamma_j; gamma == NULL stands for all ones. */
+int oracle_rms_norm(double* x, int64_t n_rows, int d, const double* gamma, double eps)
+{
+    if (!x || n_rows < 0 || d <= 0 || !(eps >= 0.0)) return ORACLE_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        double* row = x + (size_t)r * (size_t)d;
+        double ms = 0.0;
+        for (int j = 0; j < d; ++j) ms += row[j] * row[j];
+        ms /= (double)d;
+        double scale = 1.0 / sqrt(ms + eps);
+        for (int j = 0; j < d; ++j) row[j] = row[j] * scale * (gamma ? gamma[j] : 1.0);
     }
     return ORACLE_OK;
 }

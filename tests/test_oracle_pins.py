@@ -416,3 +416,70 @@ def test_float32_tables_only_perturb_by_float32_rounding():
         pair = np.abs(x.reshape(200, 4, 32, 2)).sum(-1).repeat(2, axis=-1)
         assert np.all(np.abs(a - b) <= 2.0 ** -24 * pair * 1.0001)
         assert np.any(a != b)
+
+
+# ------------------------------------------------------------------------------ QK RMS-norm
+# "Training an LLM from scratch (part 2)", section "1. RMSNorm": y = x / sqrt(E[x^2] + eps) * gamma
+# over the last axis; the paired-head page's rotary kernel applies it to each head row of q and k.
+
+def test_rms_norm_matches_torch_float64():
+    import torch
+
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((7, 5, 64)) * rng.uniform(0.1, 9.0, (7, 5, 1))
+    g = rng.uniform(0.5, 2.0, 64)
+    for gamma, eps in ((None, 1e-6), (g, 1e-6), (g, 0.3)):
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,),
+                                           None if gamma is None else torch.from_numpy(gamma), eps)
+        np.testing.assert_allclose(oracle.rms_norm(x, gamma, eps), ref.numpy(), rtol=1e-14, atol=0)
+
+
+def test_rms_norm_gives_unit_rms_rows_and_keeps_direction():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((6, 4, 32)) * np.arange(1, 25).reshape(6, 4, 1)  # rows of every scale
+    y = oracle.rms_norm(x, eps=0.0)
+    np.testing.assert_allclose(np.sqrt((y ** 2).mean(-1)), 1.0, rtol=1e-14)  # each row on its own
+    cos = (x * y).sum(-1) / np.linalg.norm(x, axis=-1) / np.linalg.norm(y, axis=-1)
+    np.testing.assert_allclose(cos, 1.0, rtol=1e-14)
+    # with eps the mean square is ms / (ms + eps)
+    ms = (x ** 2).mean(-1)
+    y = oracle.rms_norm(x, eps=0.5)
+    np.testing.assert_allclose((y ** 2).mean(-1), ms / (ms + 0.5), rtol=1e-13)
+
+
+def test_rms_norm_scale_and_sign_invariance_and_weights():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((3, 2, 16))
+    g = rng.uniform(-2.0, 2.0, 16)
+    base = oracle.rms_norm(x, eps=0.0)
+    np.testing.assert_allclose(oracle.rms_norm(37.5 * x, eps=0.0), base, rtol=1e-14)
+    np.testing.assert_allclose(oracle.rms_norm(-x, eps=0.0), -base, rtol=1e-14)
+    np.testing.assert_allclose(oracle.rms_norm(x, g, eps=0.0), base * g, rtol=1e-14)
+    # a constant row c becomes c / sqrt(c^2 + eps)
+    c = np.full((1, 1, 8), -3.0)
+    np.testing.assert_allclose(oracle.rms_norm(c, eps=7.0), -3.0 / 4.0, rtol=1e-15)
+
+
+def test_norm_then_rope_keeps_the_normalised_length():
+    # the rotation is orthogonal: after the norm each head row has length sqrt(hd) (eps = 0)
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((9, 6, 128)) * 5.0
+    pos = rng.integers(0, 1000, 9).astype(np.int32)
+    y = oracle.rope(oracle.rms_norm(x, eps=0.0), pos, paired=True, stagger=True)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.sqrt(128.0), rtol=1e-13)
+
+
+def test_norm_rope_stored_skips_rotation_outside_the_table():
+    rng = np.random.default_rng(15)
+    x = synth_bf16(rng.standard_normal((4, 2, 16)))
+    pos = np.array([0, -1, 5, 99], dtype=np.int32)
+    y = oracle.norm_rope_stored(x, pos, "bf16", eps=1e-6, tab_rows=10)
+    n = oracle.round_bf16(oracle.rms_norm(x, eps=1e-6))
+    np.testing.assert_array_equal(y[1], n[1])   # position -1: normalised, not rotated
+    np.testing.assert_array_equal(y[3], n[3])   # position 99 >= 10 rows
+    np.testing.assert_array_equal(y[0], n[0])   # position 0: rotation by 0
+    assert not np.array_equal(y[2], n[2])       # position 5: rotated
+
+
+def synth_bf16(x):
+    return oracle.round_bf16(x)
