@@ -2,7 +2,10 @@
 inputs resident in HBM. Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--window W]
-                    [--paired 0|1] [--impl reference]
+                    [--paired 0|1] [--qk-norm] [--impl reference]
+
+--qk-norm replaces pha_rope with pha_qk_norm_rope (the QK RMS-norm of every head row, then RoPE,
+in one kernel).
 
 Default workload: the paired-head varlen packed batch (65,536 tokens, documents ~ geometric(512)
 capped at 2048, 6 heads -> 3 pairs, head_dim 128, bf16, causal, window 128 slots, staggered
@@ -150,7 +153,7 @@ def oracle_sample(w, budget_tokens: int):
     return w.with_(doc_lens=tuple(lens))
 
 
-def time_oracle(w, budget_tokens: int):
+def time_oracle(w, budget_tokens: int, qk_norm: bool = False):
     """Oracle (float64 C) run of one step (RoPE stored in the buffer dtype + attention) on a
     bounded sample of the workload. Returns (TFLOP/s, seconds, sample workload, threads)."""
     import oracle
@@ -160,8 +163,12 @@ def time_oracle(w, budget_tokens: int):
     q, k, v = (synth.to_f64(inp[n]) for n in ("q", "k", "v"))
     pos = inp["positions"].numpy()
     t0 = time.perf_counter()
-    qr = oracle.rope_stored(q, pos, w.dtype, w.paired, w.stagger, w.rope_base)
-    kr = oracle.rope_stored(k, pos, w.dtype, w.paired, w.stagger, w.rope_base)
+    if qk_norm:
+        qr = oracle.norm_rope_stored(q, pos, w.dtype, w.paired, w.stagger, w.rope_base)
+        kr = oracle.norm_rope_stored(k, pos, w.dtype, w.paired, w.stagger, w.rope_base)
+    else:
+        qr = oracle.rope_stored(q, pos, w.dtype, w.paired, w.stagger, w.rope_base)
+        kr = oracle.rope_stored(k, pos, w.dtype, w.paired, w.stagger, w.rope_base)
     oracle.attn_fwd(qr, kr, v, inp["cu_seqlens"].numpy(), w.causal, w.window, w.paired, w.scale)
     dt = time.perf_counter() - t0
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
@@ -180,6 +187,8 @@ def main():
     ap.add_argument("--paired", type=int, default=None)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qk-norm", action="store_true",
+                    help="QK RMS-norm + RoPE (pha_qk_norm_rope) instead of RoPE alone")
     ap.add_argument("--oracle-tokens", type=int, default=16384)
     args = ap.parse_args()
     w = pick_workload(args)
@@ -206,8 +215,14 @@ def main():
     step = AttentionStep(StepShape.of(w, tab_rows), dev)
     stream = torch.cuda.current_stream(dev)
 
+    def rotary(qq, kk, pp):
+        if args.qk_norm:
+            step.norm_rope(qq, kk, pp)
+        else:
+            step.rope(qq, kk, pp)
+
     def run_step():
-        step.rope(q, k, pos)
+        rotary(q, k, pos)
         step.attn(q, k, v, cu)
 
     for _ in range(max(args.warmup, 3)):
@@ -229,7 +244,7 @@ def main():
     t_start.record(stream)
     for s in range(args.steps):
         ev[s][0].record(stream)
-        step.rope(q, k, pos)
+        rotary(q, k, pos)
         ev[s][1].record(stream)
         step.attn(q, k, v, cu)
         ev[s][2].record(stream)
@@ -260,7 +275,7 @@ def main():
         dv.copy_(host["v"], non_blocking=True)
         dcu.copy_(host["cu_seqlens"], non_blocking=True)
         dpos.copy_(host["positions"], non_blocking=True)
-        step.rope(dq, dk, dpos)
+        rotary(dq, dk, dpos)
         o, lse = step.attn(dq, dk, dv, dcu)
         o_host.copy_(o, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
@@ -285,8 +300,9 @@ def main():
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     tab_width = (2 if w.paired else 1) * w.head_dim
+    rname = "qk_norm_rope" if args.qk_norm else "rope"
     kernels = {
-        "rope": {"ms": rope_ms, "bytes": rope_bytes(w, tab_width),
+        rname: {"ms": rope_ms, "bytes": rope_bytes(w, tab_width),
                  "gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9},
         "attention": {"ms": attn_ms, "flops": flops, "bytes": attn_bytes(w),
                       "tflops": attn_tflops,
@@ -294,8 +310,8 @@ def main():
     }
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     attn_bound = "hbm" if flops / attn_bytes(w) < ridge else "tensor"
-    dominant = "attention" if attn_ms >= rope_ms else "rope"
-    if dominant == "rope" or attn_bound == "hbm":
+    dominant = "attention" if attn_ms >= rope_ms else rname
+    if dominant == rname or attn_bound == "hbm":
         kname = dominant
         achieved = kernels[kname]["gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -315,7 +331,8 @@ def main():
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded N(0,1) q/k/v; geometric document lengths)",
-        "config": {**workload_config(w), "parallelism": f"dp{world} (independent documents per rank)",
+        "config": {**workload_config(w), "qk_norm": bool(args.qk_norm),
+                   "parallelism": f"dp{world} (independent documents per rank)",
                    "l2": "inputs larger than L2 (q,k,v + tables > 126 MB); no flush"},
         "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
         "attention_only_tflops": attn_tflops,
@@ -329,11 +346,12 @@ def main():
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, secs, s, thr = time_oracle(w, args.oracle_tokens)
+        tf, secs, s, thr = time_oracle(w, args.oracle_tokens, args.qk_norm)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                 "seconds": secs,
                                 "sample": f"first {s.batch} documents ({s.total} tokens) of the "
-                                          f"workload: float64 RoPE + attention, full rows"}
+                                          f"workload: float64 {'QK RMS-norm + ' if args.qk_norm else ''}"
+                                          f"RoPE + attention, full rows"}
     if rank == 0:
         print(json.dumps(line))
     pdist.finalize(dist)

@@ -91,6 +91,25 @@ pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab
                     int stagger_offset, pha_stream_t stream);
 
 /*
+ * pha_qk_norm_rope -- the QK RMS-norm of every head row, then pha_rope, in one pass (in place).
+ *   The paired-head page's rotary kernel also applies the QK RMS-norm ("modded-nanogpt Paired Head
+ *   Attention record", section "4. interleave index in the Triton kernel"); RMSNorm is
+ *   y = x / sqrt(mean(x^2) + eps) * weight over the last dimension ("Training an LLM from scratch
+ *   (part 2)", section "1. RMSNorm"). Each (token, head) row of q and of k is normalised over
+ *   head_dim in float32 and multiplied by q_weight / k_weight (float[head_dim], 16-byte aligned, or
+ *   NULL for ones), then rotated as pha_rope rotates, with one rounding to dtype at the end.
+ *   Tokens whose position lies outside [0, tab_rows) are normalised but not rotated.
+ *   eps: >= 0, finite. Other arguments, layouts and errors: as pha_rope.
+ *   Supported head_dim: those whose row of 16-byte chunks (head_dim/8 for bf16, head_dim/4 for f32)
+ *   divides 32; others return PHA_ERR_UNSUPPORTED.
+ */
+pha_status pha_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
+                            float eps, const float* cos_tab, const float* sin_tab, int tab_rows,
+                            int tab_width, const int32_t* positions, int total_tokens,
+                            int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype,
+                            int paired, int stagger_offset, pha_stream_t stream);
+
+/*
  * pha_attn_workspace_bytes -- device workspace that pha_attn_fwd needs: a 256-byte header,
  * int32[batch + 1] of per-document scratch (padded to 16 bytes) and the varlen work list, 16
  * bytes for each of at most batch * ceil(L/256) * H' (query block, head) items (L = max_len,

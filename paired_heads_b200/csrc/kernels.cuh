@@ -63,6 +63,13 @@ cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin
                         int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
                         cudaStream_t stream);
 
+// RoPE preceded by the QK RMS-norm of every head row (weights may be NULL = ones).
+cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
+                                float eps, const float* cos_tab, const float* sin_tab,
+                                int tab_rows, int tab_width, const int32_t* positions,
+                                int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                                int is_bf16, int paired, int stagger_offset, cudaStream_t stream);
+
 cudaError_t launch_attn_f32(const AttnProblem& p, cudaStream_t stream);
 
 // Builds the varlen work list (band items when `band`, else block items) into `items` (capacity

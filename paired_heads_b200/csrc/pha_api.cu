@@ -102,6 +102,37 @@ pha_status pha_rope(void* q, void* k, const float* cos_tab, const float* sin_tab
                : PHA_ERR_CUDA;
 }
 
+pha_status pha_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
+                            float eps, const float* cos_tab, const float* sin_tab, int tab_rows,
+                            int tab_width, const int32_t* positions, int total_tokens,
+                            int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype,
+                            int paired, int stagger_offset, pha_stream_t stream) {
+    if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
+    const int span = dtype == PHA_BF16 ? 16 : 8;
+    if (tab_rows < 0 || total_tokens < 0 || n_heads <= 0 || n_kv_heads < 0 || head_dim <= 0 ||
+        head_dim % span != 0 || (paired != 0 && paired != 1) || !(eps >= 0.f) || !(eps < INFINITY))
+        return PHA_ERR_INVALID;
+    if (total_tokens > 0 &&
+        (!q || !aligned16(q) || (n_kv_heads > 0 && (!k || !aligned16(k))) || !cos_tab ||
+         !sin_tab || !aligned16(cos_tab) || !aligned16(sin_tab) || !positions))
+        return PHA_ERR_INVALID;
+    if ((q_weight && !aligned16(q_weight)) || (k_weight && !aligned16(k_weight)))
+        return PHA_ERR_INVALID;
+    if (!paired && (tab_width != head_dim || stagger_offset != 0)) return PHA_ERR_INVALID;
+    if (paired && (tab_width != 2 * head_dim ||
+                   (stagger_offset != 0 && stagger_offset != head_dim)))
+        return PHA_ERR_INVALID;
+    // the 16-byte chunks of one head row must sit on a power-of-two group of lanes of a warp
+    const int cph = head_dim / (dtype == PHA_BF16 ? 8 : 4);
+    if (32 % cph != 0) return PHA_ERR_UNSUPPORTED;
+    if (total_tokens == 0) return PHA_OK;
+    return launch_qk_norm_rope(q, k, q_weight, k_weight, eps, cos_tab, sin_tab, tab_rows, tab_width,
+                               positions, total_tokens, n_heads, n_kv_heads, head_dim,
+                               dtype == PHA_BF16, paired, stagger_offset, stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
 size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired) {
     (void)head_dim;
     if (batch <= 0 || max_len < 0 || n_heads <= 0 || (paired && (n_heads & 1))) return 0;

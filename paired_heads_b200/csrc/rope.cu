@@ -93,19 +93,39 @@ __device__ __forceinline__ uint32_t rot_pair_bf16(float x0, float x1, float c, f
     return bf16_bits_rne(e0) | (bf16_bits_rne(e1) << 16);
 }
 
-// 16-byte chunks of a row: 8 bf16 (4 pairs) or 4 f32 (2 pairs), rotated with the chunk's table
-// values c[j], s[j] (j = element within the chunk).
+// 16-byte chunks of a row: 8 bf16 (4 pairs) or 4 f32 (2 pairs). to_floats gives the exact values;
+// rotate_f rotates E float values with the chunk's table values c[j], s[j] (j = element within
+// the chunk) and rounds once to the buffer type; pack_f only rounds.
 template <typename T>
 struct Chunk16;
 
 template <>
 struct Chunk16<__nv_bfloat16> {
     static constexpr int E = 8;
+    __device__ static void to_floats(uint4 a, float (&x)[E]) {
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[2 * e] = __uint_as_float(w[e] << 16);
+            x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    }
+    __device__ static uint4 rotate_f(const float (&x)[E], const float (&c)[E], const float (&s)[E]) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)  // both members of a pair share one angle: c[2e] == c[2e+1]
+            o[e] = rot_pair_bf16(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e]);
+        return make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    __device__ static uint4 pack_f(const float (&x)[E]) {
+        return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                          pack_bf16x2(x[6], x[7]));
+    }
     __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
         uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)  // both members of a pair share one angle: c[2e] == c[2e+1]
+        for (int e = 0; e < 4; ++e)
             o[e] = rot_pair_bf16(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u),
                                  c[2 * e], s[2 * e]);
         return make_uint4(o[0], o[1], o[2], o[3]);
@@ -115,9 +135,13 @@ struct Chunk16<__nv_bfloat16> {
 template <>
 struct Chunk16<float> {
     static constexpr int E = 4;
-    __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
-        const float x[E] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z),
-                            __uint_as_float(a.w)};
+    __device__ static void to_floats(uint4 a, float (&x)[E]) {
+        x[0] = __uint_as_float(a.x);
+        x[1] = __uint_as_float(a.y);
+        x[2] = __uint_as_float(a.z);
+        x[3] = __uint_as_float(a.w);
+    }
+    __device__ static uint4 rotate_f(const float (&x)[E], const float (&c)[E], const float (&s)[E]) {
         float y[E];
 #pragma unroll
         for (int e = 0; e < E; e += 2) {
@@ -130,6 +154,15 @@ struct Chunk16<float> {
         return make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
                           __float_as_uint(y[3]));
     }
+    __device__ static uint4 pack_f(const float (&x)[E]) {
+        return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
+                          __float_as_uint(x[3]));
+    }
+    __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
+        float x[E];
+        to_floats(a, x);
+        return rotate_f(x, c, s);
+    }
 };
 
 // One warp per token. The token's q row (n_heads * head_dim contiguous elements) followed by its
@@ -139,15 +172,27 @@ struct Chunk16<float> {
 // HBM once and then served from L1.
 constexpr int kRopeBatch = 4;
 
-template <typename T>
-__global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restrict__ k,
+// NORM: each head row is first RMS-normalised over head_dim in float32 ("Training an LLM from
+// scratch (part 2)", section "1. RMSNorm": x / sqrt(mean(x^2) + eps) * weight; weight NULL = 1),
+// then rotated; one rounding at the end. The chunks of one head row sit on cph consecutive lanes
+// (cph divides 32), so the row's sum of squares is a shuffle reduction over those lanes. Tokens
+// whose position lies outside the table are normalised but not rotated.
+// Resident 256-thread blocks per SM: four (64 registers) for the plain bf16 rotation, the
+// bandwidth-bound case; three (80 registers, no spills) for the others.
+template <typename T, bool NORM>
+constexpr int rope_min_blocks() { return (sizeof(T) == 2 && !NORM) ? 4 : 3; }
+
+template <typename T, bool NORM>
+__global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel(T* __restrict__ q, T* __restrict__ k,
                                                    const float* __restrict__ cos_tab,
                                                    const float* __restrict__ sin_tab,
                                                    int tab_rows, int tab_width,
                                                    const int32_t* __restrict__ positions,
                                                    int64_t total_tokens, int n_heads,
                                                    int n_kv_heads, int head_dim, int paired,
-                                                   int stagger_offset) {
+                                                   int stagger_offset,
+                                                   const float* __restrict__ q_weight,
+                                                   const float* __restrict__ k_weight, float eps) {
     constexpr int E = Chunk16<T>::E;
     const int cph = head_dim / E;                  // chunks per head row
     const int q_chunks = n_heads * cph;
@@ -177,6 +222,21 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
                 su[e] = sv.x; su[e + 1] = sv.y; su[e + 2] = sv.z; su[e + 3] = sv.w;
             }
         }
+        // NORM: a lane's chunks always sit at element offset (lane % cph) * E of their head row
+        // (cph divides 32), so its q and k weights are the same for every chunk and token.
+        float wq[E], wk[E];
+        if (NORM) {
+            const int off = (lane % cph) * E;
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+                const float4 a = q_weight ? __ldg(reinterpret_cast<const float4*>(q_weight + off + e))
+                                          : make_float4(1.f, 1.f, 1.f, 1.f);
+                const float4 b = k_weight ? __ldg(reinterpret_cast<const float4*>(k_weight + off + e))
+                                          : make_float4(1.f, 1.f, 1.f, 1.f);
+                wq[e] = a.x; wq[e + 1] = a.y; wq[e + 2] = a.z; wq[e + 3] = a.w;
+                wk[e] = b.x; wk[e + 1] = b.y; wk[e + 2] = b.z; wk[e + 3] = b.w;
+            }
+        }
         for (int base = 0; base < n_chunks; base += 32 * kRopeBatch) {
             uint4 raw[kRopeBatch];
 #pragma unroll
@@ -184,11 +244,40 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
                 const int i = base + 32 * j + lane;
                 if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
             }
-            if (!in_range) continue;  // positions outside the table: leave the token unchanged
+            float inv[kRopeBatch];
+            if (NORM) {
+                // 1 / rms of the head row of each chunk (all lanes take part in the shuffles)
+#pragma unroll
+                for (int j = 0; j < kRopeBatch; ++j) {
+                    float ss = 0.f;
+                    if (base + 32 * j + lane < n_chunks) {
+                        float x[E];
+                        Chunk16<T>::to_floats(raw[j], x);
+#pragma unroll
+                        for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+                    }
+                    for (int o = cph >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                    inv[j] = rsqrtf(ss / static_cast<float>(head_dim) + eps);
+                }
+            } else if (!in_range) {
+                continue;  // positions outside the table: leave the token unchanged
+            }
 #pragma unroll
             for (int j = 0; j < kRopeBatch; ++j) {
                 const int i = base + 32 * j + lane;
                 if (i >= n_chunks) break;
+                float x[E];
+                if (NORM) {
+                    Chunk16<T>::to_floats(raw[j], x);
+                    const bool is_q = i < q_chunks;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) x[e] = x[e] * inv[j] * (is_q ? wq[e] : wk[e]);
+                    if (!in_range) {
+                        const uint4 y = Chunk16<T>::pack_f(x);
+                        if (i < q_chunks) qrow[i] = y; else krow[i - q_chunks] = y;
+                        continue;
+                    }
+                }
                 float c[E], s[E];
                 if (uniform_cols) {
 #pragma unroll
@@ -210,7 +299,7 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restr
                 }
                 // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign
                 // is -1 on the even member and +1 on the odd member (a rotation by +angle).
-                const uint4 y = Chunk16<T>::rotate(raw[j], c, s);
+                const uint4 y = NORM ? Chunk16<T>::rotate_f(x, c, s) : Chunk16<T>::rotate(raw[j], c, s);
                 if (i < q_chunks) qrow[i] = y; else krow[i - q_chunks] = y;
             }
         }
@@ -229,24 +318,47 @@ cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int hea
     return cudaGetLastError();
 }
 
-cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
-                        int tab_width, const int32_t* positions, int total_tokens, int n_heads,
-                        int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
-                        cudaStream_t stream) {
+template <bool NORM>
+static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, const float* sin_tab,
+                                    int tab_rows, int tab_width, const int32_t* positions,
+                                    int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                                    int is_bf16, int paired, int stagger_offset,
+                                    const float* q_weight, const float* k_weight, float eps,
+                                    cudaStream_t stream) {
     if (total_tokens == 0) return cudaSuccess;
     const int threads = 256;  // 8 warps = 8 tokens per block
     const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
     const unsigned blocks = static_cast<unsigned>(blocks64 < (1 << 30) ? blocks64 : (1 << 30));
     if (is_bf16)
-        rope_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
+        rope_kernel<__nv_bfloat16, NORM><<<blocks, threads, 0, stream>>>(
             static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), cos_tab, sin_tab,
             tab_rows, tab_width, positions, total_tokens, n_heads, n_kv_heads, head_dim, paired,
-            stagger_offset);
+            stagger_offset, q_weight, k_weight, eps);
     else
-        rope_kernel<float><<<blocks, threads, 0, stream>>>(
+        rope_kernel<float, NORM><<<blocks, threads, 0, stream>>>(
             static_cast<float*>(q), static_cast<float*>(k), cos_tab, sin_tab, tab_rows, tab_width,
-            positions, total_tokens, n_heads, n_kv_heads, head_dim, paired, stagger_offset);
+            positions, total_tokens, n_heads, n_kv_heads, head_dim, paired, stagger_offset,
+            q_weight, k_weight, eps);
     return cudaGetLastError();
+}
+
+cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
+                        int tab_width, const int32_t* positions, int total_tokens, int n_heads,
+                        int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
+                        cudaStream_t stream) {
+    return launch_rope_impl<false>(q, k, cos_tab, sin_tab, tab_rows, tab_width, positions,
+                                   total_tokens, n_heads, n_kv_heads, head_dim, is_bf16, paired,
+                                   stagger_offset, nullptr, nullptr, 0.f, stream);
+}
+
+cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
+                                float eps, const float* cos_tab, const float* sin_tab,
+                                int tab_rows, int tab_width, const int32_t* positions,
+                                int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                                int is_bf16, int paired, int stagger_offset, cudaStream_t stream) {
+    return launch_rope_impl<true>(q, k, cos_tab, sin_tab, tab_rows, tab_width, positions,
+                                  total_tokens, n_heads, n_kv_heads, head_dim, is_bf16, paired,
+                                  stagger_offset, q_weight, k_weight, eps, stream);
 }
 
 }  // namespace pha

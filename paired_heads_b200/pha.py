@@ -48,8 +48,10 @@ _lib.pha_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i
 _lib.pha_attn_status.argtypes = [_p, ctypes.POINTER(_i), ctypes.POINTER(_i), _p]
 _lib.pha_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                       ctypes.c_float, _p, _p, _p]
+_lib.pha_qk_norm_rope.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _p, _i, _i, _p, _i, _i, _i,
+                                  _i, _i, _i, _i, _p]
 for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status",
-           "pha_attn_fwd_noalloc"):
+           "pha_attn_fwd_noalloc", "pha_qk_norm_rope"):
     getattr(_lib, _f).restype = _i
 
 
@@ -123,6 +125,24 @@ def pha_rope(q, k, cos_tab, sin_tab, positions, paired: bool = False, stagger_of
                                      tab_width, _ptr(positions), total_tokens, n_heads, n_kv_heads,
                                      head_dim, dtype, int(paired), stagger_offset,
                                      _stream(stream, q)))
+
+
+def pha_qk_norm_rope(q, k, cos_tab, sin_tab, positions, q_weight=None, k_weight=None,
+                     eps: float = 1e-6, paired: bool = False, stagger_offset: int = 0, stream=None,
+                     *, tab_rows=None, tab_width=None, total_tokens=None, n_heads=None,
+                     n_kv_heads=None, head_dim=None, dtype=None):
+    """In-place QK RMS-norm (per head row, optional float32 weights of length head_dim) followed
+    by RoPE of q [T][H][hd] and k [T][Hkv][hd]."""
+    if total_tokens is None:
+        total_tokens, n_heads, head_dim = q.shape
+        n_kv_heads = 0 if k is None else k.shape[1]
+        tab_rows, tab_width = cos_tab.shape
+        dtype = _dtype_code(q)
+    _check("pha_qk_norm_rope",
+           _lib.pha_qk_norm_rope(_ptr(q), _ptr(k), _ptr(q_weight), _ptr(k_weight), float(eps),
+                                 _ptr(cos_tab), _ptr(sin_tab), tab_rows, tab_width, _ptr(positions),
+                                 total_tokens, n_heads, n_kv_heads, head_dim, dtype, int(paired),
+                                 stagger_offset, _stream(stream, q)))
 
 
 def pha_attn_workspace_bytes(batch: int, max_len: int, n_heads: int, head_dim: int,

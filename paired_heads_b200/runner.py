@@ -58,6 +58,12 @@ class AttentionStep:
         pha.pha_rope(q, k, self.cos_tab, self.sin_tab, positions, paired=self.s.paired,
                      stagger_offset=self.stagger_offset, stream=stream)
 
+    def norm_rope(self, q, k, positions, q_weight=None, k_weight=None, eps=1e-6, stream=None):
+        """QK RMS-norm of every head row, then RoPE, in place (one kernel)."""
+        pha.pha_qk_norm_rope(q, k, self.cos_tab, self.sin_tab, positions, q_weight, k_weight, eps,
+                             paired=self.s.paired, stagger_offset=self.stagger_offset,
+                             stream=stream)
+
     def attn(self, q, k, v, cu_seqlens, stream=None):
         pha.pha_attn_fwd(q, k, v, cu_seqlens, self.s.max_len, self.o, self.lse, self.workspace,
                          causal=self.s.causal, window=self.s.window, paired=self.s.paired,

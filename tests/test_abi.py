@@ -28,8 +28,8 @@ def _declared():
 
 def test_header_declares_the_entry_points():
     assert _declared() == ["pha_attn_fwd", "pha_attn_fwd_noalloc", "pha_attn_status",
-                           "pha_attn_workspace_bytes", "pha_rope", "pha_rope_tables",
-                           "pha_status_string"]
+                           "pha_attn_workspace_bytes", "pha_qk_norm_rope", "pha_rope",
+                           "pha_rope_tables", "pha_status_string"]
 
 
 def test_library_exports_every_declared_symbol(pha):
@@ -142,3 +142,33 @@ def test_rope_tables_argument_errors(pha):
     assert lib.pha_rope_tables(A, A, 4, 63, 0, ctypes.c_double(1e4), None) == -1
     assert lib.pha_rope_tables(A, A, 4, 64, 0, ctypes.c_double(0.0), None) == -1
     assert lib.pha_rope_tables(A, A, -1, 64, 1, ctypes.c_double(1e4), None) == -1
+
+
+def _norm_rope(pha, **kw):
+    args = dict(q=A, k=A, qw=None, kw=None, eps=1e-6, cos=A, sin=A, rows=16, width=64, pos=A,
+                total=4, H=2, Hkv=2, hd=64, dtype=pha.PHA_BF16, paired=0, stagger=0)
+    args.update(kw)
+    return pha.library().pha_qk_norm_rope(
+        args["q"], args["k"], args["qw"], args["kw"], ctypes.c_float(args["eps"]), args["cos"],
+        args["sin"], args["rows"], args["width"], args["pos"], args["total"], args["H"],
+        args["Hkv"], args["hd"], args["dtype"], args["paired"], args["stagger"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(eps=-1.0), -1),                      # eps >= 0
+    (dict(eps=float("inf")), -1),
+    (dict(eps=float("nan")), -1),
+    (dict(qw=MIS), -1),                        # weights 16-byte aligned
+    (dict(kw=MIS), -1),
+    (dict(width=128), -1),                     # table checks as pha_rope
+    (dict(paired=1, width=128, stagger=32), -1),
+    (dict(q=MIS), -1),
+    (dict(hd=48, width=48), -2),               # 6 chunks per head row: not a divisor of 32
+    (dict(dtype=1, hd=24, width=24), -2),
+])
+def test_norm_rope_argument_errors(pha, kw, code):
+    assert _norm_rope(pha, **kw) == code
+
+
+def test_norm_rope_empty_is_a_no_op(pha):
+    assert _norm_rope(pha, total=0) == 0
