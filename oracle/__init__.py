@@ -137,6 +137,17 @@ def norm_rope_stored(x, positions, dtype: str, paired: bool = False, stagger: bo
     return y.astype(np.float32).astype(np.float64)
 
 
+def add_stored(v, aux, dtype: str):
+    """v + aux (the value embedding added to v before attention: "modded-nanogpt Paired Head
+    Attention record" page, section "3. the paired branch of the forward pass"), as the pipeline
+    stores it in the buffer's dtype. Both operands are exact in float64, so the sum is exact and
+    is rounded once."""
+    y = _f64(v) + _f64(aux)
+    if dtype == "bf16":
+        return round_bf16(y)
+    return y.astype(np.float32).astype(np.float64)
+
+
 def interleave(x):
     """Explicit paired interleave [T][H][d] -> [2T][H/2][d] (copy loop in C)."""
     x = _f64(x)

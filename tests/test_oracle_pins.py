@@ -483,3 +483,31 @@ def test_norm_rope_stored_skips_rotation_outside_the_table():
 
 def synth_bf16(x):
     return oracle.round_bf16(x)
+
+
+# ------------------------------------------------------------------------------ value embedding
+# "modded-nanogpt Paired Head Attention record", section "3. the paired branch of the forward pass":
+# v = v + aux_v (reshaped to v's shape on the paired path) before the varlen attention call.
+
+def test_add_stored_matches_torch_bf16_and_f32_addition():
+    import torch
+
+    rng = np.random.default_rng(21)
+    a = torch.from_numpy(rng.standard_normal(20000).astype(np.float32) * 3).to(torch.bfloat16)
+    b = torch.from_numpy(rng.standard_normal(20000).astype(np.float32)).to(torch.bfloat16)
+    got = oracle.add_stored(a.double().numpy(), b.double().numpy(), "bf16")
+    np.testing.assert_array_equal(got, (a + b).double().numpy())
+    af, bf = a.float() * 1.7, b.float() / 3
+    got = oracle.add_stored(af.double().numpy(), bf.double().numpy(), "f32")
+    np.testing.assert_array_equal(got, (af + bf).double().numpy())
+
+
+def test_value_embedding_shifts_output_by_its_weighted_mean():
+    # attention is linear in v: O(q, k, v + aux) = O(q, k, v) + O(q, k, aux) (float64, no rounding)
+    rng = np.random.default_rng(22)
+    q, k, v, a = (rng.standard_normal((50, 4, 8)) for _ in range(4))
+    cu = np.array([0, 20, 50], dtype=np.int32)
+    o1, _ = oracle.attn_fwd(q, k, v + a, cu, True, 7, True)
+    o2, _ = oracle.attn_fwd(q, k, v, cu, True, 7, True)
+    o3, _ = oracle.attn_fwd(q, k, a, cu, True, 7, True)
+    np.testing.assert_allclose(o1, o2 + o3, rtol=1e-12, atol=1e-12)
