@@ -2,10 +2,11 @@
 inputs resident in HBM. Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--window W]
-                    [--paired 0|1] [--qk-norm] [--impl reference]
+                    [--paired 0|1] [--qk-norm] [--aux-v] [--impl reference]
 
 --qk-norm replaces pha_rope with pha_qk_norm_rope (the QK RMS-norm of every head row, then RoPE,
-in one kernel).
+in one kernel). --aux-v adds a value embedding (a second v-shaped tensor) to v inside the
+attention kernel (pha_attn_fwd_aux_v).
 
 Default workload: the paired-head varlen packed batch (65,536 tokens, documents ~ geometric(512)
 capped at 2048, 6 heads -> 3 pairs, head_dim 128, bf16, causal, window 128 slots, staggered
@@ -189,6 +190,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--qk-norm", action="store_true",
                     help="QK RMS-norm + RoPE (pha_qk_norm_rope) instead of RoPE alone")
+    ap.add_argument("--aux-v", action="store_true",
+                    help="add a value embedding to v inside attention (pha_attn_fwd_aux_v)")
     ap.add_argument("--oracle-tokens", type=int, default=16384)
     args = ap.parse_args()
     w = pick_workload(args)
@@ -221,9 +224,21 @@ def main():
         else:
             step.rope(qq, kk, pp)
 
+    aux = None
+    if args.aux_v:
+        if not step.aux_v_supported:
+            raise SystemExit("--aux-v needs the band kernel (bf16, causal, window <= 128)")
+        g = torch.Generator().manual_seed(7 + 1000 * rank)
+        aux = torch.randn(tuple(v.shape), generator=g).to(v.dtype).to(dev)
+
+    def attention(qq, kk, vv, cc, aa):
+        if args.aux_v:
+            return step.attn_aux_v(qq, kk, vv, aa, cc)
+        return step.attn(qq, kk, vv, cc)
+
     def run_step():
         rotary(q, k, pos)
-        step.attn(q, k, v, cu)
+        attention(q, k, v, cu, aux)
 
     for _ in range(max(args.warmup, 3)):
         run_step()
@@ -246,7 +261,7 @@ def main():
         ev[s][0].record(stream)
         rotary(q, k, pos)
         ev[s][1].record(stream)
-        step.attn(q, k, v, cu)
+        attention(q, k, v, cu, aux)
         ev[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -264,6 +279,9 @@ def main():
 
     # ---- end to end through the public API with host buffers
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "cu_seqlens", "positions")}
+    if args.aux_v:
+        host["aux_v"] = aux.cpu().pin_memory()
+    daux = torch.empty_like(v) if args.aux_v else None
     o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
     lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -275,8 +293,10 @@ def main():
         dv.copy_(host["v"], non_blocking=True)
         dcu.copy_(host["cu_seqlens"], non_blocking=True)
         dpos.copy_(host["positions"], non_blocking=True)
+        if args.aux_v:
+            daux.copy_(host["aux_v"], non_blocking=True)
         rotary(dq, dk, dpos)
-        o, lse = step.attn(dq, dk, dv, dcu)
+        o, lse = attention(dq, dk, dv, dcu, daux)
         o_host.copy_(o, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
 
@@ -301,15 +321,17 @@ def main():
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     tab_width = (2 if w.paired else 1) * w.head_dim
     rname = "qk_norm_rope" if args.qk_norm else "rope"
+    # the value embedding is one more v-shaped read of the attention kernel
+    ab = attn_bytes(w) + (float(w.total * w.n_kv_heads * w.head_dim * 2) if args.aux_v else 0.0)
     kernels = {
         rname: {"ms": rope_ms, "bytes": rope_bytes(w, tab_width),
                  "gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9},
-        "attention": {"ms": attn_ms, "flops": flops, "bytes": attn_bytes(w),
+        "attention": {"ms": attn_ms, "flops": flops, "bytes": ab,
                       "tflops": attn_tflops,
-                      "gbs": attn_bytes(w) / (attn_ms * 1e-3) / 1e9},
+                      "gbs": ab / (attn_ms * 1e-3) / 1e9},
     }
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    attn_bound = "hbm" if flops / attn_bytes(w) < ridge else "tensor"
+    attn_bound = "hbm" if flops / ab < ridge else "tensor"
     dominant = "attention" if attn_ms >= rope_ms else rname
     if dominant == rname or attn_bound == "hbm":
         kname = dominant
@@ -331,7 +353,7 @@ def main():
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded N(0,1) q/k/v; geometric document lengths)",
-        "config": {**workload_config(w), "qk_norm": bool(args.qk_norm),
+        "config": {**workload_config(w), "qk_norm": bool(args.qk_norm), "aux_v": bool(args.aux_v),
                    "parallelism": f"dp{world} (independent documents per rank)",
                    "l2": "inputs larger than L2 (q,k,v + tables > 126 MB); no flush"},
         "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],

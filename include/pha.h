@@ -156,6 +156,25 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
                         pha_stream_t stream);
 
 /*
+ * pha_attn_fwd_aux_v -- pha_attn_fwd with a value embedding added to v on the way in:
+ *   attention over (q, k, v + aux_v), with v + aux_v rounded to dtype as a tensor addition in
+ *   dtype rounds it ("modded-nanogpt Paired Head Attention record" page, section "3. the paired
+ *   branch of the forward pass": v = v + aux_v, reshaped like v on the paired path). aux_v has v's
+ *   shape, dtype and layout ([total_tokens][n_kv_heads][head_dim], 16-byte aligned); neither v nor
+ *   aux_v is modified (the sum is formed tile by tile in shared memory).
+ *   Other arguments, results and errors: as pha_attn_fwd.
+ *   Supported: bf16, causal, 1 <= window <= 128 (the band kernel), head_dim in {64, 128};
+ *      anything else returns PHA_ERR_UNSUPPORTED before any launch. aux_v NULL with
+ *      total_tokens > 0: PHA_ERR_INVALID.
+ */
+pha_status pha_attn_fwd_aux_v(const void* q, const void* k, const void* v, const void* aux_v,
+                              const int32_t* cu_seqlens, int batch, int max_len,
+                              int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                              pha_dtype dtype, int causal, int window, int paired, float scale,
+                              void* o, float* lse, void* workspace, size_t workspace_bytes,
+                              pha_stream_t stream);
+
+/*
  * pha_attn_status -- synchronise `stream` and read the device-side status that the last
  * pha_attn_fwd on this workspace recorded: 0 = fine; 1 = cu_seqlens malformed (decreasing,
  * negative start, beyond total_tokens, or a document longer than max_len); 2 = more work

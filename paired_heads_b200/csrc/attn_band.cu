@@ -33,11 +33,13 @@
 
 namespace pha {
 
-constexpr int kBandThreads = 352;
+constexpr int kBandThreads = 352;     // 8 softmax warps, producer, 2 MMA issuers
+constexpr int kBandAuxThreads = 480;  // + an adder warpgroup (value embedding)
 
 struct BandBars {
     uint64_t q_full[3], q_empty[3];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+    uint64_t v_add[4];  // value embedding: the landed V tile has had aux_v added
     uint64_t s_full[2], p_full[2], pv_done[2], o_ready[2];
     uint64_t drain[2];
     uint32_t tmem_base;
@@ -95,8 +97,47 @@ struct ItemWalk {
     }
 };
 
+// Adder warpgroup (value embedding): adds rows [row0, row0 + 128) of aux_v (head hs of the slot
+// view, heads_slot heads per slot row, the same layout as v) to the landed V tile in shared memory,
+// rounding each sum to bf16 as a bf16 tensor addition does. Rows past the tensor are left as they
+// are. Thread t of the 128 takes 16-byte unit t % (hd / 8) of every (1024 / hd)-th row; all of its
+// global loads are issued before the first add.
 template <int HD>
-__global__ void __launch_bounds__(kBandThreads, 1)
+__device__ __forceinline__ void add_aux_tile(uint8_t* tile, const __nv_bfloat16* aux, int row0, int hs,
+                                             int heads_slot, int64_t slots, int at) {
+    constexpr int kUnits = HD / 8;
+    constexpr int kRowsPerPass = 128 / kUnits;
+    constexpr int kPasses = kBlockN / kRowsPerPass;
+    const int unit = at % kUnits;
+    uint4 a[kPasses];
+#pragma unroll
+    for (int k = 0; k < kPasses; ++k) {
+        const int r = at / kUnits + k * kRowsPerPass;
+        const int64_t slot = static_cast<int64_t>(row0) + r;
+        a[k] = slot < slots ? __ldg(reinterpret_cast<const uint4*>(
+                                  aux + (slot * heads_slot + hs) * HD + unit * 8))
+                            : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < kPasses; ++k) {
+        const int r = at / kUnits + k * kRowsPerPass;
+        if (static_cast<int64_t>(row0) + r >= slots) break;
+        // unit u of row r in the 128-byte-swizzled [128 rows][64 bf16] chunks of the tile
+        uint4* addr = reinterpret_cast<uint4*>(tile + (unit >> 3) * (kBlockN * 128) + r * 128 +
+                                               (((unit & 7) ^ (r & 7)) << 4));
+        const uint4 v = *addr;
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w}, aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)  // bf16 + bf16 is exact in float32; one rounding to bf16
+            o[e] = pack_bf16x2(__uint_as_float(vw[e] << 16) + __uint_as_float(aw[e] << 16),
+                               __uint_as_float(vw[e] & 0xFFFF0000u) + __uint_as_float(aw[e] & 0xFFFF0000u));
+        *addr = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+template <int HD, bool AUXV>
+__global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
     attn_band_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnProblem p,
@@ -124,6 +165,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             mbar_init(&bars->q_empty[s], 5);
         }
         for (int s = 0; s < 4; ++s) {
+            mbar_init(&bars->v_add[s], 128);
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 2);
             mbar_init(&bars->v_full[s], 1);
@@ -221,6 +263,33 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             }
         }
         __syncwarp();
+    } else if (AUXV && warp >= 11) {
+        // ------------------------------------------------------------ adder warpgroup
+        // V tiles in the producer's order; each gets aux_v added once it has landed, then is
+        // published to the MMA issuers.
+        const int at = threadIdx.x - kBandThreads;
+        const int64_t slots = static_cast<int64_t>(p.total_tokens) * p.slot_mult;
+        const __nv_bfloat16* aux = static_cast<const __nv_bfloat16*>(p.v_aux);
+        uint32_t vc = 0;
+        bool ok = true;
+        ItemWalk wk;
+        for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+            if (!wk.has()) continue;
+            const BandItem it = decode_band(wk.cur);
+            const int gk = it.head / G;
+            const int kv_first = it.q0 - (it.hp ? kBlockN : 0);
+            for (int s = 0; ok && s < it.n_qt + it.hp; ++s) {
+                const uint32_t sv = vc % S;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[sv], (vc / S) & 1, abort_flag,
+                                                       dev_status));
+                if (!ok) break;
+                add_aux_tile<HD>(smem + L::kOffV + sv * L::kKV, aux, kv_first + s * kBlockN, gk,
+                                 p.kv_heads, slots, at);
+                fence_proxy_async_smem();  // the tensor cores read the tile next
+                mbar_arrive(&bars->v_add[sv]);
+                ++vc;
+            }
+        }
     } else if (warp >= 9) {
         // ------------------------------------------------------------ MMA issuer of warpgroup w
         const int w = warp - 9;
@@ -278,7 +347,10 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     } else {
                         mbar_arrive(&bars->k_empty[st]);
                     }
-                    if (!mbar_wait(&bars->v_full[st], ph, abort_flag, dev_status)) {
+                    // every fill is observed in order, used or not (the adder's barrier when the
+                    // value embedding is on), so no wait can alias a fill one lap later
+                    if (!mbar_wait(AUXV ? &bars->v_add[st] : &bars->v_full[st], ph, abort_flag,
+                                   dev_status)) {
                         ok = false;
                         break;
                     }
@@ -491,19 +563,20 @@ __global__ void __launch_bounds__(kBandThreads, 1)
     if (warp == 9) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-template <int HD>
+template <int HD, bool AUXV>
 static cudaError_t launch_band_hd(const AttnProblem& p, const CUtensorMap& tq,
                                   const CUtensorMap& tk, const CUtensorMap& tv, const int4* items,
                                   WorkspaceHeader* hdr, cudaStream_t stream) {
     using L = TcLayout<HD>;
-    cudaError_t e = cudaFuncSetAttribute(attn_band_kernel<HD>,
+    cudaError_t e = cudaFuncSetAttribute(attn_band_kernel<HD, AUXV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    attn_band_kernel<HD><<<sms, kBandThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p, items, hdr);
+    attn_band_kernel<HD, AUXV><<<sms, AUXV ? kBandAuxThreads : kBandThreads, L::kSmemBytes, stream>>>(
+        tq, tk, tv, p, items, hdr);
     return cudaGetLastError();
 }
 
@@ -511,8 +584,13 @@ cudaError_t launch_attn_band(const AttnProblem& p, const CUtensorMap& tm_q,
                              const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int4* items,
                              WorkspaceHeader* hdr, cudaStream_t stream) {
     if (!band_applies(p)) return cudaErrorInvalidValue;
-    if (p.head_dim == 128) return launch_band_hd<128>(p, tm_q, tm_k, tm_v, items, hdr, stream);
-    if (p.head_dim == 64) return launch_band_hd<64>(p, tm_q, tm_k, tm_v, items, hdr, stream);
+    const bool aux = p.v_aux != nullptr;
+    if (p.head_dim == 128)
+        return aux ? launch_band_hd<128, true>(p, tm_q, tm_k, tm_v, items, hdr, stream)
+                   : launch_band_hd<128, false>(p, tm_q, tm_k, tm_v, items, hdr, stream);
+    if (p.head_dim == 64)
+        return aux ? launch_band_hd<64, true>(p, tm_q, tm_k, tm_v, items, hdr, stream)
+                   : launch_band_hd<64, false>(p, tm_q, tm_k, tm_v, items, hdr, stream);
     return cudaErrorInvalidValue;
 }
 

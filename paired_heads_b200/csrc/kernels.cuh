@@ -53,6 +53,9 @@ struct AttnProblem {
     float scale;
     void* o;
     float* lse;
+    // Value embedding (pha_attn_fwd_aux_v): added to v, with v's layout, before attention;
+    // nullptr: none.
+    const void* v_aux;
 };
 
 cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,

@@ -140,11 +140,15 @@ size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_di
            static_cast<size_t>(max_work_items(batch, max_len, n_heads, paired)) * sizeof(int4);
 }
 
-pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
-                        int batch, int max_len, int total_tokens, int n_heads, int n_kv_heads,
-                        int head_dim, pha_dtype dtype, int causal, int window, int paired,
-                        float scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
-                        pha_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+pha_status attn_fwd_impl(const void* q, const void* k, const void* v, const void* v_aux,
+                         const int32_t* cu_seqlens, int batch, int max_len, int total_tokens,
+                         int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype, int causal,
+                         int window, int paired, float scale, void* o, float* lse, void* workspace,
+                         size_t workspace_bytes, pha_stream_t stream) {
     if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
     // With no tokens the q / k / v / o / lse buffers may be empty (NULL); cu_seqlens is still read.
     const bool have = total_tokens > 0;
@@ -177,6 +181,12 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
     p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
     p.o = o;
     p.lse = lse;
+    if (v_aux) {
+        // value embedding: the band kernel only (bf16, causal, 1 <= window <= 128)
+        if (dtype != PHA_BF16 || !band_applies(p)) return PHA_ERR_UNSUPPORTED;
+        if (!aligned16(v_aux)) return PHA_ERR_INVALID;
+        p.v_aux = v_aux;
+    }
 
     if (dtype == PHA_F32) {
         if (total_tokens == 0) return PHA_OK;
@@ -209,6 +219,32 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
     const cudaError_t e = band ? launch_attn_band(p, tq, tk, tv, items, hdr, stream)
                                : launch_attn_tc(p, tq, tk, tv, items, hdr, stream);
     return e == cudaSuccess ? PHA_OK : PHA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                        int batch, int max_len, int total_tokens, int n_heads, int n_kv_heads,
+                        int head_dim, pha_dtype dtype, int causal, int window, int paired,
+                        float scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                        pha_stream_t stream) {
+    return attn_fwd_impl(q, k, v, nullptr, cu_seqlens, batch, max_len, total_tokens, n_heads,
+                         n_kv_heads, head_dim, dtype, causal, window, paired, scale, o, lse,
+                         workspace, workspace_bytes, stream);
+}
+
+pha_status pha_attn_fwd_aux_v(const void* q, const void* k, const void* v, const void* aux_v,
+                              const int32_t* cu_seqlens, int batch, int max_len,
+                              int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                              pha_dtype dtype, int causal, int window, int paired, float scale,
+                              void* o, float* lse, void* workspace, size_t workspace_bytes,
+                              pha_stream_t stream) {
+    if (total_tokens > 0 && !aux_v) return PHA_ERR_INVALID;
+    return attn_fwd_impl(q, k, v, total_tokens > 0 ? aux_v : nullptr, cu_seqlens, batch, max_len,
+                         total_tokens, n_heads, n_kv_heads, head_dim, dtype, causal, window,
+                         paired, scale, o, lse, workspace, workspace_bytes, stream);
 }
 
 pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream) {

@@ -48,10 +48,12 @@ _lib.pha_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i
 _lib.pha_attn_status.argtypes = [_p, ctypes.POINTER(_i), ctypes.POINTER(_i), _p]
 _lib.pha_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                       ctypes.c_float, _p, _p, _p]
+_lib.pha_attn_fwd_aux_v.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                    ctypes.c_float, _p, _p, _p, _sz, _p]
 _lib.pha_qk_norm_rope.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _p, _i, _i, _p, _i, _i, _i,
                                   _i, _i, _i, _i, _p]
 for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status",
-           "pha_attn_fwd_noalloc", "pha_qk_norm_rope"):
+           "pha_attn_fwd_noalloc", "pha_qk_norm_rope", "pha_attn_fwd_aux_v"):
     getattr(_lib, _f).restype = _i
 
 
@@ -167,6 +169,26 @@ def pha_attn_fwd(q, k, v, cu_seqlens, max_len: int, o, lse, workspace, *, causal
                                              dtype, int(causal), int(window), int(paired),
                                              float(scale), _ptr(o), _ptr(lse), _ptr(workspace),
                                              workspace_bytes, _stream(stream, q)))
+
+
+def pha_attn_fwd_aux_v(q, k, v, aux_v, cu_seqlens, max_len: int, o, lse, workspace, *,
+                       causal: bool = True, window: int = 0, paired: bool = False,
+                       scale: float = 0.0, stream=None, batch=None, total_tokens=None,
+                       n_heads=None, n_kv_heads=None, head_dim=None, dtype=None,
+                       workspace_bytes=None):
+    """Varlen attention forward over (q, k, v + aux_v) into o and lse (v, aux_v unchanged)."""
+    if total_tokens is None:
+        total_tokens, n_heads, head_dim = q.shape
+        n_kv_heads = k.shape[1]
+        batch = cu_seqlens.shape[0] - 1
+        dtype = _dtype_code(q)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pha_attn_fwd_aux_v",
+           _lib.pha_attn_fwd_aux_v(_ptr(q), _ptr(k), _ptr(v), _ptr(aux_v), _ptr(cu_seqlens), batch,
+                                   max_len, total_tokens, n_heads, n_kv_heads, head_dim, dtype,
+                                   int(causal), int(window), int(paired), float(scale), _ptr(o),
+                                   _ptr(lse), _ptr(workspace), workspace_bytes, _stream(stream, q)))
 
 
 def pha_attn_fwd_noalloc(q, k, v, cu_seqlens, max_len: int, o, lse, *, causal: bool = True,

@@ -70,6 +70,21 @@ class AttentionStep:
                          scale=self.s.scale, stream=stream)
         return self.o, self.lse
 
+    @property
+    def aux_v_supported(self) -> bool:
+        """Whether pha_attn_fwd_aux_v covers this shape (the band kernel: bf16, causal,
+        1 <= window <= 128, head_dim 64 or 128)."""
+        s = self.s
+        return (s.dtype == "bf16" and s.causal and 1 <= s.window <= 128
+                and s.head_dim in (64, 128))
+
+    def attn_aux_v(self, q, k, v, aux_v, cu_seqlens, stream=None):
+        """Attention over (q, k, v + aux_v); v and aux_v are left unchanged."""
+        pha.pha_attn_fwd_aux_v(q, k, v, aux_v, cu_seqlens, self.s.max_len, self.o, self.lse,
+                               self.workspace, causal=self.s.causal, window=self.s.window,
+                               paired=self.s.paired, scale=self.s.scale, stream=stream)
+        return self.o, self.lse
+
     def __call__(self, q, k, v, cu_seqlens, positions, stream=None):
         """RoPE q and k in place, then attention. Returns (o, lse) (buffers owned by the step)."""
         self.rope(q, k, positions, stream)

@@ -27,9 +27,9 @@ def _declared():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["pha_attn_fwd", "pha_attn_fwd_noalloc", "pha_attn_status",
-                           "pha_attn_workspace_bytes", "pha_qk_norm_rope", "pha_rope",
-                           "pha_rope_tables", "pha_status_string"]
+    assert _declared() == ["pha_attn_fwd", "pha_attn_fwd_aux_v", "pha_attn_fwd_noalloc",
+                           "pha_attn_status", "pha_attn_workspace_bytes", "pha_qk_norm_rope",
+                           "pha_rope", "pha_rope_tables", "pha_status_string"]
 
 
 def test_library_exports_every_declared_symbol(pha):
@@ -172,3 +172,29 @@ def test_norm_rope_argument_errors(pha, kw, code):
 
 def test_norm_rope_empty_is_a_no_op(pha):
     assert _norm_rope(pha, total=0) == 0
+
+
+def _attn_aux(pha, **kw):
+    args = dict(q=A, k=A, v=A, aux=A, cu=A, batch=1, max_len=128, total=128, H=4, Hkv=4, hd=64,
+                dtype=pha.PHA_BF16, causal=1, window=128, paired=0, scale=0.0, o=A, lse=A, ws=A,
+                ws_bytes=10)
+    args.update(kw)
+    return pha.library().pha_attn_fwd_aux_v(
+        args["q"], args["k"], args["v"], args["aux"], args["cu"], args["batch"], args["max_len"],
+        args["total"], args["H"], args["Hkv"], args["hd"], args["dtype"], args["causal"],
+        args["window"], args["paired"], ctypes.c_float(args["scale"]), args["o"], args["lse"],
+        args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(), -3),                              # valid: only the (too small) workspace stops it
+    (dict(aux=None), -1),
+    (dict(aux=MIS), -1),
+    (dict(window=0), -2),                      # the band kernel only
+    (dict(window=129), -2),
+    (dict(dtype=1), -2),
+    (dict(hd=96), -2),
+    (dict(H=6, Hkv=4), -1),
+])
+def test_attn_aux_v_argument_errors(pha, kw, code):
+    assert _attn_aux(pha, **kw) == code
