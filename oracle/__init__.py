@@ -60,6 +60,11 @@ def _load():
         lib.oracle_attn_fwd.argtypes = [_f64p, _f64p, _f64p, _i32p, _c, _c, _c, _c, _c, _c, _c,
                                         _d, _f64p, _f64p]
         lib.oracle_rms_norm.argtypes = [_f64p, _l, _c, ctypes.c_void_p, _d]
+        lib.oracle_attn_bwd.argtypes = [_f64p, _f64p, _f64p, _f64p, _i32p, _c, _c, _c, _c, _c, _c,
+                                        _c, _d, _f64p, _f64p, _f64p]
+        lib.oracle_rope_bwd.argtypes = [_f64p, _i32p, _l, _c, _c, _c, _c, _d, _c]
+        lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_rope_bwd.restype = ctypes.c_int
         for f in ("oracle_rms_norm", "oracle_rope", "oracle_round_bf16", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
                   "oracle_attention_rows", "oracle_attn_fwd"):
             getattr(lib, f).restype = ctypes.c_int
@@ -231,3 +236,29 @@ def attn_rows(q, k, v, cu_seqlens, rows, causal=True, window=0, paired=False, sc
                                          hd, int(causal), int(window), scale, slot_rows, n, o,
                                          lse), "attn_rows")
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, cu_seqlens, causal=True, window=0, paired=False, scale=None):
+    """Gradients (dq, dk, dv) of attn_fwd's O with respect to q, k, v for the upstream gradient
+    dout (float64; token-major like attn_fwd). P is recomputed from q and k."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    T, H, hd = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / np.sqrt(hd) if scale is None or scale <= 0 else float(scale)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    _check(_load().oracle_attn_bwd(q, k, v, dout, cu, len(cu) - 1, H, Hkv, hd, int(causal),
+                                   int(window), int(paired), scale, dq, dk, dv), "attn_bwd")
+    return dq, dk, dv
+
+
+def rope_bwd(dy, positions, paired: bool = False, stagger: bool = False, base: float = 10000.0,
+             table_f32: bool = False):
+    """Gradient of rope() with respect to its input for the upstream gradient dy: the transposed
+    rotation of every pair (returns a new float64 array)."""
+    y = _f64(dy).copy()
+    T, H, hd = y.shape
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    _check(_load().oracle_rope_bwd(y, pos, T, H, hd, int(paired), int(stagger), float(base),
+                                   int(table_f32)), "rope_bwd")
+    return y

@@ -312,3 +312,152 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v, const int
     free(qi); free(ki); free(vi); free(oi); free(li); free(cu);
     return rc;
 }
+
+/* ------------------------------------------------------------------ backward (gradients)
+ * The gradients of the attention above with respect to q, k, v for an upstream gradient dO, by
+ * the chain rule through the row softmax (the standard identity: with P_ij the softmax weights,
+ * dP_ij = dO_i . v_j, dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik), dQ_i = scale sum_j dS_ij k_j,
+ * dK_j = scale sum_i dS_ij q_i, dV_j = sum_i P_ij dO_i). P is recomputed here from q and k with
+ * the same two-pass softmax as attend_row; nothing saved by the forward is used. */
+
+/* Slot-major buffers as oracle_attention; dq[S][H][hd], dk, dv[S][Hkv][hd] (overwritten). */
+int oracle_attention_bwd(const double* q, const double* k, const double* v, const double* dout,
+                         const int64_t* cu, int B, int H, int Hkv, int hd, int causal, int window,
+                         double scale, double* dq, double* dk, double* dv)
+{
+    if (!q || !k || !v || !dout || !cu || !dq || !dk || !dv || B < 0 || H <= 0 || Hkv <= 0 ||
+        (H % Hkv) != 0 || hd <= 0 || !check_cu(cu, B))
+        return ORACLE_EINVAL;
+    const int G = H / Hkv;
+    const int64_t S = cu[B];
+    memset(dq, 0, sizeof(double) * (size_t)S * H * hd);
+    memset(dk, 0, sizeof(double) * (size_t)S * Hkv * hd);
+    memset(dv, 0, sizeof(double) * (size_t)S * Hkv * hd);
+    for (int b = 0; b < B; ++b) {
+        const int64_t lo = cu[b], hi = cu[b + 1];
+        const int64_t L = hi - lo;
+        if (L <= 0) continue;
+        /* one kv head per task: its dk, dv rows receive every query head of its group */
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int g = 0; g < Hkv; ++g) {
+            double* p = (double*)malloc(sizeof(double) * (size_t)L);
+            double* dp = (double*)malloc(sizeof(double) * (size_t)L);
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                for (int64_t i = lo; i < hi; ++i) {
+                    const double* qi = q + ((size_t)i * H + h) * hd;
+                    const double* gi = dout + ((size_t)i * H + h) * hd;
+                    double m = -INFINITY;
+                    for (int64_t j = lo; j < hi; ++j) {
+                        p[j - lo] = -INFINITY;
+                        if (!visible(i, j, lo, hi, causal, window)) continue;
+                        const double* kj = k + ((size_t)j * Hkv + g) * hd;
+                        double sc = 0.0;
+                        for (int e = 0; e < hd; ++e) sc += qi[e] * kj[e];
+                        p[j - lo] = sc * scale;
+                        if (p[j - lo] > m) m = p[j - lo];
+                    }
+                    if (m == -INFINITY) continue;
+                    double l = 0.0;
+                    for (int64_t j = lo; j < hi; ++j) {
+                        p[j - lo] = (p[j - lo] == -INFINITY) ? 0.0 : exp(p[j - lo] - m);
+                        l += p[j - lo];
+                    }
+                    double dsum = 0.0;
+                    for (int64_t j = lo; j < hi; ++j) {
+                        p[j - lo] /= l;
+                        dp[j - lo] = 0.0;
+                        if (p[j - lo] == 0.0) continue;
+                        const double* vj = v + ((size_t)j * Hkv + g) * hd;
+                        for (int e = 0; e < hd; ++e) dp[j - lo] += gi[e] * vj[e];
+                        dsum += p[j - lo] * dp[j - lo];
+                    }
+                    double* dqi = dq + ((size_t)i * H + h) * hd;
+                    for (int64_t j = lo; j < hi; ++j) {
+                        if (p[j - lo] == 0.0) continue;
+                        const double ds = p[j - lo] * (dp[j - lo] - dsum);
+                        const double* kj = k + ((size_t)j * Hkv + g) * hd;
+                        double* dkj = dk + ((size_t)j * Hkv + g) * hd;
+                        double* dvj = dv + ((size_t)j * Hkv + g) * hd;
+                        for (int e = 0; e < hd; ++e) {
+                            dqi[e] += scale * ds * kj[e];
+                            dkj[e] += scale * ds * qi[e];
+                            dvj[e] += p[j - lo] * gi[e];
+                        }
+                    }
+                }
+            }
+            free(p);
+            free(dp);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Token-major wrapper like oracle_attn_fwd: paired = 1 interleaves q, k, v, dout explicitly, runs
+ * the slot-major backward on the doubled documents and de-interleaves dq, dk, dv. */
+int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
+                    const int32_t* cu_seqlens, int B, int H, int Hkv, int hd, int causal,
+                    int window, int paired, double scale, double* dq, double* dk, double* dv)
+{
+    if (!q || !k || !v || !dout || !cu_seqlens || !dq || !dk || !dv || B < 0 || H <= 0 ||
+        Hkv <= 0 || (H % Hkv) != 0 || hd <= 0)
+        return ORACLE_EINVAL;
+    if (paired && ((H % 2) != 0 || (Hkv % 2) != 0)) return ORACLE_EINVAL;
+    const int64_t T = cu_seqlens[B];
+    int64_t* cu = (int64_t*)malloc(sizeof(int64_t) * (size_t)(B + 1));
+    if (!cu) return ORACLE_ENOMEM;
+    for (int b = 0; b <= B; ++b) cu[b] = (paired ? 2 : 1) * (int64_t)cu_seqlens[b];
+    int rc;
+    if (!paired) {
+        rc = oracle_attention_bwd(q, k, v, dout, cu, B, H, Hkv, hd, causal, window, scale, dq, dk,
+                                  dv);
+        free(cu);
+        return rc;
+    }
+    const size_t nq = (size_t)T * H * hd, nk = (size_t)T * Hkv * hd;
+    double* buf = (double*)malloc(sizeof(double) * (4 * nq + 4 * nk));
+    if (!buf) { free(cu); return ORACLE_ENOMEM; }
+    double *qi = buf, *gi = qi + nq, *dqi = gi + nq, *ki = dqi + nq, *vi = ki + nk, *dki = vi + nk,
+           *dvi = dki + nk;
+    oracle_interleave(q, qi, T, H, hd);
+    oracle_interleave(dout, gi, T, H, hd);
+    oracle_interleave(k, ki, T, Hkv, hd);
+    oracle_interleave(v, vi, T, Hkv, hd);
+    rc = oracle_attention_bwd(qi, ki, vi, gi, cu, B, H / 2, Hkv / 2, hd, causal, window, scale,
+                              dqi, dki, dvi);
+    if (rc == ORACLE_OK) {
+        oracle_deinterleave(dqi, dq, T, H, hd);
+        oracle_deinterleave(dki, dk, T, Hkv, hd);
+        oracle_deinterleave(dvi, dv, T, Hkv, hd);
+    }
+    free(buf);
+    free(cu);
+    return rc;
+}
+
+/* Gradient of oracle_rope with respect to its input: the transposed rotation of every pair,
+ * dx0 = c dy0 + s dy1, dx1 = -s dy0 + c dy1 (in place on dy[n_tok][n_head][hd]). */
+int oracle_rope_bwd(double* dy, const int32_t* pos, int64_t n_tok, int n_head, int hd,
+                    int paired, int stagger, double base, int table_f32)
+{
+    if (!dy || !pos || n_tok < 0 || n_head <= 0 || hd <= 0 || (hd % 2) != 0) return ORACLE_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n_tok; ++t) {
+        for (int h = 0; h < n_head; ++h) {
+            double* row = dy + ((size_t)t * (size_t)n_head + (size_t)h) * (size_t)hd;
+            double phase = rope_phase(pos[t], h, paired, stagger);
+            for (int i = 0; i < hd / 2; ++i) {
+                double theta = phase * rope_freq(i, hd, base);
+                double c = cos(theta), s = sin(theta);
+                if (table_f32) {
+                    c = (double)(float)c;
+                    s = (double)(float)s;
+                }
+                double a = row[2 * i], b = row[2 * i + 1];
+                row[2 * i] = a * c + b * s;
+                row[2 * i + 1] = -a * s + b * c;
+            }
+        }
+    }
+    return ORACLE_OK;
+}

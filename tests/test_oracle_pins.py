@@ -511,3 +511,90 @@ def test_value_embedding_shifts_output_by_its_weighted_mean():
     o2, _ = oracle.attn_fwd(q, k, v, cu, True, 7, True)
     o3, _ = oracle.attn_fwd(q, k, a, cu, True, 7, True)
     np.testing.assert_allclose(o1, o2 + o3, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------ backward
+# Gradients of the attention (and of RoPE) with respect to their inputs, for an upstream gradient
+# dO; pinned to finite differences of the forward oracle and to torch's float64 autograd.
+
+def _loss_grad_fd(f, x, g, eps=1e-6):
+    """Central differences of <f(x), g> with respect to every element of x."""
+    out = np.empty_like(x)
+    flat, of = x.reshape(-1), out.reshape(-1)
+    for n in range(flat.size):
+        old = flat[n]
+        flat[n] = old + eps
+        up = float((f(x) * g).sum())
+        flat[n] = old - eps
+        dn = float((f(x) * g).sum())
+        flat[n] = old
+        of[n] = (up - dn) / (2 * eps)
+    return out
+
+
+@pytest.mark.parametrize("case", [
+    # T per doc, H, Hkv, hd, causal, window, paired
+    ((5, 7), 2, 2, 4, True, 0, False),
+    ((6, 3), 4, 2, 4, True, 2, False),
+    ((4, 5), 4, 2, 4, True, 3, True),
+    ((6,), 2, 1, 4, False, 0, False),
+])
+def test_attention_backward_matches_finite_differences(case):
+    lens, H, Hkv, hd, causal, window, paired = case
+    rng = np.random.default_rng(sum(lens) + H + window)
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q, k, v, g = (rng.standard_normal((T, h, hd)) for h in (H, Hkv, Hkv, H))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, cu, causal, window, paired)
+    fwd = lambda qq, kk, vv: oracle.attn_fwd(qq, kk, vv, cu, causal, window, paired)[0]
+    np.testing.assert_allclose(dq, _loss_grad_fd(lambda x: fwd(x, k, v), q.copy(), g), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _loss_grad_fd(lambda x: fwd(q, x, v), k.copy(), g), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _loss_grad_fd(lambda x: fwd(q, k, x), v.copy(), g), rtol=1e-6, atol=1e-8)
+
+
+def test_attention_backward_matches_torch_autograd_float64():
+    import torch
+
+    rng = np.random.default_rng(31)
+    T, H, Hkv, hd, window = 40, 4, 2, 8, 9
+    cu = np.array([0, 17, 40], dtype=np.int32)
+    q, k, v, g = (rng.standard_normal((T, h, hd)) for h in (H, Hkv, Hkv, H))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, cu, True, window, False)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    doc = torch.from_numpy(np.searchsorted(cu[1:], np.arange(T), side="right"))
+    mask = (doc[:, None] == doc[None, :]) & (j <= i) & (i - j < window)
+    kk = tk.repeat_interleave(H // Hkv, dim=1)
+    vv = tv.repeat_interleave(H // Hkv, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(0, 1), kk.transpose(0, 1), vv.transpose(0, 1), attn_mask=mask).transpose(0, 1)
+    (o * torch.from_numpy(g)).sum().backward()
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_paired_backward_equals_standard_backward_on_interleaved_tensors():
+    rng = np.random.default_rng(32)
+    lens, H, Hkv, hd = (9, 6), 4, 2, 4
+    T = sum(lens)
+    cu = np.array([0, 9, 15], dtype=np.int32)
+    q, k, v, g = (rng.standard_normal((T, h, hd)) for h in (H, Hkv, Hkv, H))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, cu, True, 5, True)
+    il = oracle.interleave
+    dqs, dks, dvs = oracle.attn_bwd(il(q), il(k), il(v), il(g), 2 * cu, True, 5, False)
+    np.testing.assert_array_equal(dq, oracle.deinterleave(dqs))
+    np.testing.assert_array_equal(dk, oracle.deinterleave(dks))
+    np.testing.assert_array_equal(dv, oracle.deinterleave(dvs))
+
+
+@pytest.mark.parametrize("paired,stagger", [(False, False), (True, True)])
+def test_rope_backward_is_adjoint_and_inverse(paired, stagger):
+    rng = np.random.default_rng(33)
+    x, y = rng.standard_normal((2, 7, 6, 16))
+    pos = rng.integers(0, 3000, 7).astype(np.int32)
+    rx = oracle.rope(x, pos, paired, stagger)
+    bty = oracle.rope_bwd(y, pos, paired, stagger)
+    assert abs(float((rx * y).sum() - (x * bty).sum())) < 1e-11   # <R x, y> = <x, R^T y>
+    np.testing.assert_allclose(oracle.rope_bwd(rx, pos, paired, stagger), x, rtol=0, atol=1e-12)
