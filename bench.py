@@ -2,11 +2,12 @@
 inputs resident in HBM. Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--window W]
-                    [--paired 0|1] [--qk-norm] [--aux-v] [--impl reference]
+                    [--paired 0|1] [--qk-norm] [--aux-v] [--backward] [--impl reference]
 
 --qk-norm replaces pha_rope with pha_qk_norm_rope (the QK RMS-norm of every head row, then RoPE,
 in one kernel). --aux-v adds a value embedding (a second v-shaped tensor) to v inside the
-attention kernel (pha_attn_fwd_aux_v).
+attention kernel (pha_attn_fwd_aux_v). --backward also times the backward (pha_attn_bwd +
+pha_rope_bwd) after the forward step and reports it under "backward" (not in `value`).
 
 Default workload: the paired-head varlen packed batch (65,536 tokens, documents ~ geometric(512)
 capped at 2048, 6 heads -> 3 pairs, head_dim 128, bf16, causal, window 128 slots, staggered
@@ -190,6 +191,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--qk-norm", action="store_true",
                     help="QK RMS-norm + RoPE (pha_qk_norm_rope) instead of RoPE alone")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward (pha_attn_bwd + pha_rope_bwd)")
     ap.add_argument("--aux-v", action="store_true",
                     help="add a value embedding to v inside attention (pha_attn_fwd_aux_v)")
     ap.add_argument("--oracle-tokens", type=int, default=16384)
@@ -276,6 +279,32 @@ def main():
 
     elapsed_ms = pdist.max_over_ranks(dist, elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
+
+    # ---- backward (optional): gradients of the step for a fixed upstream gradient
+    bwd = None
+    if args.backward:
+        g_up = torch.randn(tuple(q.shape), generator=torch.Generator().manual_seed(11)).to(q.dtype).to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        for _ in range(3):
+            step.attn_bwd(q, k, v, g_up, cu, dq, dk, dv)
+            step.rope_bwd(dq, dk, pos)
+        torch.cuda.synchronize(dev)
+        nb = max(3, min(args.steps, 20))
+        ba, bm, bb = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        att = 0.0
+        pdist.barrier(dist)
+        ba.record(stream)
+        for _ in range(nb):
+            step.attn_bwd(q, k, v, g_up, cu, dq, dk, dv)
+            step.rope_bwd(dq, dk, pos)
+        bb.record(stream)
+        torch.cuda.synchronize(dev)
+        b_ms = pdist.max_over_ranks(dist, ba.elapsed_time(bb) / nb, dev)
+        bwd_flops = 2.5 * attn_flops(w)
+        bwd = {"ms": b_ms, "steps": nb, "flops": bwd_flops,
+               "tflops": bwd_flops * world / (b_ms * 1e-3) / 1e12,
+               "kernels": "dq (query-major) + dk/dv (key-major) on CUDA cores, then pha_rope_bwd",
+               "flop_count": "2.5 x the forward's causal-counted FLOPs (S, dP, dV, dK, dQ)"}
 
     # ---- end to end through the public API with host buffers
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "cu_seqlens", "positions")}
@@ -367,6 +396,8 @@ def main():
         "work_items": n_items,
         "clocks": clk,
     }
+    if bwd is not None:
+        line["backward"] = bwd
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, s, thr = time_oracle(w, args.oracle_tokens, args.qk_norm)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",

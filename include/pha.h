@@ -175,6 +175,49 @@ pha_status pha_attn_fwd_aux_v(const void* q, const void* k, const void* v, const
                               pha_stream_t stream);
 
 /*
+ * pha_rope_bwd -- backward of pha_rope: the gradients with respect to the unrotated q and k, from
+ *   the gradients with respect to the rotated ones (in place). The rotation of each pair is
+ *   orthogonal, so its gradient is the transposed rotation, i.e. the rotation by -angle
+ *   (the paired-head page's note that the backward of its rotary kernel uses the same PAIRED
+ *   index branch: "modded-nanogpt Paired Head Attention record", section "4. interleave index in
+ *   the Triton kernel"). Arguments, layouts, rounding and errors: as pha_rope, with dq, dk in place
+ *   of q, k. Tokens whose position lies outside the table are left unchanged.
+ */
+pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* sin_tab,
+                        int tab_rows, int tab_width, const int32_t* positions, int total_tokens,
+                        int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                        int stagger_offset, pha_stream_t stream);
+
+/*
+ * pha_attn_bwd_workspace_bytes -- device scratch pha_attn_bwd needs: float[total_tokens][n_heads]
+ *   (the row sums D_i = sum_j P_ij dP_ij), rounded up to 256 bytes. 0 for invalid arguments.
+ */
+size_t pha_attn_bwd_workspace_bytes(int total_tokens, int n_heads);
+
+/*
+ * pha_attn_bwd -- backward of pha_attn_fwd: dq, dk, dv for the upstream gradient dout.
+ *   With P the forward's attention weights, P_ij = exp(scale q_i.k_j - lse_i) over the visible
+ *   keys (recomputed from q, k and the forward's lse; nothing else is saved):
+ *     dP_ij = dout_i . v_j,  D_i = sum_j P_ij dP_ij,  dS_ij = P_ij (dP_ij - D_i),
+ *     dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i.
+ *   q, k, v, cu_seqlens, batch, max_len, total_tokens, heads, head_dim, dtype, causal, window,
+ *   paired, scale: exactly as given to the forward (the paired path uses the same slot view and
+ *   doubled documents). lse: the forward's float[total_tokens][n_heads] (required). dout: like o.
+ *   dq: like q; dk, dv: like k, v (all written; rows outside every document get zeros).
+ *   workspace: at least pha_attn_bwd_workspace_bytes(total_tokens, n_heads), 16-byte aligned.
+ *   Arithmetic: float32 on CUDA cores (one warp per query row for dq, one per key row for dk and
+ *   dv, no atomics); dtype bf16 or f32, head_dim <= 128.
+ *   Errors: as pha_attn_fwd (PHA_ERR_INVALID, PHA_ERR_UNSUPPORTED for head_dim > 128 and for
+ *   non-causal windows, PHA_ERR_WORKSPACE); lse NULL with total_tokens > 0: PHA_ERR_INVALID.
+ */
+pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const float* lse,
+                        const void* dout, const int32_t* cu_seqlens, int batch, int max_len,
+                        int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                        pha_dtype dtype, int causal, int window, int paired, float scale, void* dq,
+                        void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                        pha_stream_t stream);
+
+/*
  * pha_attn_status -- synchronise `stream` and read the device-side status that the last
  * pha_attn_fwd on this workspace recorded: 0 = fine; 1 = cu_seqlens malformed (decreasing,
  * negative start, beyond total_tokens, or a document longer than max_len); 2 = more work

@@ -66,6 +66,17 @@ cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin
                         int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,
                         cudaStream_t stream);
 
+// Backward of RoPE: the rotation by -angle, in place on the gradients of q and k.
+cudaError_t launch_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* sin_tab,
+                            int tab_rows, int tab_width, const int32_t* positions, int total_tokens,
+                            int n_heads, int n_kv_heads, int head_dim, int is_bf16, int paired,
+                            int stagger_offset, cudaStream_t stream);
+
+// Backward of attention: dq, dk, dv (same layouts and dtype as q, k, v) for the upstream gradient
+// dout (layout of o); dsum is float[slots][heads] scratch (D_i). Needs p.lse.
+cudaError_t launch_attn_bwd(const AttnProblem& p, const void* dout, float* dsum, void* dq, void* dk,
+                            void* dv, int is_bf16, cudaStream_t stream);
+
 // RoPE preceded by the QK RMS-norm of every head row (weights may be NULL = ones).
 cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
                                 float eps, const float* cos_tab, const float* sin_tab,

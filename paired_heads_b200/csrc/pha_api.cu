@@ -133,6 +133,82 @@ pha_status pha_qk_norm_rope(void* q, void* k, const float* q_weight, const float
                : PHA_ERR_CUDA;
 }
 
+pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* sin_tab,
+                        int tab_rows, int tab_width, const int32_t* positions, int total_tokens,
+                        int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                        int stagger_offset, pha_stream_t stream) {
+    // the same arguments and checks as pha_rope
+    if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
+    const int span = dtype == PHA_BF16 ? 16 : 8;
+    if (tab_rows < 0 || total_tokens < 0 || n_heads <= 0 || n_kv_heads < 0 || head_dim <= 0 ||
+        head_dim % span != 0 || (paired != 0 && paired != 1))
+        return PHA_ERR_INVALID;
+    if (total_tokens > 0 &&
+        (!dq || !aligned16(dq) || (n_kv_heads > 0 && (!dk || !aligned16(dk))) || !cos_tab ||
+         !sin_tab || !aligned16(cos_tab) || !aligned16(sin_tab) || !positions))
+        return PHA_ERR_INVALID;
+    if (!paired && (tab_width != head_dim || stagger_offset != 0)) return PHA_ERR_INVALID;
+    if (paired && (tab_width != 2 * head_dim ||
+                   (stagger_offset != 0 && stagger_offset != head_dim)))
+        return PHA_ERR_INVALID;
+    if (total_tokens == 0) return PHA_OK;
+    return launch_rope_bwd(dq, dk, cos_tab, sin_tab, tab_rows, tab_width, positions, total_tokens,
+                           n_heads, n_kv_heads, head_dim, dtype == PHA_BF16, paired, stagger_offset,
+                           stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
+size_t pha_attn_bwd_workspace_bytes(int total_tokens, int n_heads) {
+    if (total_tokens < 0 || n_heads <= 0) return 0;
+    return (static_cast<size_t>(total_tokens) * n_heads * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const float* lse,
+                        const void* dout, const int32_t* cu_seqlens, int batch, int max_len,
+                        int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                        pha_dtype dtype, int causal, int window, int paired, float scale, void* dq,
+                        void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                        pha_stream_t stream) {
+    if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
+    const bool have = total_tokens > 0;
+    if ((have && (!q || !k || !v || !lse || !dout || !dq || !dk || !dv || !aligned16(q) ||
+                  !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+                  !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))) ||
+        !cu_seqlens || batch <= 0 || max_len < 0 || total_tokens < 0 ||
+        total_tokens > (1 << 29) || n_heads <= 0 || n_kv_heads <= 0 || n_heads > 4096 ||
+        n_heads % n_kv_heads != 0 || head_dim <= 0 || (causal != 0 && causal != 1) ||
+        (paired != 0 && paired != 1) || !(scale == scale))
+        return PHA_ERR_INVALID;
+    if (paired && ((n_heads & 1) || (n_kv_heads & 1))) return PHA_ERR_INVALID;
+    if (!causal && window > 0) return PHA_ERR_UNSUPPORTED;
+    if (head_dim > 128) return PHA_ERR_UNSUPPORTED;
+    const size_t need = pha_attn_bwd_workspace_bytes(total_tokens, n_heads);
+    if (have && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) || workspace_bytes < need))
+        return PHA_ERR_WORKSPACE;
+    if (!have) return PHA_OK;
+    AttnProblem p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.cu_seqlens = cu_seqlens;
+    p.batch = batch;
+    p.max_len = max_len;
+    p.total_tokens = total_tokens;
+    p.slot_mult = paired ? 2 : 1;
+    p.heads = paired ? n_heads / 2 : n_heads;
+    p.kv_heads = paired ? n_kv_heads / 2 : n_kv_heads;
+    p.head_dim = head_dim;
+    p.causal = causal;
+    p.window = window > 0 ? window : 0;
+    p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
+    p.lse = const_cast<float*>(lse);
+    return launch_attn_bwd(p, dout, static_cast<float*>(workspace), dq, dk, dv, dtype == PHA_BF16,
+                           stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
 size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired) {
     (void)head_dim;
     if (batch <= 0 || max_len < 0 || n_heads <= 0 || (paired && (n_heads & 1))) return 0;

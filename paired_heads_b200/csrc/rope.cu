@@ -182,7 +182,9 @@ constexpr int kRopeBatch = 4;
 template <typename T, bool NORM>
 constexpr int rope_min_blocks() { return (sizeof(T) == 2 && !NORM) ? 4 : 3; }
 
-template <typename T, bool NORM>
+// NEG: the backward of RoPE (the gradient with respect to the input is the transposed rotation,
+// i.e. the rotation by -angle): the sines enter negated, which is exact.
+template <typename T, bool NORM, bool NEG = false>
 __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel(T* __restrict__ q, T* __restrict__ k,
                                                    const float* __restrict__ cos_tab,
                                                    const float* __restrict__ sin_tab,
@@ -219,7 +221,8 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
                 const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col0 + e));
                 const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col0 + e));
                 cu[e] = cv.x; cu[e + 1] = cv.y; cu[e + 2] = cv.z; cu[e + 3] = cv.w;
-                su[e] = sv.x; su[e + 1] = sv.y; su[e + 2] = sv.z; su[e + 3] = sv.w;
+                su[e] = NEG ? -sv.x : sv.x; su[e + 1] = NEG ? -sv.y : sv.y;
+                su[e + 2] = NEG ? -sv.z : sv.z; su[e + 3] = NEG ? -sv.w : sv.w;
             }
         }
         // NORM: a lane's chunks always sit at element offset (lane % cph) * E of their head row
@@ -294,7 +297,8 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
                         const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col + e));
                         const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col + e));
                         c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
-                        s[e] = sv.x; s[e + 1] = sv.y; s[e + 2] = sv.z; s[e + 3] = sv.w;
+                        s[e] = NEG ? -sv.x : sv.x; s[e + 1] = NEG ? -sv.y : sv.y;
+                        s[e + 2] = NEG ? -sv.z : sv.z; s[e + 3] = NEG ? -sv.w : sv.w;
                     }
                 }
                 // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign
@@ -318,7 +322,7 @@ cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int hea
     return cudaGetLastError();
 }
 
-template <bool NORM>
+template <bool NORM, bool NEG = false>
 static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, const float* sin_tab,
                                     int tab_rows, int tab_width, const int32_t* positions,
                                     int total_tokens, int n_heads, int n_kv_heads, int head_dim,
@@ -330,12 +334,12 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
     const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
     const unsigned blocks = static_cast<unsigned>(blocks64 < (1 << 30) ? blocks64 : (1 << 30));
     if (is_bf16)
-        rope_kernel<__nv_bfloat16, NORM><<<blocks, threads, 0, stream>>>(
+        rope_kernel<__nv_bfloat16, NORM, NEG><<<blocks, threads, 0, stream>>>(
             static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), cos_tab, sin_tab,
             tab_rows, tab_width, positions, total_tokens, n_heads, n_kv_heads, head_dim, paired,
             stagger_offset, q_weight, k_weight, eps);
     else
-        rope_kernel<float, NORM><<<blocks, threads, 0, stream>>>(
+        rope_kernel<float, NORM, NEG><<<blocks, threads, 0, stream>>>(
             static_cast<float*>(q), static_cast<float*>(k), cos_tab, sin_tab, tab_rows, tab_width,
             positions, total_tokens, n_heads, n_kv_heads, head_dim, paired, stagger_offset,
             q_weight, k_weight, eps);
@@ -349,6 +353,15 @@ cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin
     return launch_rope_impl<false>(q, k, cos_tab, sin_tab, tab_rows, tab_width, positions,
                                    total_tokens, n_heads, n_kv_heads, head_dim, is_bf16, paired,
                                    stagger_offset, nullptr, nullptr, 0.f, stream);
+}
+
+cudaError_t launch_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* sin_tab,
+                            int tab_rows, int tab_width, const int32_t* positions, int total_tokens,
+                            int n_heads, int n_kv_heads, int head_dim, int is_bf16, int paired,
+                            int stagger_offset, cudaStream_t stream) {
+    return launch_rope_impl<false, true>(dq, dk, cos_tab, sin_tab, tab_rows, tab_width, positions,
+                                         total_tokens, n_heads, n_kv_heads, head_dim, is_bf16,
+                                         paired, stagger_offset, nullptr, nullptr, 0.f, stream);
 }
 
 cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,

@@ -50,10 +50,16 @@ _lib.pha_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i
                                       ctypes.c_float, _p, _p, _p]
 _lib.pha_attn_fwd_aux_v.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                     ctypes.c_float, _p, _p, _p, _sz, _p]
+_lib.pha_rope_bwd.argtypes = [_p, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.pha_attn_bwd_workspace_bytes.argtypes = [_i, _i]
+_lib.pha_attn_bwd_workspace_bytes.restype = _sz
+_lib.pha_attn_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                              ctypes.c_float, _p, _p, _p, _p, _sz, _p]
 _lib.pha_qk_norm_rope.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _p, _i, _i, _p, _i, _i, _i,
                                   _i, _i, _i, _i, _p]
 for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status",
-           "pha_attn_fwd_noalloc", "pha_qk_norm_rope", "pha_attn_fwd_aux_v"):
+           "pha_attn_fwd_noalloc", "pha_qk_norm_rope", "pha_attn_fwd_aux_v", "pha_rope_bwd",
+           "pha_attn_bwd"):
     getattr(_lib, _f).restype = _i
 
 
@@ -145,6 +151,45 @@ def pha_qk_norm_rope(q, k, cos_tab, sin_tab, positions, q_weight=None, k_weight=
                                  _ptr(cos_tab), _ptr(sin_tab), tab_rows, tab_width, _ptr(positions),
                                  total_tokens, n_heads, n_kv_heads, head_dim, dtype, int(paired),
                                  stagger_offset, _stream(stream, q)))
+
+
+def pha_rope_bwd(dq, dk, cos_tab, sin_tab, positions, paired: bool = False, stagger_offset: int = 0,
+                 stream=None, *, tab_rows=None, tab_width=None, total_tokens=None, n_heads=None,
+                 n_kv_heads=None, head_dim=None, dtype=None):
+    """In place: gradients with respect to the rotated q, k -> with respect to the unrotated ones."""
+    if total_tokens is None:
+        total_tokens, n_heads, head_dim = dq.shape
+        n_kv_heads = 0 if dk is None else dk.shape[1]
+        tab_rows, tab_width = cos_tab.shape
+        dtype = _dtype_code(dq)
+    _check("pha_rope_bwd", _lib.pha_rope_bwd(_ptr(dq), _ptr(dk), _ptr(cos_tab), _ptr(sin_tab),
+                                             tab_rows, tab_width, _ptr(positions), total_tokens,
+                                             n_heads, n_kv_heads, head_dim, dtype, int(paired),
+                                             stagger_offset, _stream(stream, dq)))
+
+
+def pha_attn_bwd_workspace_bytes(total_tokens: int, n_heads: int) -> int:
+    return int(_lib.pha_attn_bwd_workspace_bytes(total_tokens, n_heads))
+
+
+def pha_attn_bwd(q, k, v, lse, dout, cu_seqlens, max_len: int, dq, dk, dv, workspace, *,
+                 causal: bool = True, window: int = 0, paired: bool = False, scale: float = 0.0,
+                 stream=None, batch=None, total_tokens=None, n_heads=None, n_kv_heads=None,
+                 head_dim=None, dtype=None, workspace_bytes=None):
+    """Backward of pha_attn_fwd: writes dq, dk, dv for the upstream gradient dout."""
+    if total_tokens is None:
+        total_tokens, n_heads, head_dim = q.shape
+        n_kv_heads = k.shape[1]
+        batch = cu_seqlens.shape[0] - 1
+        dtype = _dtype_code(q)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pha_attn_bwd",
+           _lib.pha_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(dout), _ptr(cu_seqlens),
+                             batch, max_len, total_tokens, n_heads, n_kv_heads, head_dim, dtype,
+                             int(causal), int(window), int(paired), float(scale), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), workspace_bytes,
+                             _stream(stream, q)))
 
 
 def pha_attn_workspace_bytes(batch: int, max_len: int, n_heads: int, head_dim: int,

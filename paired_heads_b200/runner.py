@@ -85,6 +85,22 @@ class AttentionStep:
                                paired=self.s.paired, scale=self.s.scale, stream=stream)
         return self.o, self.lse
 
+    def rope_bwd(self, dq, dk, positions, stream=None):
+        """In place: gradients w.r.t. the rotated q, k -> w.r.t. the unrotated q, k."""
+        pha.pha_rope_bwd(dq, dk, self.cos_tab, self.sin_tab, positions, paired=self.s.paired,
+                         stagger_offset=self.stagger_offset, stream=stream)
+
+    def attn_bwd(self, q, k, v, dout, cu_seqlens, dq, dk, dv, stream=None):
+        """Backward of the last attention call's shape: dq, dk, dv for dout, using self.lse (the
+        forward must have run on the same q, k, v). Returns (dq, dk, dv)."""
+        if getattr(self, "bwd_workspace", None) is None:
+            nbytes = pha.pha_attn_bwd_workspace_bytes(self.s.total_tokens, self.s.n_heads)
+            self.bwd_workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        pha.pha_attn_bwd(q, k, v, self.lse, dout, cu_seqlens, self.s.max_len, dq, dk, dv,
+                         self.bwd_workspace, causal=self.s.causal, window=self.s.window,
+                         paired=self.s.paired, scale=self.s.scale, stream=stream)
+        return dq, dk, dv
+
     def __call__(self, q, k, v, cu_seqlens, positions, stream=None):
         """RoPE q and k in place, then attention. Returns (o, lse) (buffers owned by the step)."""
         self.rope(q, k, positions, stream)

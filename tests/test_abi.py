@@ -27,9 +27,10 @@ def _declared():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["pha_attn_fwd", "pha_attn_fwd_aux_v", "pha_attn_fwd_noalloc",
-                           "pha_attn_status", "pha_attn_workspace_bytes", "pha_qk_norm_rope",
-                           "pha_rope", "pha_rope_tables", "pha_status_string"]
+    assert _declared() == ["pha_attn_bwd", "pha_attn_bwd_workspace_bytes", "pha_attn_fwd",
+                           "pha_attn_fwd_aux_v", "pha_attn_fwd_noalloc", "pha_attn_status",
+                           "pha_attn_workspace_bytes", "pha_qk_norm_rope", "pha_rope",
+                           "pha_rope_bwd", "pha_rope_tables", "pha_status_string"]
 
 
 def test_library_exports_every_declared_symbol(pha):
@@ -198,3 +199,46 @@ def _attn_aux(pha, **kw):
 ])
 def test_attn_aux_v_argument_errors(pha, kw, code):
     assert _attn_aux(pha, **kw) == code
+
+
+def _attn_bwd(pha, **kw):
+    args = dict(q=A, k=A, v=A, lse=A, g=A, cu=A, batch=1, max_len=128, total=128, H=4, Hkv=4,
+                hd=64, dtype=pha.PHA_BF16, causal=1, window=0, paired=0, scale=0.0, dq=A, dk=A,
+                dv=A, ws=A, ws_bytes=10)
+    args.update(kw)
+    return pha.library().pha_attn_bwd(
+        args["q"], args["k"], args["v"], args["lse"], args["g"], args["cu"], args["batch"],
+        args["max_len"], args["total"], args["H"], args["Hkv"], args["hd"], args["dtype"],
+        args["causal"], args["window"], args["paired"], ctypes.c_float(args["scale"]), args["dq"],
+        args["dk"], args["dv"], args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(), -3),                              # valid: only the (too small) workspace stops it
+    (dict(lse=None), -1),
+    (dict(lse=A + 2), -1),
+    (dict(g=None), -1),
+    (dict(dk=MIS), -1),
+    (dict(H=6, Hkv=4), -1),
+    (dict(H=6, Hkv=3, paired=1), -1),
+    (dict(causal=0, window=16), -2),
+    (dict(hd=160), -2),
+    (dict(dtype=7), -1),
+    (dict(total=0, ws=None), 0),               # nothing to do
+])
+def test_attn_bwd_argument_errors(pha, kw, code):
+    assert _attn_bwd(pha, **kw) == code
+
+
+def test_attn_bwd_workspace_bytes(pha):
+    assert pha.pha_attn_bwd_workspace_bytes(65536, 6) == 65536 * 6 * 4
+    assert pha.pha_attn_bwd_workspace_bytes(3, 1) == 256
+    assert pha.pha_attn_bwd_workspace_bytes(-1, 2) == 0
+
+
+def test_rope_bwd_argument_errors(pha):
+    lib = pha.library()
+    args = [A, A, A, A, 16, 64, A, 4, 2, 2, 64, pha.PHA_BF16, 0, 0, None]
+    assert lib.pha_rope_bwd(*args[:5], 128, *args[6:]) == -1        # table width
+    assert lib.pha_rope_bwd(MIS, *args[1:]) == -1
+    assert lib.pha_rope_bwd(*args[:7], 0, *args[8:]) == 0           # no tokens
