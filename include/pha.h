@@ -189,30 +189,40 @@ pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* s
                         int stagger_offset, pha_stream_t stream);
 
 /*
- * pha_attn_bwd_workspace_bytes -- device scratch pha_attn_bwd needs: float[total_tokens][n_heads]
- *   (the row sums D_i = sum_j P_ij dP_ij), rounded up to 256 bytes. 0 for invalid arguments.
+ * pha_attn_bwd_workspace_bytes -- device scratch pha_attn_bwd needs: the forward's scheduling
+ *   area (pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired), rounded up to 256
+ *   bytes; its header is what pha_attn_status reads) followed by float[total_tokens][n_heads]
+ *   (the row sums D_i), rounded up to 256 bytes. 0 for invalid arguments.
  */
-size_t pha_attn_bwd_workspace_bytes(int total_tokens, int n_heads);
+size_t pha_attn_bwd_workspace_bytes(int batch, int max_len, int total_tokens, int n_heads,
+                                    int head_dim, int paired);
 
 /*
  * pha_attn_bwd -- backward of pha_attn_fwd: dq, dk, dv for the upstream gradient dout.
  *   With P the forward's attention weights, P_ij = exp(scale q_i.k_j - lse_i) over the visible
- *   keys (recomputed from q, k and the forward's lse; nothing else is saved):
- *     dP_ij = dout_i . v_j,  D_i = sum_j P_ij dP_ij,  dS_ij = P_ij (dP_ij - D_i),
- *     dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i.
+ *   keys (recomputed from q, k and the forward's lse; no score matrix is saved):
+ *     dP_ij = dout_i . v_j,  D_i = sum_j P_ij dP_ij = dout_i . o_i,  dS_ij = P_ij (dP_ij - D_i),
+ *     dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i
+ *   (FlashAttention's backward; "Training an LLM from scratch (part 2)", section "4. GQA &
+ *   FlashAttention"). D is taken from the forward's output o, as stored (bf16 or f32).
  *   q, k, v, cu_seqlens, batch, max_len, total_tokens, heads, head_dim, dtype, causal, window,
  *   paired, scale: exactly as given to the forward (the paired path uses the same slot view and
- *   doubled documents). lse: the forward's float[total_tokens][n_heads] (required). dout: like o.
- *   dq: like q; dk, dv: like k, v (all written; rows outside every document get zeros).
- *   workspace: at least pha_attn_bwd_workspace_bytes(total_tokens, n_heads), 16-byte aligned.
- *   Arithmetic: float32 on CUDA cores (one warp per query row for dq, one per key row for dk and
- *   dv, no atomics); dtype bf16 or f32, head_dim <= 128.
+ *   doubled documents). o, lse: the forward's outputs (lse float[total_tokens][n_heads]; both
+ *   required). dout: like o. dq: like q; dk, dv: like k, v (all written; rows outside every
+ *   document get zeros). workspace: at least pha_attn_bwd_workspace_bytes(...), 16-byte aligned;
+ *   pha_attn_status(workspace) reports the device status afterwards (malformed cu_seqlens, a
+ *   kernel wait that gave up).
+ *   Arithmetic: bf16 with causal 1 <= window <= 128 and head_dim 64 or 128 (the band case): the
+ *   tensor cores (tcgen05, bf16 operands with P and dS rounded to bf16, float32 accumulation in
+ *   TMEM), one kernel for dq and one for dk, dv; otherwise float32 on CUDA cores (dtype bf16 or
+ *   f32, head_dim <= 128). No atomics on either path.
  *   Errors: as pha_attn_fwd (PHA_ERR_INVALID, PHA_ERR_UNSUPPORTED for head_dim > 128 and for
- *   non-causal windows, PHA_ERR_WORKSPACE); lse NULL with total_tokens > 0: PHA_ERR_INVALID.
+ *   non-causal windows, PHA_ERR_WORKSPACE); o or lse NULL with total_tokens > 0: PHA_ERR_INVALID.
+ *   With total_tokens == 0 the call returns PHA_OK after checking its arguments, launching nothing.
  */
-pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const float* lse,
-                        const void* dout, const int32_t* cu_seqlens, int batch, int max_len,
-                        int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, const int32_t* cu_seqlens, int batch,
+                        int max_len, int total_tokens, int n_heads, int n_kv_heads, int head_dim,
                         pha_dtype dtype, int causal, int window, int paired, float scale, void* dq,
                         void* dk, void* dv, void* workspace, size_t workspace_bytes,
                         pha_stream_t stream);

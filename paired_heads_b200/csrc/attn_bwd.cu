@@ -1,20 +1,21 @@
-// attn_bwd.cu -- backward of the varlen (paired-head) attention forward: dq, dk, dv for an upstream
-// gradient dO, on CUDA cores in float32.
+// attn_bwd.cu -- backward of the varlen (paired-head) attention forward on CUDA cores in float32
+// (every shape), and the two small kernels both backward paths share.
 //
 // The gradients through the row softmax (with P the attention weights of the forward,
 // P_ij = exp(scale q_i . k_j - lse_i) over the visible keys):
 //   dP_ij = dO_i . v_j,  D_i = sum_j P_ij dP_ij,  dS_ij = P_ij (dP_ij - D_i),
 //   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dO_i.
 // P is recomputed from q, k and the forward's lse (FlashAttention's recomputation: "Training an
-// LLM from scratch (part 2)", section "4. GQA & FlashAttention" -- no score matrix is stored).
-// The paired-head variant is the same slot view of the buffers and the same doubled documents as
-// the forward ("modded-nanogpt Paired Head Attention record" page, sections "3. the paired branch
-// of the forward pass" and "sequence length and window handling").
+// LLM from scratch (part 2)", section "4. GQA & FlashAttention" -- no score matrix is stored), and
+// D_i = sum_j P_ij (dO_i . v_j) = dO_i . O_i is taken from the forward's output O (one pass over
+// O and dO, attn_bwd_dsum_kernel). The paired-head variant is the same slot view of the buffers
+// and the same doubled documents as the forward ("modded-nanogpt Paired Head Attention record"
+// page, sections "3. the paired branch of the forward pass" and "sequence length and window
+// handling").
 //
-// Two kernels, no atomics, each on blocks of 32 consecutive rows of one head:
+// CUDA-core path: two kernels, no atomics, each on blocks of 32 consecutive rows of one head:
 //   dq   (query-major): 32 query slots of one head; the keys they see are staged 32 at a time in
-//        shared memory (float32). Pass 1 gives D_i, pass 2 accumulates dq_i; D_i is stored for the
-//        second kernel.
+//        shared memory (float32), accumulating dq_i.
 //   dkdv (key-major):   32 key slots of one kv head; for each query head of the group the queries
 //        that see them are staged 32 at a time (q, dO, lse, D), accumulating dk_j and dv_j.
 // Eight consecutive lanes share a row. Lane r of the eight holds the float4 chunks r, r + 8, ... of
@@ -142,7 +143,7 @@ __device__ __forceinline__ void store_row(T* dst, const float4 (&x)[NC], int hd,
 template <int HP, typename T>
 __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dq_kernel(AttnProblem p,
                                                                    const T* __restrict__ dout,
-                                                                   float* __restrict__ dsum,
+                                                                   const float* __restrict__ dsum,
                                                                    T* __restrict__ dq) {
     constexpr int NC = HP / (4 * kLanesPerRow);
     extern __shared__ float4 bsm4[];
@@ -189,8 +190,8 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dq_kernel(AttnProblem p,
     const T* kg = static_cast<const T*>(p.k) + static_cast<int64_t>(g) * hd;
     const T* vg = static_cast<const T*>(p.v) + static_cast<int64_t>(g) * hd;
     const int64_t kstride = static_cast<int64_t>(Hkv) * hd;
-    float d = 0.f;
-    for (int pass = 0; pass < 2; ++pass) {
+    const float d = in_doc ? dsum[row] : 0.f;
+    {
         for (long long c0 = J0; c0 < J1; c0 += kStage) {
             const int n = static_cast<int>(J1 - c0 < kStage ? J1 - c0 : kStage);
             __syncthreads();  // every warp is done with the previous chunk
@@ -212,20 +213,13 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dq_kernel(AttnProblem p,
                 }
                 group_sum2(s, dp);
                 const float pij = (j >= j0 && j < j1) ? exp2f(fmaf(s, scale2, -lse2)) : 0.f;
-                if (pass == 0) {
-                    d = fmaf(pij, dp, d);
-                } else {
-                    const float ds = pij * (dp - d) * p.scale;
+                const float ds = pij * (dp - d) * p.scale;
 #pragma unroll
-                    for (int t = 0; t < NC; ++t) axpy4(acc[t], ds, kk[t]);
-                }
+                for (int t = 0; t < NC; ++t) axpy4(acc[t], ds, kk[t]);
             }
         }
     }
-    if (i < slots) {
-        store_row<NC>(dq + row * hd, acc, hd, r8);
-        if (r8 == 0) dsum[row] = d;
-    }
+    if (i < slots) store_row<NC>(dq + row * hd, acc, hd, r8);
 }
 
 template <int HP, typename T>
@@ -323,8 +317,73 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(AttnProblem 
     }
 }
 
+// D_i = dO_i . O_i for every row (slot, head) of the slot view: 8 lanes per row, VEC elements per
+// load (rows are 16-byte aligned when VEC > 1).
+template <typename T, int VEC>
+__global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const T* __restrict__ o,
+                                                            const T* __restrict__ dout,
+                                                            float* __restrict__ dsum, int64_t rows,
+                                                            int hd) {
+    const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t r = gid / kLanesPerRow;
+    const int r8 = static_cast<int>(gid % kLanesPerRow);
+    float acc = 0.f, acc2 = 0.f;
+    if (r < rows) {
+        const T* orow = o + r * hd;
+        const T* grow = dout + r * hd;
+        for (int e = r8 * VEC; e < hd; e += kLanesPerRow * VEC) {
+            if (VEC == 1) {
+                acc = fmaf(ld(orow + e), ld(grow + e), acc);
+            } else {
+                const uint4 a = __ldg(reinterpret_cast<const uint4*>(orow + e));
+                const uint4 b = __ldg(reinterpret_cast<const uint4*>(grow + e));
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    if (sizeof(T) == 2) {
+                        acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
+                        acc2 = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u),
+                                    __uint_as_float(bw[w] & 0xFFFF0000u), acc2);
+                    } else {
+                        acc = fmaf(__uint_as_float(aw[w]), __uint_as_float(bw[w]), acc);
+                    }
+                }
+            }
+        }
+    }
+    acc += acc2;
+    float unused = 0.f;
+    group_sum2(acc, unused);
+    if (r < rows && r8 == 0) dsum[r] = acc;
+}
+
+// Zeros rows [0, cu[0] * mult) and [cu[batch] * mult, slots) (outside every document) of dq, dk,
+// dv (bf16, row widths multiples of 8 elements).
+__global__ void __launch_bounds__(256) attn_bwd_zero_outside_kernel(AttnProblem p,
+                                                                    __nv_bfloat16* dq,
+                                                                    __nv_bfloat16* dk,
+                                                                    __nv_bfloat16* dv) {
+    const int64_t slots = static_cast<int64_t>(p.total_tokens) * p.slot_mult;
+    const int64_t head = min(static_cast<int64_t>(p.cu_seqlens[0]) * p.slot_mult, slots);
+    const int64_t tail = max(min(static_cast<int64_t>(p.cu_seqlens[p.batch]) * p.slot_mult, slots),
+                             head);
+    const int64_t wq = static_cast<int64_t>(p.heads) * p.head_dim / 8;     // 16-byte units
+    const int64_t wk = static_cast<int64_t>(p.kv_heads) * p.head_dim / 8;
+    const int64_t rows = head + (slots - tail);
+    const int64_t n = rows * (wq + 2 * wk);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < n;
+         x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t rr = x / (wq + 2 * wk), c = x % (wq + 2 * wk);
+        const int64_t slot = rr < head ? rr : tail + (rr - head);
+        if (c < wq) reinterpret_cast<uint4*>(dq)[slot * wq + c] = z;
+        else if (c < wq + wk) reinterpret_cast<uint4*>(dk)[slot * wk + (c - wq)] = z;
+        else reinterpret_cast<uint4*>(dv)[slot * wk + (c - wq - wk)] = z;
+    }
+}
+
 template <int HP, typename T>
-void launch_bwd_hp(const AttnProblem& p, const T* dout, float* dsum, T* dq, T* dk, T* dv,
+void launch_bwd_hp(const AttnProblem& p, const T* dout, const float* dsum, T* dq, T* dk, T* dv,
                    unsigned tiles, cudaStream_t stream) {
     const size_t smem_dq = 2 * static_cast<size_t>(kStage) * HP * sizeof(float);
     const size_t smem_kv = smem_dq + 2 * kStage * sizeof(float);
@@ -334,7 +393,7 @@ void launch_bwd_hp(const AttnProblem& p, const T* dout, float* dsum, T* dq, T* d
 }
 
 template <typename T>
-void launch_bwd_t(const AttnProblem& p, const void* dout, float* dsum, void* dq, void* dk, void* dv,
+void launch_bwd_t(const AttnProblem& p, const void* dout, const float* dsum, void* dq, void* dk, void* dv,
                   unsigned tiles, cudaStream_t stream) {
     const T* go = static_cast<const T*>(dout);
     T *a = static_cast<T*>(dq), *b = static_cast<T*>(dk), *c = static_cast<T*>(dv);
@@ -345,8 +404,37 @@ void launch_bwd_t(const AttnProblem& p, const void* dout, float* dsum, void* dq,
 
 }  // namespace
 
-cudaError_t launch_attn_bwd(const AttnProblem& p, const void* dout, float* dsum, void* dq, void* dk,
-                            void* dv, int is_bf16, cudaStream_t stream) {
+cudaError_t launch_attn_bwd_dsum(const AttnProblem& p, const void* o, const void* dout,
+                                 float* dsum, int is_bf16, cudaStream_t stream) {
+    const int64_t rows = static_cast<int64_t>(p.total_tokens) * p.slot_mult * p.heads;
+    if (rows == 0) return cudaSuccess;
+    const int hd = p.head_dim;
+    const unsigned blocks = static_cast<unsigned>((rows * kLanesPerRow + 255) / 256);
+    if (is_bf16) {
+        const auto* a = static_cast<const __nv_bfloat16*>(o);
+        const auto* b = static_cast<const __nv_bfloat16*>(dout);
+        if (hd % 8 == 0) attn_bwd_dsum_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, stream>>>(a, b, dsum, rows, hd);
+        else attn_bwd_dsum_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, stream>>>(a, b, dsum, rows, hd);
+    } else {
+        const auto* a = static_cast<const float*>(o);
+        const auto* b = static_cast<const float*>(dout);
+        if (hd % 4 == 0) attn_bwd_dsum_kernel<float, 4><<<blocks, 256, 0, stream>>>(a, b, dsum, rows, hd);
+        else attn_bwd_dsum_kernel<float, 1><<<blocks, 256, 0, stream>>>(a, b, dsum, rows, hd);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_zero_outside(const AttnProblem& p, void* dq, void* dk, void* dv,
+                                         cudaStream_t stream) {
+    if (p.total_tokens == 0) return cudaSuccess;
+    attn_bwd_zero_outside_kernel<<<148, 256, 0, stream>>>(p, static_cast<__nv_bfloat16*>(dq),
+                                                          static_cast<__nv_bfloat16*>(dk),
+                                                          static_cast<__nv_bfloat16*>(dv));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd(const AttnProblem& p, const void* dout, const float* dsum, void* dq,
+                            void* dk, void* dv, int is_bf16, cudaStream_t stream) {
     const int64_t slots = static_cast<int64_t>(p.total_tokens) * p.slot_mult;
     if (slots == 0) return cudaSuccess;
     if (p.head_dim > 128) return cudaErrorInvalidValue;

@@ -1,0 +1,489 @@
+// attn_bwd_tc.cu -- backward of the band attention (causal, window <= 128 key slots, bf16,
+// head_dim 64 or 128) on the sm_100a tensor cores.
+//
+// The gradients through the row softmax, with P recomputed from q, k and the forward's lse and
+// D_i = dO_i . O_i precomputed (FlashAttention's backward: "Training an LLM from scratch (part 2)",
+// section "4. GQA & FlashAttention"):
+//   dP = dO V^T,  dS = P o (dP - D),  dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
+// Tiles of 128 slots are counted from the document start, as in the forward's band decomposition
+// ("modded-nanogpt Paired Head Attention record" page, section "sequence length and window
+// handling"): query tile j sees key tiles j - 1 and j, so key tile j is seen by query tiles j and
+// j + 1. One kernel template, two instances:
+//   key-major (dK, dV): outer tile = key tile (X = K, V), inner steps = the query tiles that see
+//     it, for every query head of its group (Y = Q, dO):  S^T = K Q^T, dP^T = V dO^T, then
+//     dV += P^T dO and dK += dS^T Q with P^T, dS^T in TMEM as the A operand.
+//   query-major (dQ): outer tile = query tile (X = Q, dO), inner steps = the key tiles it sees
+//     (Y = K, V): S = Q K^T, dP = dO V^T, then dQ += dS K.
+// In both, the 128 x 128 scores go to TMEM columns [0, 128), dP to [128, 256); the bf16 P and dS
+// overwrite the first half of each; the accumulators sit at 256 (dV or dQ) and 256 + hd (dK).
+// A tile loaded for the K-major S / dP product (rows = slots, [64-column chunks] 128-byte
+// swizzled) is the MN-major B operand of the second product as it stands.
+//
+// CTA = 6 warps, persistent, one per SM, band items in snake order:
+//   warps 0-3  elementwise: row = TMEM lane; P, dS from S, dP; the epilogue (accumulators ->
+//              bf16 -> global)
+//   warp 4     producer: X tiles (one buffer), Y tiles (two stages) by TMA; in the key-major
+//              instance also lse * log2(e) and D of the step's 128 queries into shared memory
+//   warp 5     MMA issuer, owner of the 512 TMEM columns
+// Every wait is bounded (1 s); on expiry the CTA records a status, drains its own copies and
+// MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "attn_common.cuh"
+#include "kernels.cuh"
+
+namespace pha {
+
+namespace {
+
+constexpr int kBwdTcThreads = 192;
+
+template <int HD>
+struct BwdLayout {
+    static constexpr int kChunk = 128 * 128;   // one [128 rows][64 bf16] swizzled chunk (bytes)
+    static constexpr int kTile = 128 * HD * 2;
+    static constexpr int kYStages = 2;
+    static constexpr int kOffX = 0;                                  // X0, X1
+    static constexpr int kOffY = kOffX + 2 * kTile;                  // [stage] Y0, Y1
+    static constexpr int kOffVec = kOffY + kYStages * 2 * kTile;     // [stage] lse2[128], D[128]
+    static constexpr int kOffBar = kOffVec + kYStages * 2 * 128 * 4;
+    static constexpr int kBarBytes = 256;
+    static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + slack to align to 1024
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmAcc = 256;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct BwdBars {
+    uint64_t x_full, x_empty;
+    uint64_t y_full[2], y_empty[2];
+    uint64_t s_full, p_full, m2_done, acc_full, acc_empty, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// The steps of one outer tile (u-th tile of a band item).
+struct OuterTile {
+    int row0;     // first slot of the outer tile
+    int n_sub;    // inner steps
+    int nq;       // key-major: query tiles per head (1 or 2)
+};
+
+template <bool KEYMAJOR>
+__device__ __forceinline__ OuterTile outer_tile(const BandItem& it, int u, int G) {
+    OuterTile o;
+    o.row0 = it.q0 + kBlockM * u;
+    if (KEYMAJOR) {
+        o.nq = o.row0 + kBlockM < it.doc_end ? 2 : 1;  // the diagonal query tile, then the next
+        o.n_sub = G * o.nq;
+    } else {
+        o.nq = 0;
+        o.n_sub = (u + it.hp >= 1) ? 2 : 1;  // the previous key tile (if any), then the diagonal
+    }
+    return o;
+}
+
+// Inner step s of an outer tile: the head and first slot of its Y tiles.
+template <bool KEYMAJOR>
+__device__ __forceinline__ void inner_step(const BandItem& it, const OuterTile& o, int s, int G,
+                                           int& y_head, int& y_row) {
+    if (KEYMAJOR) {
+        const int g = it.head / G;
+        y_head = g * G + s / o.nq;
+        y_row = o.row0 + kBlockM * (s % o.nq);
+    } else {
+        y_head = it.head / G;
+        y_row = o.row0 - (s + 1 < o.n_sub ? kBlockN : 0);
+    }
+}
+
+// Items of the key-major instance: one per kv head (the item of the group's first query head).
+template <bool KEYMAJOR>
+__device__ __forceinline__ bool item_used(const BandItem& it, int G) {
+    return !KEYMAJOR || it.head % G == 0;
+}
+
+template <int HD, bool KEYMAJOR>
+__global__ void __launch_bounds__(kBwdTcThreads, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_do, const AttnProblem p,
+                       const float* __restrict__ dsum, __nv_bfloat16* __restrict__ out_a,
+                       __nv_bfloat16* __restrict__ out_b, const int4* __restrict__ items,
+                       WorkspaceHeader* hdr) {
+    // out_a: dQ (query-major) or dK (key-major); out_b: dV (key-major)
+    using L = BwdLayout<HD>;
+    static_assert(sizeof(BwdBars) <= L::kBarBytes, "barrier block");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+    const uint32_t sbase = smem_u32(smem);
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + L::kOffBar);
+    float* vec = reinterpret_cast<float*>(smem + L::kOffVec);
+    volatile int* abort_flag = &bars->abort;
+    int* dev_status = &hdr->status;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (warp == 4 && lane == 0) {
+        mbar_init(&bars->x_full, 1);
+        mbar_init(&bars->x_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            // the TMA arrival, plus (key-major) the 32 producer lanes after writing lse2 / D
+            mbar_init(&bars->y_full[s], KEYMAJOR ? 33 : 1);
+            mbar_init(&bars->y_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->m2_done, 1);
+        mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->acc_empty, 128);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+    }
+    if (warp == 5) {
+        tmem_alloc(&bars->tmem_base, L::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
+    const int H = p.heads, Hkv = p.kv_heads, G = H / Hkv;
+    // X = (K, V) and Y = (Q, dO) (key-major), or the other way round
+    const CUtensorMap* mx0 = KEYMAJOR ? &tm_k : &tm_q;
+    const CUtensorMap* mx1 = KEYMAJOR ? &tm_v : &tm_do;
+    const CUtensorMap* my0 = KEYMAJOR ? &tm_q : &tm_k;
+    const CUtensorMap* my1 = KEYMAJOR ? &tm_do : &tm_v;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        uint32_t oc = 0, sc = 0;  // outer tiles / inner steps issued so far
+        bool ok = true;
+        ItemWalk wk;
+        for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+            if (!wk.has()) continue;
+            const BandItem it = decode_band(wk.cur);
+            if (!item_used<KEYMAJOR>(it, G)) continue;
+            const int x_head = KEYMAJOR ? it.head / G : it.head;
+            for (int u = 0; ok && u < it.n_qt; ++u) {
+                const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_empty, (oc & 1) ^ 1, abort_flag,
+                                                       dev_status));
+                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->x_full, 2 * L::kTile);
+                    for (int c = 0; c < HD / 64; ++c) {
+                        tma_load_2d(smem + L::kOffX + c * L::kChunk, mx0, x_head * HD + 64 * c,
+                                    o.row0, &bars->x_full);
+                        tma_load_2d(smem + L::kOffX + L::kTile + c * L::kChunk, mx1,
+                                    x_head * HD + 64 * c, o.row0, &bars->x_full);
+                    }
+                }
+                ++oc;
+                for (int s = 0; s < o.n_sub; ++s) {
+                    const uint32_t st = sc & 1;
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_empty[st], ((sc >> 1) & 1) ^ 1,
+                                                           abort_flag, dev_status));
+                    if (!ok) break;
+                    int y_head, y_row;
+                    inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&bars->y_full[st], 2 * L::kTile);
+                        uint8_t* y = smem + L::kOffY + st * 2 * L::kTile;
+                        for (int c = 0; c < HD / 64; ++c) {
+                            tma_load_2d(y + c * L::kChunk, my0, y_head * HD + 64 * c, y_row,
+                                        &bars->y_full[st]);
+                            tma_load_2d(y + L::kTile + c * L::kChunk, my1, y_head * HD + 64 * c,
+                                        y_row, &bars->y_full[st]);
+                        }
+                    }
+                    if (KEYMAJOR) {
+                        // lse * log2(e) and D of the step's queries (0 past the document end)
+                        float* l2 = vec + st * 256;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int c = 4 * lane + e, qs = y_row + c;
+                            const bool in = qs < it.doc_end;
+                            const int64_t r = static_cast<int64_t>(qs) * H + y_head;
+                            l2[c] = in ? p.lse[r] * kLog2e : 0.f;
+                            l2[128 + c] = in ? dsum[r] : 0.f;
+                        }
+                        mbar_arrive(&bars->y_full[st]);
+                    }
+                    ++sc;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            // Wait (bounded) for the copies this warp issued last into every buffer.
+            if (oc > 0) drain_wait(&bars->x_full, (oc - 1) & 1);
+            for (uint32_t n = sc > 2 ? sc - 2 : 0; n < sc; ++n)
+                drain_wait(&bars->y_full[n & 1], (n >> 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc1 = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+            constexpr uint32_t idesc2 = idesc_bf16_f32(kBlockM, HD, 0, 1);
+            const uint32_t tm_s = tmem + L::kTmS, tm_dp = tmem + L::kTmDP;
+            const uint32_t tm_acc_p = tmem + L::kTmAcc;                         // dV
+            const uint32_t tm_acc_ds = tmem + L::kTmAcc + (KEYMAJOR ? HD : 0);  // dK or dQ
+            const uint32_t x0 = sbase + L::kOffX, x1 = x0 + L::kTile;
+            uint32_t oc = 0, sc = 0;
+            bool ok = true;
+            ItemWalk wk;
+            for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+                if (!wk.has()) continue;
+                const BandItem it = decode_band(wk.cur);
+                if (!item_used<KEYMAJOR>(it, G)) continue;
+                for (int u = 0; ok && u < it.n_qt; ++u) {
+                    const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                    if (!mbar_wait(&bars->x_full, oc & 1, abort_flag, dev_status)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int s = 0; s < o.n_sub; ++s) {
+                        const uint32_t st = sc & 1;
+                        const uint32_t y0 = sbase + L::kOffY + st * 2 * L::kTile, y1 = y0 + L::kTile;
+                        if (!mbar_wait(&bars->y_full[st], (sc >> 1) & 1, abort_flag, dev_status) ||
+                            (sc > 0 && !mbar_wait(&bars->m2_done, (sc - 1) & 1, abort_flag,
+                                                  dev_status))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            umma_f16_ss(tm_s, desc_kmajor(x0, kk), desc_kmajor(y0, kk), idesc1,
+                                        kk == 0 ? 0u : 1u);
+                            umma_f16_ss(tm_dp, desc_kmajor(x1, kk), desc_kmajor(y1, kk), idesc1,
+                                        kk == 0 ? 0u : 1u);
+                        }
+                        umma_commit(&bars->s_full);
+                        if (s + 1 == o.n_sub) umma_commit(&bars->x_empty);
+                        if (!mbar_wait(&bars->p_full, sc & 1, abort_flag, dev_status) ||
+                            (s == 0 && oc > 0 &&
+                             !mbar_wait(&bars->acc_empty, (oc - 1) & 1, abort_flag, dev_status))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                            umma_f16_ts(tm_acc_ds, tm_dp + 8 * kk, desc_v(y0, kk), idesc2, acc);
+                            if (KEYMAJOR)
+                                umma_f16_ts(tm_acc_p, tm_s + 8 * kk, desc_v(y1, kk), idesc2, acc);
+                        }
+                        umma_commit(&bars->m2_done);
+                        umma_commit(&bars->y_empty[st]);
+                        if (s + 1 == o.n_sub) umma_commit(&bars->acc_full);
+                        ++sc;
+                    }
+                    ++oc;
+                }
+            }
+            // Wait (bounded) until every MMA this thread issued has finished.
+            umma_commit(&bars->drain);
+            drain_wait(&bars->drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ elementwise warpgroup
+        const int row = threadIdx.x;         // TMEM lane == row of the outer tile
+        const int r0 = warp * 32;            // first row of this warp
+        const uint32_t tm_lane = tmem + (static_cast<uint32_t>(r0) << 16);
+        const float scale_log2 = p.scale * kLog2e;
+        const int window = p.window;
+        uint32_t oc = 0, sc = 0;
+        bool ok = true;
+        ItemWalk wk;
+        for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+            if (!wk.has()) continue;
+            const BandItem it = decode_band(wk.cur);
+            if (!item_used<KEYMAJOR>(it, G)) continue;
+            for (int u = 0; ok && u < it.n_qt; ++u) {
+                const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                const int slot = o.row0 + row;  // key slot (key-major) or query slot
+                const bool valid = slot < it.doc_end;
+                float lse2 = 0.f, dd = 0.f;  // query-major: this row's lse * log2(e) and D
+                if (!KEYMAJOR && valid) {
+                    const int64_t r = static_cast<int64_t>(slot) * H + it.head;
+                    lse2 = p.lse[r] * kLog2e;
+                    dd = dsum[r];
+                }
+                for (int s = 0; s < o.n_sub; ++s) {
+                    const uint32_t st = sc & 1;
+                    int y_head, y_row;
+                    inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
+                    // visible columns [c_lo, c_hi] of this row
+                    int c_lo, c_hi;
+                    if (KEYMAJOR) {  // queries slot .. slot + window - 1, inside the document
+                        c_lo = slot - y_row;
+                        c_hi = min(slot + window - 1, it.doc_end - 1) - y_row;
+                    } else {         // keys slot - window + 1 .. slot
+                        c_lo = slot - window + 1 - y_row;
+                        c_hi = valid ? slot - y_row : c_lo - 1;
+                    }
+                    if (KEYMAJOR)
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full[st], (sc >> 1) & 1,
+                                                               abort_flag, dev_status));
+                    if (ok)
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, sc & 1, abort_flag,
+                                                               dev_status));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int w_lo = __reduce_min_sync(0xffffffffu, c_lo);
+                    const int w_hi = __reduce_max_sync(0xffffffffu, c_hi);
+                    const float* l2v = vec + st * 256;
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pk[16], dk[16];
+                        if (32 * c > w_hi || 32 * c + 31 < w_lo) {  // no row of the warp sees it
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pk[e] = dk[e] = 0u;
+                        } else {
+                            uint32_t sv[32], dv[32];
+                            tmem_ld32(tm_lane + L::kTmS + 32 * c, sv);
+                            tmem_ld32(tm_lane + L::kTmDP + 32 * c, dv);
+                            tmem_wait_ld();
+                            regs_after_wait(sv);
+                            regs_after_wait(dv);
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) {
+                                float pr[2], dr[2];
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int col = 32 * c + e + h;
+                                    float l2 = lse2, d = dd;
+                                    if (KEYMAJOR) {
+                                        l2 = l2v[col];
+                                        d = l2v[128 + col];
+                                    }
+                                    const bool vis = col >= c_lo && col <= c_hi;
+                                    const float pe = ex2(fmaf(__uint_as_float(sv[e + h]), scale_log2, -l2));
+                                    pr[h] = vis ? pe : 0.f;
+                                    dr[h] = pr[h] * (__uint_as_float(dv[e + h]) - d);
+                                }
+                                pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+                                dk[e >> 1] = pack_bf16x2(dr[0], dr[1]);
+                            }
+                        }
+                        if (KEYMAJOR) tmem_st16(tm_lane + L::kTmS + 16 * c, pk);
+                        tmem_st16(tm_lane + L::kTmDP + 16 * c, dk);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&bars->p_full);
+                    ++sc;
+                }
+                if (!ok) break;
+                // epilogue: accumulators -> bf16 rows of dQ, or of dK (scaled) and dV
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bars->acc_full, oc & 1, abort_flag, dev_status));
+                if (!ok) break;
+                ++oc;
+                tc_fence_after();
+                const int out_heads = KEYMAJOR ? Hkv : H;
+                const int out_head = KEYMAJOR ? it.head / G : it.head;
+                const int64_t base = (static_cast<int64_t>(slot) * out_heads + out_head) * HD;
+#pragma unroll 1
+                for (int a = 0; a < (KEYMAJOR ? 2 : 1); ++a) {
+                    // a = 0: the dS product (dQ or dK, times scale); a = 1: dV
+                    const uint32_t col0 = L::kTmAcc + (KEYMAJOR && a == 0 ? HD : 0);
+                    const float mul = a == 0 ? p.scale : 1.f;
+                    __nv_bfloat16* dst = (a == 0 ? out_a : out_b) + base;
+#pragma unroll 1
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(tm_lane + col0 + 32 * c, v);
+                        tmem_wait_ld();
+                        regs_after_wait(v);
+                        if (valid) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const uint4 w4 = make_uint4(
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * mul, __uint_as_float(v[8 * q4 + 1]) * mul),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * mul, __uint_as_float(v[8 * q4 + 3]) * mul),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * mul, __uint_as_float(v[8 * q4 + 5]) * mul),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * mul, __uint_as_float(v[8 * q4 + 7]) * mul));
+                                *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q4) = w4;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->acc_empty);
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, L::kTmemCols);
+}
+
+template <int HD, bool KEYMAJOR>
+cudaError_t launch_bwd_tc_one(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const CUtensorMap& tdo, const float* dsum,
+                              __nv_bfloat16* out_a, __nv_bfloat16* out_b, const int4* items,
+                              WorkspaceHeader* hdr, int sms, cudaStream_t stream) {
+    using L = BwdLayout<HD>;
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<HD, KEYMAJOR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attn_bwd_tc_kernel<HD, KEYMAJOR><<<sms, kBwdTcThreads, L::kSmemBytes, stream>>>(
+        tq, tk, tv, tdo, p, dsum, out_a, out_b, items, hdr);
+    return cudaGetLastError();
+}
+
+template <int HD>
+cudaError_t launch_bwd_tc_hd(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, const CUtensorMap& tdo, const float* dsum,
+                             void* dq, void* dk, void* dv, const int4* items, WorkspaceHeader* hdr,
+                             cudaStream_t stream) {
+    int dev = 0, sms = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    if ((e = launch_bwd_tc_one<HD, false>(p, tq, tk, tv, tdo, dsum, static_cast<__nv_bfloat16*>(dq),
+                                          nullptr, items, hdr, sms, stream)) != cudaSuccess)
+        return e;
+    return launch_bwd_tc_one<HD, true>(p, tq, tk, tv, tdo, dsum, static_cast<__nv_bfloat16*>(dk),
+                                       static_cast<__nv_bfloat16*>(dv), items, hdr, sms, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
+                               const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                               const CUtensorMap& tm_do, const float* dsum, void* dq, void* dk,
+                               void* dv, const int4* items, WorkspaceHeader* hdr,
+                               cudaStream_t stream) {
+    if (!band_applies(p)) return cudaErrorInvalidValue;
+    if (p.head_dim == 128)
+        return launch_bwd_tc_hd<128>(p, tm_q, tm_k, tm_v, tm_do, dsum, dq, dk, dv, items, hdr, stream);
+    if (p.head_dim == 64)
+        return launch_bwd_tc_hd<64>(p, tm_q, tm_k, tm_v, tm_do, dsum, dq, dk, dv, items, hdr, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pha

@@ -133,4 +133,56 @@ __device__ __forceinline__ uint64_t row_exp64(const uint32_t* v, int base, int c
     return sum2;
 }
 
+// Band work item (see kernels.cuh), decoded.
+struct BandItem {
+    int q0, n_qt, hp, head, doc_end;
+};
+
+__device__ __forceinline__ BandItem decode_band(int4 w) {
+    BandItem it;
+    it.q0 = w.x;
+    it.head = w.y >> 16;
+    it.hp = (w.y >> 15) & 1;
+    it.n_qt = w.y & 0x7FFF;
+    it.doc_end = w.z;
+    return it;
+}
+
+// Index of this CTA's k-th item: the longest-first list is dealt out in rows of gridDim.x items,
+// left to right on even rows and right to left on odd rows. -1 past the end of the list, -2 when
+// the last (partial) row has no item for this CTA.
+__device__ __forceinline__ int band_item_index(int k, int n_items) {
+    const int64_t base = static_cast<int64_t>(k) * gridDim.x;
+    if (base >= n_items) return -1;
+    const int64_t idx = base + ((k & 1) ? gridDim.x - 1 - blockIdx.x : blockIdx.x);
+    return idx < n_items ? static_cast<int>(idx) : -2;
+}
+
+// Walks this CTA's items in order, keeping the next one's descriptor in flight.
+struct ItemWalk {
+    const int4* items;
+    int n_items, k, idx, nidx;
+    int4 cur, nxt;
+    __device__ __forceinline__ void start(const int4* it, int n) {
+        items = it;
+        n_items = n;
+        k = 0;
+        idx = band_item_index(0, n);
+        cur = idx >= 0 ? __ldg(items + idx) : make_int4(0, 0, 0, 0);
+        prefetch();
+    }
+    __device__ __forceinline__ void prefetch() {
+        nidx = idx == -1 ? -1 : band_item_index(k + 1, n_items);
+        nxt = nidx >= 0 ? __ldg(items + nidx) : make_int4(0, 0, 0, 0);
+    }
+    __device__ __forceinline__ bool done() const { return idx == -1; }
+    __device__ __forceinline__ bool has() const { return idx >= 0; }
+    __device__ __forceinline__ void advance() {
+        idx = nidx;
+        cur = nxt;
+        ++k;
+        prefetch();
+    }
+};
+
 }  // namespace pha

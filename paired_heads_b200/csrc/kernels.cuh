@@ -72,10 +72,28 @@ cudaError_t launch_rope_bwd(void* dq, void* dk, const float* cos_tab, const floa
                             int n_heads, int n_kv_heads, int head_dim, int is_bf16, int paired,
                             int stagger_offset, cudaStream_t stream);
 
-// Backward of attention: dq, dk, dv (same layouts and dtype as q, k, v) for the upstream gradient
-// dout (layout of o); dsum is float[slots][heads] scratch (D_i). Needs p.lse.
-cudaError_t launch_attn_bwd(const AttnProblem& p, const void* dout, float* dsum, void* dq, void* dk,
-                            void* dv, int is_bf16, cudaStream_t stream);
+// Backward of attention, D_i = dO_i . O_i into dsum (float[slots][heads]), from the forward's
+// output o and the upstream gradient dout (both laid out like q).
+cudaError_t launch_attn_bwd_dsum(const AttnProblem& p, const void* o, const void* dout,
+                                 float* dsum, int is_bf16, cudaStream_t stream);
+
+// Backward of attention on CUDA cores (any shape): dq, dk, dv (same layouts and dtype as q, k, v)
+// for dout, from D in dsum. Needs p.lse. Rows outside every document get zeros.
+cudaError_t launch_attn_bwd(const AttnProblem& p, const void* dout, const float* dsum, void* dq,
+                            void* dk, void* dv, int is_bf16, cudaStream_t stream);
+
+// Zeros the rows of dq, dk, dv (bf16) outside every document.
+cudaError_t launch_attn_bwd_zero_outside(const AttnProblem& p, void* dq, void* dk, void* dv,
+                                         cudaStream_t stream);
+
+// Backward of the band attention on the tensor cores (bf16, band_applies, head_dim 64 / 128) over
+// a band work list: the dQ kernel, then the dK / dV kernel. tm_do is a map over dout like tm_q.
+// Writes the rows inside the documents only.
+cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
+                               const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                               const CUtensorMap& tm_do, const float* dsum, void* dq, void* dk,
+                               void* dv, const int4* items, WorkspaceHeader* hdr,
+                               cudaStream_t stream);
 
 // RoPE preceded by the QK RMS-norm of every head row (weights may be NULL = ones).
 cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,

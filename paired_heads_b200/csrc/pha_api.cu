@@ -159,22 +159,28 @@ pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* s
                : PHA_ERR_CUDA;
 }
 
-size_t pha_attn_bwd_workspace_bytes(int total_tokens, int n_heads) {
-    if (total_tokens < 0 || n_heads <= 0) return 0;
-    return (static_cast<size_t>(total_tokens) * n_heads * sizeof(float) + 255) & ~static_cast<size_t>(255);
+size_t pha_attn_bwd_workspace_bytes(int batch, int max_len, int total_tokens, int n_heads,
+                                    int head_dim, int paired) {
+    if (total_tokens < 0) return 0;
+    const size_t sched = pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired);
+    if (sched == 0) return 0;
+    return ((sched + 255) & ~static_cast<size_t>(255)) +
+           ((static_cast<size_t>(total_tokens) * n_heads * sizeof(float) + 255) &
+            ~static_cast<size_t>(255));
 }
 
-pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const float* lse,
-                        const void* dout, const int32_t* cu_seqlens, int batch, int max_len,
-                        int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, const int32_t* cu_seqlens, int batch,
+                        int max_len, int total_tokens, int n_heads, int n_kv_heads, int head_dim,
                         pha_dtype dtype, int causal, int window, int paired, float scale, void* dq,
                         void* dk, void* dv, void* workspace, size_t workspace_bytes,
                         pha_stream_t stream) {
     if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
     const bool have = total_tokens > 0;
-    if ((have && (!q || !k || !v || !lse || !dout || !dq || !dk || !dv || !aligned16(q) ||
-                  !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
-                  !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))) ||
+    if ((have && (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !aligned16(q) ||
+                  !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+                  !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+                  (reinterpret_cast<uintptr_t>(lse) & 3u))) ||
         !cu_seqlens || batch <= 0 || max_len < 0 || total_tokens < 0 ||
         total_tokens > (1 << 29) || n_heads <= 0 || n_kv_heads <= 0 || n_heads > 4096 ||
         n_heads % n_kv_heads != 0 || head_dim <= 0 || (causal != 0 && causal != 1) ||
@@ -183,10 +189,10 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const float
     if (paired && ((n_heads & 1) || (n_kv_heads & 1))) return PHA_ERR_INVALID;
     if (!causal && window > 0) return PHA_ERR_UNSUPPORTED;
     if (head_dim > 128) return PHA_ERR_UNSUPPORTED;
-    const size_t need = pha_attn_bwd_workspace_bytes(total_tokens, n_heads);
-    if (have && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) || workspace_bytes < need))
-        return PHA_ERR_WORKSPACE;
-    if (!have) return PHA_OK;
+    if (!have) return PHA_OK;  // nothing to do (no launch, the workspace is not touched)
+    const size_t need =
+        pha_attn_bwd_workspace_bytes(batch, max_len, total_tokens, n_heads, head_dim, paired);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PHA_ERR_WORKSPACE;
     AttnProblem p{};
     p.q = q;
     p.k = k;
@@ -203,10 +209,41 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const float
     p.window = window > 0 ? window : 0;
     p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
     p.lse = const_cast<float*>(lse);
-    return launch_attn_bwd(p, dout, static_cast<float*>(workspace), dq, dk, dv, dtype == PHA_BF16,
-                           stream) == cudaSuccess
-               ? PHA_OK
-               : PHA_ERR_CUDA;
+
+    // Workspace: the forward's scheduling area (header, document offsets, work items), then D.
+    const size_t sched = (pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired) + 255) &
+                         ~static_cast<size_t>(255);
+    auto* base = static_cast<uint8_t*>(workspace);
+    auto* hdr = reinterpret_cast<WorkspaceHeader*>(base);
+    auto* doc_blocks = reinterpret_cast<int*>(base + kWorkspaceHeaderBytes);
+    const size_t fixed = kWorkspaceHeaderBytes + workspace_doc_bytes(batch);
+    auto* items = reinterpret_cast<int4*>(base + fixed);
+    const int64_t cap64 = static_cast<int64_t>((sched - fixed) / sizeof(int4));
+    const int capacity = cap64 > 0x7FFFFFFF ? 0x7FFFFFFF : static_cast<int>(cap64);
+    float* dsum = reinterpret_cast<float*>(base + sched);
+
+    // Tensor cores for the band case (bf16, causal, 1 <= window <= 128, head_dim 64 / 128);
+    // CUDA cores otherwise. The scheduler also checks cu_seqlens (pha_attn_status).
+    const bool tc = dtype == PHA_BF16 && band_applies(p) && (head_dim == 64 || head_dim == 128);
+    if (launch_schedule(p, tc, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+        return PHA_ERR_CUDA;
+    if (launch_attn_bwd_dsum(p, o, dout, dsum, dtype == PHA_BF16, stream) != cudaSuccess)
+        return PHA_ERR_CUDA;
+    if (!tc)
+        return launch_attn_bwd(p, dout, dsum, dq, dk, dv, dtype == PHA_BF16, stream) == cudaSuccess
+                   ? PHA_OK
+                   : PHA_ERR_CUDA;
+    const uint64_t rows = static_cast<uint64_t>(total_tokens) * p.slot_mult;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_slot_map(&tq, q, static_cast<uint64_t>(p.heads) * head_dim, rows) ||
+        !encode_slot_map(&tk, k, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
+        !encode_slot_map(&tv, v, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
+        !encode_slot_map(&tdo, dout, static_cast<uint64_t>(p.heads) * head_dim, rows))
+        return PHA_ERR_CUDA;
+    if (launch_attn_bwd_zero_outside(p, dq, dk, dv, stream) != cudaSuccess ||
+        launch_attn_bwd_tc(p, tq, tk, tv, tdo, dsum, dq, dk, dv, items, hdr, stream) != cudaSuccess)
+        return PHA_ERR_CUDA;
+    return PHA_OK;
 }
 
 size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_dim, int paired) {

@@ -51,10 +51,10 @@ _lib.pha_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i
 _lib.pha_attn_fwd_aux_v.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                     ctypes.c_float, _p, _p, _p, _sz, _p]
 _lib.pha_rope_bwd.argtypes = [_p, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _i, _p]
-_lib.pha_attn_bwd_workspace_bytes.argtypes = [_i, _i]
+_lib.pha_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 _lib.pha_attn_bwd_workspace_bytes.restype = _sz
-_lib.pha_attn_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
-                              ctypes.c_float, _p, _p, _p, _p, _sz, _p]
+_lib.pha_attn_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                              _i, ctypes.c_float, _p, _p, _p, _p, _sz, _p]
 _lib.pha_qk_norm_rope.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _p, _i, _i, _p, _i, _i, _i,
                                   _i, _i, _i, _i, _p]
 for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status",
@@ -168,15 +168,18 @@ def pha_rope_bwd(dq, dk, cos_tab, sin_tab, positions, paired: bool = False, stag
                                              stagger_offset, _stream(stream, dq)))
 
 
-def pha_attn_bwd_workspace_bytes(total_tokens: int, n_heads: int) -> int:
-    return int(_lib.pha_attn_bwd_workspace_bytes(total_tokens, n_heads))
+def pha_attn_bwd_workspace_bytes(batch: int, max_len: int, total_tokens: int, n_heads: int,
+                                 head_dim: int, paired: bool) -> int:
+    return int(_lib.pha_attn_bwd_workspace_bytes(batch, max_len, total_tokens, n_heads, head_dim,
+                                                 int(paired)))
 
 
-def pha_attn_bwd(q, k, v, lse, dout, cu_seqlens, max_len: int, dq, dk, dv, workspace, *,
+def pha_attn_bwd(q, k, v, o, lse, dout, cu_seqlens, max_len: int, dq, dk, dv, workspace, *,
                  causal: bool = True, window: int = 0, paired: bool = False, scale: float = 0.0,
                  stream=None, batch=None, total_tokens=None, n_heads=None, n_kv_heads=None,
                  head_dim=None, dtype=None, workspace_bytes=None):
-    """Backward of pha_attn_fwd: writes dq, dk, dv for the upstream gradient dout."""
+    """Backward of pha_attn_fwd (o, lse: its outputs): writes dq, dk, dv for the upstream
+    gradient dout."""
     if total_tokens is None:
         total_tokens, n_heads, head_dim = q.shape
         n_kv_heads = k.shape[1]
@@ -185,10 +188,10 @@ def pha_attn_bwd(q, k, v, lse, dout, cu_seqlens, max_len: int, dq, dk, dv, works
     if workspace_bytes is None:
         workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("pha_attn_bwd",
-           _lib.pha_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(dout), _ptr(cu_seqlens),
-                             batch, max_len, total_tokens, n_heads, n_kv_heads, head_dim, dtype,
-                             int(causal), int(window), int(paired), float(scale), _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(workspace), workspace_bytes,
+           _lib.pha_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                             _ptr(cu_seqlens), batch, max_len, total_tokens, n_heads, n_kv_heads,
+                             head_dim, dtype, int(causal), int(window), int(paired), float(scale),
+                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace_bytes,
                              _stream(stream, q)))
 
 

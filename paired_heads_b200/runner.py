@@ -91,14 +91,16 @@ class AttentionStep:
                          stagger_offset=self.stagger_offset, stream=stream)
 
     def attn_bwd(self, q, k, v, dout, cu_seqlens, dq, dk, dv, stream=None):
-        """Backward of the last attention call's shape: dq, dk, dv for dout, using self.lse (the
-        forward must have run on the same q, k, v). Returns (dq, dk, dv)."""
+        """Backward of the last attention call (same q, k, v; its o and lse are used): dq, dk, dv
+        for dout. Returns (dq, dk, dv)."""
+        s = self.s
         if getattr(self, "bwd_workspace", None) is None:
-            nbytes = pha.pha_attn_bwd_workspace_bytes(self.s.total_tokens, self.s.n_heads)
+            nbytes = pha.pha_attn_bwd_workspace_bytes(s.batch, s.max_len, s.total_tokens,
+                                                      s.n_heads, s.head_dim, s.paired)
             self.bwd_workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
-        pha.pha_attn_bwd(q, k, v, self.lse, dout, cu_seqlens, self.s.max_len, dq, dk, dv,
-                         self.bwd_workspace, causal=self.s.causal, window=self.s.window,
-                         paired=self.s.paired, scale=self.s.scale, stream=stream)
+        pha.pha_attn_bwd(q, k, v, self.o, self.lse, dout, cu_seqlens, s.max_len, dq, dk, dv,
+                         self.bwd_workspace, causal=s.causal, window=s.window, paired=s.paired,
+                         scale=s.scale, stream=stream)
         return dq, dk, dv
 
     def __call__(self, q, k, v, cu_seqlens, positions, stream=None):

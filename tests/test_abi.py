@@ -202,12 +202,12 @@ def test_attn_aux_v_argument_errors(pha, kw, code):
 
 
 def _attn_bwd(pha, **kw):
-    args = dict(q=A, k=A, v=A, lse=A, g=A, cu=A, batch=1, max_len=128, total=128, H=4, Hkv=4,
+    args = dict(q=A, k=A, v=A, o=A, lse=A, g=A, cu=A, batch=1, max_len=128, total=128, H=4, Hkv=4,
                 hd=64, dtype=pha.PHA_BF16, causal=1, window=0, paired=0, scale=0.0, dq=A, dk=A,
                 dv=A, ws=A, ws_bytes=10)
     args.update(kw)
     return pha.library().pha_attn_bwd(
-        args["q"], args["k"], args["v"], args["lse"], args["g"], args["cu"], args["batch"],
+        args["q"], args["k"], args["v"], args["o"], args["lse"], args["g"], args["cu"], args["batch"],
         args["max_len"], args["total"], args["H"], args["Hkv"], args["hd"], args["dtype"],
         args["causal"], args["window"], args["paired"], ctypes.c_float(args["scale"]), args["dq"],
         args["dk"], args["dv"], args["ws"], args["ws_bytes"], None)
@@ -217,6 +217,8 @@ def _attn_bwd(pha, **kw):
     (dict(), -3),                              # valid: only the (too small) workspace stops it
     (dict(lse=None), -1),
     (dict(lse=A + 2), -1),
+    (dict(o=None), -1),
+    (dict(o=MIS), -1),
     (dict(g=None), -1),
     (dict(dk=MIS), -1),
     (dict(H=6, Hkv=4), -1),
@@ -231,9 +233,17 @@ def test_attn_bwd_argument_errors(pha, kw, code):
 
 
 def test_attn_bwd_workspace_bytes(pha):
-    assert pha.pha_attn_bwd_workspace_bytes(65536, 6) == 65536 * 6 * 4
-    assert pha.pha_attn_bwd_workspace_bytes(3, 1) == 256
-    assert pha.pha_attn_bwd_workspace_bytes(-1, 2) == 0
+    def up(n):
+        return (n + 255) // 256 * 256
+    for batch, max_len, total, H, hd, paired in [(113, 2048, 65536, 6, 128, True),
+                                                 (3, 700, 1000, 4, 64, False), (1, 0, 0, 2, 16, True)]:
+        fwd = pha.pha_attn_workspace_bytes(batch, max_len, H, hd, paired)
+        assert fwd > 0
+        assert pha.pha_attn_bwd_workspace_bytes(batch, max_len, total, H, hd, paired) == \
+            up(fwd) + up(total * H * 4)
+    assert pha.pha_attn_bwd_workspace_bytes(1, 16, -1, 2, 16, False) == 0
+    assert pha.pha_attn_bwd_workspace_bytes(0, 16, 16, 2, 16, False) == 0
+    assert pha.pha_attn_bwd_workspace_bytes(1, 16, 16, 3, 16, True) == 0
 
 
 def test_rope_bwd_argument_errors(pha):

@@ -1,11 +1,24 @@
 """Backward on the GPU (pha_rope_bwd, pha_attn_bwd) against the float64 oracle's gradients, which
 recompute the softmax from q and k. Needs a B200.
 
-Tolerances: the kernels compute in float32 from the bf16 (or f32) inputs and the forward's float32
-lse, and store in the input dtype. bf16 storage rounds each gradient to 8 significant bits
-(relative error <= 2^-9); the float32 sums add ~1e-6 of the largest terms. So bf16 gradients are
-compared with rtol 8e-3 plus an absolute 2e-3 of the tensor's largest value (sums that cancel),
-f32 gradients with rtol 1e-4 plus 1e-5 of the largest value."""
+Tolerances. Both backward paths take D_i = dO_i . O_i from the forward's stored O; the
+tensor-core path (bf16, causal, 1 <= window <= 128, head_dim 64 / 128) follows FlashAttention's
+backward arithmetic ("Training an LLM from scratch (part 2)", section "4. GQA & FlashAttention"):
+P and dS rounded to bf16 as MMA operands, float32 accumulation; the CUDA-core path (every other
+shape) keeps P and dS in float32. Near a document start a row sees few keys, P is large and dq is
+a difference of large terms, so a tolerance scaled by the tensor's maximum does not describe the
+error. bf16 gradients are therefore bounded per element, from the rounding steps of the
+tensor-core path (u = 2^-8, the unit roundoff of bf16's 8 significant bits); the CUDA-core path's
+rounding steps are a subset of these:
+  O (stored bf16, from bf16 P):  |dO_e| <= 2u sum_j P_ij |v_je|
+  so D = dO . O:                 |dD_i| <= 2u A_i,  A_i = sum_j P_ij (|dO_i| . |v_j|)
+  dS (bf16 of P (dP - D)):       |ddS_ij| <= u |dS_ij| + P_ij |dD_i|
+  dq = scale dS K, dk = scale dS^T Q:  scale sum |ddS| |k| (|q|), + u |result| (stored bf16)
+  dv = P^T dO with P in bf16:    u sum_i P_ij |dO_ie| + u |dv|
+each evaluated in float64 from the inputs and the exact P, dS, and allowed 1.25 times (the float32
+sums, the exponentials and the lse add relative errors near 1e-6 of the same terms). f32
+gradients (CUDA cores, float32 throughout) are compared with rtol 1e-4 plus 1e-5 of the tensor's
+largest value."""
 import numpy as np
 import pytest
 import torch
@@ -30,6 +43,50 @@ def _close(got, ref, dt, what):
     rtol, atol = (8e-3, 2e-3 * scale) if dt == "bf16" else (1e-4, 1e-5 * scale)
     err = np.abs(g - ref) - rtol * np.abs(ref)
     assert np.all(err <= atol), (what, float(np.abs(g - ref).max()), scale)
+    assert np.all(np.isfinite(g)), what
+
+
+def _bf16_bounds(Q, K, V, G, cu, causal, window, paired, scale, hd):
+    """Per-element error bounds of the bf16 backward (module docstring), token layout."""
+    u = 2.0 ** -8
+    T = Q.shape[0]
+    m = 2 if paired else 1
+    sv = lambda x: x.reshape(T * m, x.shape[1] // m, hd)
+    Qs, Ks, Vs, Gs = sv(Q), sv(K), sv(V), sv(G)
+    grp = Qs.shape[1] // Ks.shape[1]
+    bq, bk, bv = np.zeros_like(Qs), np.zeros_like(Ks), np.zeros_like(Vs)
+    cus = np.asarray(cu, dtype=np.int64) * m
+    for a, b in zip(cus[:-1], cus[1:]):
+        n = b - a
+        if n == 0:
+            continue
+        i, j = np.arange(n)[:, None], np.arange(n)[None, :]
+        vis = np.ones((n, n), dtype=bool)
+        if causal:
+            vis &= j <= i
+            if window > 0:
+                vis &= i - j < window
+        for h in range(Qs.shape[1]):
+            g = h // grp
+            q, k, v, go = Qs[a:b, h], Ks[a:b, g], Vs[a:b, g], Gs[a:b, h]
+            S = np.where(vis, q @ k.T * scale, -np.inf)
+            P = np.exp(S - S.max(1, keepdims=True))
+            P /= P.sum(1, keepdims=True)
+            dP = go @ v.T
+            dS = P * (dP - (P * dP).sum(1, keepdims=True))
+            dD = 2 * u * (P * (np.abs(go) @ np.abs(v).T)).sum(1)
+            bq[a:b, h] += scale * (u * np.abs(dS) @ np.abs(k) + dD[:, None] * (P @ np.abs(k)))
+            bk[a:b, g] += scale * (u * np.abs(dS).T @ np.abs(q) + (P * dD[:, None]).T @ np.abs(q))
+            bv[a:b, g] += u * P.T @ np.abs(go)
+    return (bq.reshape(Q.shape), bk.reshape(K.shape), bv.reshape(V.shape))
+
+
+def _close_bound(got, ref, bound, what):
+    g = got.to(torch.float64).cpu().numpy().reshape(ref.shape)
+    lim = 1.25 * (bound + 2.0 ** -8 * np.abs(ref)) + 1e-6 * float(np.abs(ref).max())
+    err = np.abs(g - ref)
+    worst = np.unravel_index(np.argmax(err / lim), err.shape)
+    assert np.all(err <= lim), (what, worst, float(err[worst]), float(lim[worst]))
     assert np.all(np.isfinite(g)), what
 
 
@@ -67,8 +124,13 @@ def test_rope_bwd_parity(paired, stagger, dt):
 
 CASES = [
     # doc lens, H, Hkv, hd, dtype, causal, window, paired
+    # tensor-core path (bf16, causal, window <= 128, hd 64 / 128)
     ((300, 5, 190), 6, 6, 128, "bf16", True, 128, True),
     ((257, 130), 4, 2, 64, "bf16", True, 37, False),
+    ((1100, 37, 600), 6, 6, 128, "bf16", True, 128, True),   # runs split into items (has-prev)
+    ((700, 129), 8, 2, 128, "bf16", True, 100, False),      # group of 4 query heads per kv head
+    ((64, 1, 130), 2, 2, 64, "bf16", True, 1, True),        # window 1, a one-token document
+    # CUDA-core path
     ((200, 64), 8, 2, 128, "bf16", True, 0, False),
     ((150, 90), 4, 4, 64, "bf16", False, 0, True),
     ((64,), 2, 2, 16, "f32", True, 0, True),
@@ -94,12 +156,20 @@ def test_attn_bwd_parity(case):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     step.attn_bwd(q, k, v, g_up.cuda(), cu, dq, dk, dv)
     torch.cuda.synchronize()
-    rq, rk, rv = oracle.attn_bwd(synth.to_f64(inp["q"]), synth.to_f64(inp["k"]),
-                                 synth.to_f64(inp["v"]), synth.to_f64(g_up),
-                                 inp["cu_seqlens"].numpy(), causal, window, paired, w.scale)
-    _close(dq, rq, dt, "dq")
-    _close(dk, rk, dt, "dk")
-    _close(dv, rv, dt, "dv")
+    args = (synth.to_f64(inp["q"]), synth.to_f64(inp["k"]), synth.to_f64(inp["v"]),
+            synth.to_f64(g_up))
+    rq, rk, rv = oracle.attn_bwd(*args, inp["cu_seqlens"].numpy(), causal, window, paired, w.scale)
+    if dt == "bf16":
+        scale = w.scale if w.scale > 0 else 1.0 / np.sqrt(hd)
+        bq, bk, bv = _bf16_bounds(*args, inp["cu_seqlens"].numpy(), causal, window, paired,
+                                  scale, hd)
+        _close_bound(dq, rq, bq, "dq")
+        _close_bound(dk, rk, bk, "dk")
+        _close_bound(dv, rv, bv, "dv")
+    else:
+        _close(dq, rq, dt, "dq")
+        _close(dk, rk, dt, "dk")
+        _close(dv, rv, dt, "dv")
 
 
 def test_backward_through_rope_and_attention():
@@ -122,10 +192,20 @@ def test_backward_through_rope_and_attention():
     pnp = inp["positions"].numpy()
     qr = oracle.rope_stored(synth.to_f64(inp["q"]), pnp, "bf16", True, True)
     kr = oracle.rope_stored(synth.to_f64(inp["k"]), pnp, "bf16", True, True)
-    rq, rk, rv = oracle.attn_bwd(qr, kr, synth.to_f64(inp["v"]), synth.to_f64(g_up),
-                                 inp["cu_seqlens"].numpy(), True, w.window, True, w.scale)
-    rq = oracle.rope_bwd(rq, pnp, True, True, table_f32=True)
-    rk = oracle.rope_bwd(rk, pnp, True, True, table_f32=True)
-    _close(dq, rq, "bf16", "dq")
-    _close(dk, rk, "bf16", "dk")
-    _close(dv, rv, "bf16", "dv")
+    args = (qr, kr, synth.to_f64(inp["v"]), synth.to_f64(g_up))
+    rq0, rk0, rv = oracle.attn_bwd(*args, inp["cu_seqlens"].numpy(), True, w.window, True, w.scale)
+    rq = oracle.rope_bwd(rq0, pnp, True, True, table_f32=True)
+    rk = oracle.rope_bwd(rk0, pnp, True, True, table_f32=True)
+    # bounds of the tensor-core backward, plus the bf16 rounding of its stored dq, dk, carried
+    # through the rotation of each adjacent pair (|cos|, |sin| <= 1: element e of the output
+    # mixes elements e and e ^ 1 of its input)
+    scale = w.scale if w.scale > 0 else 1.0 / np.sqrt(w.head_dim)
+    bq, bk, bv = _bf16_bounds(*args, inp["cu_seqlens"].numpy(), True, w.window, True, scale,
+                              w.head_dim)
+    swap = np.arange(w.head_dim) ^ 1
+    for b, r0 in ((bq, rq0), (bk, rk0)):
+        b += 2.0 ** -8 * np.abs(r0)
+        b += b[..., swap].copy()
+    _close_bound(dq, rq, bq, "dq")
+    _close_bound(dk, rk, bk, "dk")
+    _close_bound(dv, rv, bv, "dv")
