@@ -290,20 +290,29 @@ def main():
             step.rope_bwd(dq, dk, pos)
         torch.cuda.synchronize(dev)
         nb = max(3, min(args.steps, 20))
-        ba, bm, bb = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        att = 0.0
+        bev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(nb)]
         pdist.barrier(dist)
-        ba.record(stream)
-        for _ in range(nb):
+        for e in bev:
+            e[0].record(stream)
             step.attn_bwd(q, k, v, g_up, cu, dq, dk, dv)
+            e[1].record(stream)
             step.rope_bwd(dq, dk, pos)
-        bb.record(stream)
+            e[2].record(stream)
         torch.cuda.synchronize(dev)
-        b_ms = pdist.max_over_ranks(dist, ba.elapsed_time(bb) / nb, dev)
+        b_ms = pdist.max_over_ranks(dist, bev[0][0].elapsed_time(bev[-1][2]) / nb, dev)
+        ab_ms = sum(e[0].elapsed_time(e[1]) for e in bev) / nb
+        rb_ms = sum(e[1].elapsed_time(e[2]) for e in bev) / nb
         bwd_flops = 2.5 * attn_flops(w)
+        tc_bwd = w.dtype == "bf16" and w.causal and 1 <= w.window <= 128 and w.head_dim in (64, 128)
         bwd = {"ms": b_ms, "steps": nb, "flops": bwd_flops,
                "tflops": bwd_flops * world / (b_ms * 1e-3) / 1e12,
-               "kernels": "dq (query-major) + dk/dv (key-major) on CUDA cores, then pha_rope_bwd",
+               "attn_bwd_ms": ab_ms, "rope_bwd_ms": rb_ms,
+               "attn_bwd_tflops": bwd_flops / (ab_ms * 1e-3) / 1e12,
+               "attn_bwd_frac_of_bf16_peak": bwd_flops / (ab_ms * 1e-3) / 1e12 / load_peaks()[0]["bf16_tflops"],
+               "kernels": ("pha_attn_bwd: D = dO.O, then the dQ and dK/dV kernels on the tensor cores "
+                           "(tcgen05)" if tc_bwd else
+                           "pha_attn_bwd: D = dO.O, then dq and dk/dv on CUDA cores") +
+                          "; then pha_rope_bwd",
                "flop_count": "2.5 x the forward's causal-counted FLOPs (S, dP, dV, dK, dQ)"}
 
     # ---- end to end through the public API with host buffers. Documents are independent, so the

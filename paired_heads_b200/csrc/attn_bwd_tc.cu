@@ -14,17 +14,22 @@
 //     dV += P^T dO and dK += dS^T Q with P^T, dS^T in TMEM as the A operand.
 //   query-major (dQ): outer tile = query tile (X = Q, dO), inner steps = the key tiles it sees
 //     (Y = K, V): S = Q K^T, dP = dO V^T, then dQ += dS K.
-// In both, the 128 x 128 scores go to TMEM columns [0, 128), dP to [128, 256); the bf16 P and dS
-// overwrite the first half of each; the accumulators sit at 256 (dV or dQ) and 256 + hd (dK).
+// In both, the 128 x 128 scores go to TMEM columns [0, 128), dP to [128, 256). An inner step's
+// columns are split in two halves of 64 (Y rows 64 h .. 64 h + 63), one per elementwise
+// warpgroup: the bf16 P and dS of half h overwrite the first 32 of the half's own columns
+// (64 h + [0, 32) and 128 + 64 h + [0, 32)), and are the A operand of the half's second products
+// (K = 64), issued as soon as that warpgroup is done. The accumulators sit at 256 (dV or dQ) and
+// 256 + hd (dK).
 // A tile loaded for the K-major S / dP product (rows = slots, [64-column chunks] 128-byte
 // swizzled) is the MN-major B operand of the second product as it stands.
 //
-// CTA = 6 warps, persistent, one per SM, band items in snake order:
-//   warps 0-3  elementwise: row = TMEM lane; P, dS from S, dP; the epilogue (accumulators ->
-//              bf16 -> global)
-//   warp 4     producer: X tiles (one buffer), Y tiles (two stages) by TMA; in the key-major
-//              instance also lse * log2(e) and D of the step's 128 queries into shared memory
-//   warp 5     MMA issuer, owner of the 512 TMEM columns
+// CTA = 10 warps, persistent, one per SM, band items in snake order:
+//   warps 0-7  elementwise, two warpgroups: warpgroup h takes half h of every inner step (row =
+//              TMEM lane; P, dS from S, dP) and half h of the accumulator columns in the epilogue
+//              (accumulators -> bf16 -> global); two warps per scheduler hide each other's latency
+//   warp 8     producer: X tiles (one buffer), Y tiles (two-slot ring) by TMA; in the key-major
+//              instance also lse * log2(e) and D of the fill's 128 queries into shared memory
+//   warp 9     MMA issuer, owner of the 512 TMEM columns
 // Every wait is bounded (1 s); on expiry the CTA records a status, drains its own copies and
 // MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -40,7 +45,7 @@ namespace pha {
 
 namespace {
 
-constexpr int kBwdTcThreads = 192;
+constexpr int kBwdTcThreads = 320;
 
 template <int HD>
 struct BwdLayout {
@@ -61,7 +66,8 @@ struct BwdLayout {
 struct BwdBars {
     uint64_t x_full, x_empty;
     uint64_t y_full[2], y_empty[2];
-    uint64_t s_full, p_full, m2_done, acc_full, acc_empty, drain;
+    uint64_t s_full[2], p_full[2], m2_done[2];  // per half
+    uint64_t acc_full, acc_empty, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -107,6 +113,45 @@ __device__ __forceinline__ bool item_used(const BandItem& it, int G) {
     return !KEYMAJOR || it.head % G == 0;
 }
 
+// Y fills (two-slot ring) and the inner steps that read them. With reuse, a Y tile shared by
+// consecutive outer tiles of a run is filled once: query-major, the key tile of q-tile u's
+// diagonal step is the previous-tile step of q-tile u + 1; key-major with one query head per kv
+// head, the query tile of key tile u's next-tile step is the diagonal step of key tile u + 1.
+// Without reuse (key-major, several query heads per kv head) every step has its own fill.
+struct StepFill {
+    uint32_t idx;  // position in this CTA's fill sequence: slot idx & 1, lap idx >> 1
+    bool first;    // the step is the fill's first reader (the producer loads it for this step)
+    bool last;     // ... and its last reader (the slot is released after the step)
+};
+
+template <bool KEYMAJOR>
+struct FillTrack {
+    uint32_t n = 0;      // fills so far
+    uint32_t carry = 0;  // the fill the next outer tile's shared step reads
+    __device__ __forceinline__ StepFill step(bool reuse, int u, int n_tiles, int s, int n_sub) {
+        StepFill f;
+        if (!reuse) {
+            f.idx = n++;
+            f.first = f.last = true;
+            return f;
+        }
+        // the step shared with the previous outer tile: query-major the previous key tile (the
+        // first of two steps), key-major the diagonal query tile (step 0)
+        const bool shared = KEYMAJOR ? s == 0 : s + 1 < n_sub;
+        if (shared) {
+            f.first = u == 0;  // a run's first tile has no predecessor that filled it
+            f.idx = f.first ? n++ : carry;
+            f.last = true;
+        } else {
+            f.idx = n++;
+            f.first = true;
+            f.last = u + 1 == n_tiles;  // else carried to the next outer tile
+            carry = f.idx;
+        }
+        return f;
+    }
+};
+
 template <int HD, bool KEYMAJOR>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -131,7 +176,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         mbar_init(&bars->x_full, 1);
         mbar_init(&bars->x_empty, 1);
         for (int s = 0; s < 2; ++s) {
@@ -139,11 +184,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             mbar_init(&bars->y_full[s], KEYMAJOR ? 33 : 1);
             mbar_init(&bars->y_empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->m2_done, 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&bars->s_full[h], 1);
+            mbar_init(&bars->p_full[h], 128);
+            mbar_init(&bars->m2_done[h], 1);
+        }
         mbar_init(&bars->acc_full, 1);
-        mbar_init(&bars->acc_empty, 128);
+        mbar_init(&bars->acc_empty, 256);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_mbar_init();
@@ -152,7 +199,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_do);
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&bars->tmem_base, L::kTmemCols);
         tmem_relinquish();
     }
@@ -163,16 +210,51 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads, Hkv = p.kv_heads, G = H / Hkv;
+    const bool reuse = !KEYMAJOR || G == 1;
     // X = (K, V) and Y = (Q, dO) (key-major), or the other way round
     const CUtensorMap* mx0 = KEYMAJOR ? &tm_k : &tm_q;
     const CUtensorMap* mx1 = KEYMAJOR ? &tm_v : &tm_do;
     const CUtensorMap* my0 = KEYMAJOR ? &tm_q : &tm_k;
     const CUtensorMap* my1 = KEYMAJOR ? &tm_do : &tm_v;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------ producer
-        uint32_t oc = 0, sc = 0;  // outer tiles / inner steps issued so far
+        // Per outer tile: with reuse its new Y fills, then X (the order in which their slots are
+        // released); without, X and then one fill per step.
+        uint32_t oc = 0;  // outer tiles issued so far
+        FillTrack<KEYMAJOR> ft;
         bool ok = true;
+        auto load_y = [&](const BandItem& it, const OuterTile& o, int s, uint32_t idx) -> bool {
+            const uint32_t st = idx & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->y_empty[st], ((idx >> 1) & 1) ^ 1,
+                                                   abort_flag, dev_status)))
+                return false;
+            int y_head, y_row;
+            inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars->y_full[st], 2 * L::kTile);
+                uint8_t* y = smem + L::kOffY + st * 2 * L::kTile;
+                for (int c = 0; c < HD / 64; ++c) {
+                    tma_load_2d(y + c * L::kChunk, my0, y_head * HD + 64 * c, y_row, &bars->y_full[st]);
+                    tma_load_2d(y + L::kTile + c * L::kChunk, my1, y_head * HD + 64 * c, y_row,
+                                &bars->y_full[st]);
+                }
+            }
+            if (KEYMAJOR) {
+                // lse * log2(e) and D of the fill's queries (0 past the document end)
+                float* l2 = vec + st * 256;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 4 * lane + e, qs = y_row + c;
+                    const bool in = qs < it.doc_end;
+                    const int64_t r = static_cast<int64_t>(qs) * H + y_head;
+                    l2[c] = in ? p.lse[r] * kLog2e : 0.f;
+                    l2[128 + c] = in ? dsum[r] : 0.f;
+                }
+                mbar_arrive(&bars->y_full[st]);
+            }
+            return true;
+        };
         ItemWalk wk;
         for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
             if (!wk.has()) continue;
@@ -181,6 +263,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             const int x_head = KEYMAJOR ? it.head / G : it.head;
             for (int u = 0; ok && u < it.n_qt; ++u) {
                 const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                for (int s = 0; ok && reuse && s < o.n_sub; ++s) {
+                    const StepFill f = ft.step(true, u, it.n_qt, s, o.n_sub);
+                    if (f.first) ok = load_y(it, o, s, f.idx);
+                }
+                if (!ok) break;
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_empty, (oc & 1) ^ 1, abort_flag,
                                                        dev_status));
                 if (!ok) break;
@@ -194,48 +281,18 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     }
                 }
                 ++oc;
-                for (int s = 0; s < o.n_sub; ++s) {
-                    const uint32_t st = sc & 1;
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_empty[st], ((sc >> 1) & 1) ^ 1,
-                                                           abort_flag, dev_status));
-                    if (!ok) break;
-                    int y_head, y_row;
-                    inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&bars->y_full[st], 2 * L::kTile);
-                        uint8_t* y = smem + L::kOffY + st * 2 * L::kTile;
-                        for (int c = 0; c < HD / 64; ++c) {
-                            tma_load_2d(y + c * L::kChunk, my0, y_head * HD + 64 * c, y_row,
-                                        &bars->y_full[st]);
-                            tma_load_2d(y + L::kTile + c * L::kChunk, my1, y_head * HD + 64 * c,
-                                        y_row, &bars->y_full[st]);
-                        }
-                    }
-                    if (KEYMAJOR) {
-                        // lse * log2(e) and D of the step's queries (0 past the document end)
-                        float* l2 = vec + st * 256;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = 4 * lane + e, qs = y_row + c;
-                            const bool in = qs < it.doc_end;
-                            const int64_t r = static_cast<int64_t>(qs) * H + y_head;
-                            l2[c] = in ? p.lse[r] * kLog2e : 0.f;
-                            l2[128 + c] = in ? dsum[r] : 0.f;
-                        }
-                        mbar_arrive(&bars->y_full[st]);
-                    }
-                    ++sc;
-                }
+                for (int s = 0; ok && !reuse && s < o.n_sub; ++s)
+                    ok = load_y(it, o, s, ft.step(false, u, it.n_qt, s, o.n_sub).idx);
             }
         }
         if (!ok && lane == 0) {
             // Wait (bounded) for the copies this warp issued last into every buffer.
             if (oc > 0) drain_wait(&bars->x_full, (oc - 1) & 1);
-            for (uint32_t n = sc > 2 ? sc - 2 : 0; n < sc; ++n)
+            for (uint32_t n = ft.n > 2 ? ft.n - 2 : 0; n < ft.n; ++n)
                 drain_wait(&bars->y_full[n & 1], (n >> 1) & 1);
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc1 = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
@@ -245,6 +302,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             const uint32_t tm_acc_ds = tmem + L::kTmAcc + (KEYMAJOR ? HD : 0);  // dK or dQ
             const uint32_t x0 = sbase + L::kOffX, x1 = x0 + L::kTile;
             uint32_t oc = 0, sc = 0;
+            FillTrack<KEYMAJOR> ft;
             bool ok = true;
             ItemWalk wk;
             for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
@@ -258,14 +316,22 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                         break;
                     }
                     for (int s = 0; s < o.n_sub; ++s) {
-                        const uint32_t st = sc & 1;
+                        const StepFill f = ft.step(reuse, u, it.n_qt, s, o.n_sub);
+                        const uint32_t st = f.idx & 1;
                         const uint32_t y0 = sbase + L::kOffY + st * 2 * L::kTile, y1 = y0 + L::kTile;
-                        if (!mbar_wait(&bars->y_full[st], (sc >> 1) & 1, abort_flag, dev_status) ||
-                            (sc > 0 && !mbar_wait(&bars->m2_done, (sc - 1) & 1, abort_flag,
-                                                  dev_status))) {
+                        // each fill is waited for once, by its first reader, in fill order
+                        if (f.first &&
+                            !mbar_wait(&bars->y_full[st], (f.idx >> 1) & 1, abort_flag, dev_status)) {
                             ok = false;
                             break;
                         }
+                        // S = X0 Y0^T and dP = X1 Y1^T at full width (N = 128); their columns are free
+                        // once the previous step's second products of both halves are done
+                        for (int h = 0; ok && h < 2; ++h)
+                            if (sc > 0 && !mbar_wait(&bars->m2_done[h], (sc - 1) & 1, abort_flag,
+                                                     dev_status))
+                                ok = false;
+                        if (!ok) break;
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -274,24 +340,32 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                             umma_f16_ss(tm_dp, desc_kmajor(x1, kk), desc_kmajor(y1, kk), idesc1,
                                         kk == 0 ? 0u : 1u);
                         }
-                        umma_commit(&bars->s_full);
+                        umma_commit(&bars->s_full[0]);  // one per elementwise warpgroup
+                        umma_commit(&bars->s_full[1]);
+                        if (!ok) break;
                         if (s + 1 == o.n_sub) umma_commit(&bars->x_empty);
-                        if (!mbar_wait(&bars->p_full, sc & 1, abort_flag, dev_status) ||
-                            (s == 0 && oc > 0 &&
-                             !mbar_wait(&bars->acc_empty, (oc - 1) & 1, abort_flag, dev_status))) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
+                        // second products of half h: K = the half's 64 Y rows
+                        for (int h = 0; ok && h < 2; ++h) {
+                            if (!mbar_wait(&bars->p_full[h], sc & 1, abort_flag, dev_status) ||
+                                (s == 0 && h == 0 && oc > 0 &&
+                                 !mbar_wait(&bars->acc_empty, (oc - 1) & 1, abort_flag, dev_status))) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                            umma_f16_ts(tm_acc_ds, tm_dp + 8 * kk, desc_v(y0, kk), idesc2, acc);
-                            if (KEYMAJOR)
-                                umma_f16_ts(tm_acc_p, tm_s + 8 * kk, desc_v(y1, kk), idesc2, acc);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t acc = (s > 0 || h > 0 || kk > 0) ? 1u : 0u;
+                                umma_f16_ts(tm_acc_ds, tm_dp + 64 * h + 8 * kk, desc_v(y0, 4 * h + kk),
+                                            idesc2, acc);
+                                if (KEYMAJOR)
+                                    umma_f16_ts(tm_acc_p, tm_s + 64 * h + 8 * kk, desc_v(y1, 4 * h + kk),
+                                                idesc2, acc);
+                            }
+                            umma_commit(&bars->m2_done[h]);
                         }
-                        umma_commit(&bars->m2_done);
-                        umma_commit(&bars->y_empty[st]);
+                        if (!ok) break;
+                        if (f.last) umma_commit(&bars->y_empty[st]);
                         if (s + 1 == o.n_sub) umma_commit(&bars->acc_full);
                         ++sc;
                     }
@@ -304,13 +378,15 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ elementwise warpgroup
-        const int row = threadIdx.x;         // TMEM lane == row of the outer tile
-        const int r0 = warp * 32;            // first row of this warp
+        // ------------------------------------------------------------ elementwise warpgroups
+        const int h = warp >> 2;              // the half of every step this warpgroup takes
+        const int row = threadIdx.x & 127;    // TMEM lane == row of the outer tile
+        const int r0 = (warp & 3) * 32;       // first row of this warp
         const uint32_t tm_lane = tmem + (static_cast<uint32_t>(r0) << 16);
         const float scale_log2 = p.scale * kLog2e;
         const int window = p.window;
         uint32_t oc = 0, sc = 0;
+        FillTrack<KEYMAJOR> ft;
         bool ok = true;
         ItemWalk wk;
         for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
@@ -328,7 +404,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     dd = dsum[r];
                 }
                 for (int s = 0; s < o.n_sub; ++s) {
-                    const uint32_t st = sc & 1;
+                    const StepFill f = ft.step(reuse, u, it.n_qt, s, o.n_sub);
+                    const uint32_t st = f.idx & 1;
                     int y_head, y_row;
                     inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
                     // visible columns [c_lo, c_hi] of this row
@@ -340,56 +417,63 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                         c_lo = slot - window + 1 - y_row;
                         c_hi = valid ? slot - y_row : c_lo - 1;
                     }
+                    // key-major: the fill's lse2 / D (every reader waits; a fill's slot is not
+                    // refilled before its last reader has finished, so no wait can see a later lap)
                     if (KEYMAJOR)
-                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full[st], (sc >> 1) & 1,
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full[st], (f.idx >> 1) & 1,
                                                                abort_flag, dev_status));
-                    if (ok)
-                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, sc & 1, abort_flag,
-                                                               dev_status));
                     if (!ok) break;
-                    tc_fence_after();
                     const int w_lo = __reduce_min_sync(0xffffffffu, c_lo);
                     const int w_hi = __reduce_max_sync(0xffffffffu, c_hi);
                     const float* l2v = vec + st * 256;
+                    {
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], sc & 1, abort_flag,
+                                                               dev_status));
+                        if (!ok) break;
+                        tc_fence_after();
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t pk[16], dk[16];
-                        if (32 * c > w_hi || 32 * c + 31 < w_lo) {  // no row of the warp sees it
+                        for (int c = 2 * h; c < 2 * h + 2; ++c) {
+                            uint32_t pk[16], dk[16];
+                            if (32 * c > w_hi || 32 * c + 31 < w_lo) {  // no row of the warp sees it
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = dk[e] = 0u;
-                        } else {
-                            uint32_t sv[32], dv[32];
-                            tmem_ld32(tm_lane + L::kTmS + 32 * c, sv);
-                            tmem_ld32(tm_lane + L::kTmDP + 32 * c, dv);
-                            tmem_wait_ld();
-                            regs_after_wait(sv);
-                            regs_after_wait(dv);
+                                for (int e = 0; e < 16; ++e) pk[e] = dk[e] = 0u;
+                            } else {
+                                uint32_t sv[32], dv[32];
+                                tmem_ld32(tm_lane + L::kTmS + 32 * c, sv);
+                                tmem_ld32(tm_lane + L::kTmDP + 32 * c, dv);
+                                tmem_wait_ld();
+                                regs_after_wait(sv);
+                                regs_after_wait(dv);
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
-                                float pr[2], dr[2];
+                                for (int e = 0; e < 32; e += 2) {
+                                    float pr[2], dr[2];
 #pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    const int col = 32 * c + e + h;
-                                    float l2 = lse2, d = dd;
-                                    if (KEYMAJOR) {
-                                        l2 = l2v[col];
-                                        d = l2v[128 + col];
+                                    for (int x = 0; x < 2; ++x) {
+                                        const int col = 32 * c + e + x;
+                                        float l2 = lse2, d = dd;
+                                        if (KEYMAJOR) {
+                                            l2 = l2v[col];
+                                            d = l2v[128 + col];
+                                        }
+                                        const bool vis = col >= c_lo && col <= c_hi;
+                                        const float pe = ex2(fmaf(__uint_as_float(sv[e + x]), scale_log2, -l2));
+                                        pr[x] = vis ? pe : 0.f;
+                                        dr[x] = pr[x] * (__uint_as_float(dv[e + x]) - d);
                                     }
-                                    const bool vis = col >= c_lo && col <= c_hi;
-                                    const float pe = ex2(fmaf(__uint_as_float(sv[e + h]), scale_log2, -l2));
-                                    pr[h] = vis ? pe : 0.f;
-                                    dr[h] = pr[h] * (__uint_as_float(dv[e + h]) - d);
+                                    pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+                                    dk[e >> 1] = pack_bf16x2(dr[0], dr[1]);
                                 }
-                                pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
-                                dk[e >> 1] = pack_bf16x2(dr[0], dr[1]);
                             }
+                            // packed pairs of the half's 64 columns: 32 TMEM columns from 64 h, over
+                            // columns of this half that this thread has already read
+                            if (KEYMAJOR) tmem_st16(tm_lane + L::kTmS + 16 * c + 32 * h, pk);
+                            tmem_st16(tm_lane + L::kTmDP + 16 * c + 32 * h, dk);
                         }
-                        if (KEYMAJOR) tmem_st16(tm_lane + L::kTmS + 16 * c, pk);
-                        tmem_st16(tm_lane + L::kTmDP + 16 * c, dk);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&bars->p_full[h]);
                     }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&bars->p_full);
+                    if (!ok) break;
                     ++sc;
                 }
                 if (!ok) break;
@@ -409,7 +493,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     const float mul = a == 0 ? p.scale : 1.f;
                     __nv_bfloat16* dst = (a == 0 ? out_a : out_b) + base;
 #pragma unroll 1
-                    for (int c = 0; c < HD / 32; ++c) {
+                    for (int c = h * (HD / 64); c < (h + 1) * (HD / 64); ++c) {  // this half's columns
                         uint32_t v[32];
                         tmem_ld32(tm_lane + col0 + 32 * c, v);
                         tmem_wait_ld();
@@ -437,7 +521,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, L::kTmemCols);
+    if (warp == 9) tmem_dealloc(tmem, L::kTmemCols);
 }
 
 template <int HD, bool KEYMAJOR>
