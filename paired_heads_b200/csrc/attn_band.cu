@@ -89,7 +89,8 @@ template <int HD, bool AUXV>
 __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
     attn_band_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const AttnProblem p,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_out, const AttnProblem p,
                      const int4* __restrict__ items, WorkspaceHeader* hdr) {
     using L = TcLayout<HD>;
     constexpr int S = L::kKStages;
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_out);
     }
     if (warp == 9) {
         tmem_alloc(&bars->tmem_base, L::kTmemCols);
@@ -453,13 +455,16 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                 ++o_cnt;
                 tc_fence_after();
                 const float inv_l = l > 0.f ? 1.f / l : 0.f;
-                // O / l -> bf16, staged through this tile's Q slot (its last S has completed):
-                // each warp writes its 32 rows with an XOR swizzle of the 16-byte chunks, then
-                // copies them out two rows per instruction (hd 128), so every global store of
-                // the warp covers 512 contiguous bytes. Rows past the document end are skipped.
-                constexpr int kChunks = HD / 8;  // 16-byte chunks per row
-                uint8_t* stage = smem + L::kOffQ + (n % L::kQSlots) * L::kQSub + r0 * (HD * 2);
-                const int wrow = row & 31;
+                // O / l -> bf16, staged through this tile's Q slot (its last S has completed) in
+                // the slot's own layout (the TMA box layout: [hd / 64][128 rows][128 B], 16-byte
+                // units XOR-swizzled by row % 8). A warp whose 32 rows all lie inside the document
+                // stores them with TMA stores (one 64 x 32 box per 64 columns), asynchronously;
+                // otherwise it copies its valid rows out with plain stores, two rows per
+                // instruction (hd 128), so each warp store covers 512 contiguous bytes.
+                uint8_t* slot_base = smem + L::kOffQ + (n % L::kQSlots) * L::kQSub;
+                auto unit_addr = [&](int r, int u) -> uint8_t* {
+                    return slot_base + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+                };
 #pragma unroll 1
                 for (int c = 0; c < HD / 32; ++c) {
                     uint32_t v[32];
@@ -473,30 +478,39 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                             pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv_l, __uint_as_float(v[8 * q4 + 3]) * inv_l),
                             pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv_l, __uint_as_float(v[8 * q4 + 5]) * inv_l),
                             pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv_l, __uint_as_float(v[8 * q4 + 7]) * inv_l));
-                        const int chunk = 4 * c + q4;
-                        *reinterpret_cast<uint4*>(stage + wrow * (HD * 2) +
-                                                  ((chunk ^ (wrow & (kChunks - 1))) << 4)) = w4;
+                        *reinterpret_cast<uint4*>(unit_addr(row, 4 * c + q4)) = w4;
                     }
                 }
-                __syncwarp();
-                {
+                if (r0 + 31 < nr) {
+                    fence_proxy_async_smem();  // the rows are read by the async proxy (TMA)
+                    __syncwarp();
+                    if (lane == 0) {
+                        for (int c = 0; c < HD / 64; ++c)
+                            tma_store_2d(&tm_out, it.head * HD + 64 * c, q_start + r0,
+                                         slot_base + c * L::kChunk + r0 * 128);
+                        tma_store_commit();
+                        tma_store_wait_read();  // the slot may be refilled once the rows are read
+                    }
+                    __syncwarp();
+                } else {
+                    __syncwarp();
+                    constexpr int kChunks = HD / 8;  // 16-byte units per row
                     constexpr int kRowsPerIter = 32 / kChunks;
 #pragma unroll 4
                     for (int j = 0; j < 32 / kRowsPerIter; ++j) {
                         const int rl = j * kRowsPerIter + lane / kChunks;
-                        const int chunk = lane % kChunks;
+                        const int unit = lane % kChunks;
                         if (r0 + rl < nr) {
-                            const uint4 w4 = *reinterpret_cast<const uint4*>(
-                                stage + rl * (HD * 2) + ((chunk ^ (rl & (kChunks - 1))) << 4));
+                            const uint4 w4 = *reinterpret_cast<const uint4*>(unit_addr(r0 + rl, unit));
                             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) +
                                                  (static_cast<int64_t>(q_start + r0 + rl) * H + it.head) * HD +
-                                                 chunk * 8;
+                                                 unit * 8;
                             *reinterpret_cast<uint4*>(dst) = w4;
                         }
                     }
+                    __syncwarp();
+                    fence_proxy_async_smem();  // the slot's next fill is written by the async proxy
                 }
-                __syncwarp();
-                fence_proxy_async_smem();  // the slot's next fill is written by the async proxy (TMA)
                 if (lane == 0) mbar_arrive(&bars->q_empty[n % L::kQSlots]);
                 tc_fence_before();
                 if (row < nr && p.lse)
@@ -506,6 +520,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
     }
 
     // ---------------------------------------------------------------- teardown
+    if (warp < 8 && lane == 0) tma_store_wait_all();  // the epilogue's O stores have completed
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -514,8 +529,9 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
 
 template <int HD, bool AUXV>
 static cudaError_t launch_band_hd(const AttnProblem& p, const CUtensorMap& tq,
-                                  const CUtensorMap& tk, const CUtensorMap& tv, const int4* items,
-                                  WorkspaceHeader* hdr, cudaStream_t stream) {
+                                  const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const CUtensorMap& to, const int4* items, WorkspaceHeader* hdr,
+                                  cudaStream_t stream) {
     using L = TcLayout<HD>;
     cudaError_t e = cudaFuncSetAttribute(attn_band_kernel<HD, AUXV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
@@ -525,21 +541,22 @@ static cudaError_t launch_band_hd(const AttnProblem& p, const CUtensorMap& tq,
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
     attn_band_kernel<HD, AUXV><<<sms, AUXV ? kBandAuxThreads : kBandThreads, L::kSmemBytes, stream>>>(
-        tq, tk, tv, p, items, hdr);
+        tq, tk, tv, to, p, items, hdr);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_band(const AttnProblem& p, const CUtensorMap& tm_q,
-                             const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int4* items,
-                             WorkspaceHeader* hdr, cudaStream_t stream) {
+                             const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const CUtensorMap& tm_o, const int4* items, WorkspaceHeader* hdr,
+                             cudaStream_t stream) {
     if (!band_applies(p)) return cudaErrorInvalidValue;
     const bool aux = p.v_aux != nullptr;
     if (p.head_dim == 128)
-        return aux ? launch_band_hd<128, true>(p, tm_q, tm_k, tm_v, items, hdr, stream)
-                   : launch_band_hd<128, false>(p, tm_q, tm_k, tm_v, items, hdr, stream);
+        return aux ? launch_band_hd<128, true>(p, tm_q, tm_k, tm_v, tm_o, items, hdr, stream)
+                   : launch_band_hd<128, false>(p, tm_q, tm_k, tm_v, tm_o, items, hdr, stream);
     if (p.head_dim == 64)
-        return aux ? launch_band_hd<64, true>(p, tm_q, tm_k, tm_v, items, hdr, stream)
-                   : launch_band_hd<64, false>(p, tm_q, tm_k, tm_v, items, hdr, stream);
+        return aux ? launch_band_hd<64, true>(p, tm_q, tm_k, tm_v, tm_o, items, hdr, stream)
+                   : launch_band_hd<64, false>(p, tm_q, tm_k, tm_v, tm_o, items, hdr, stream);
     return cudaErrorInvalidValue;
 }
 

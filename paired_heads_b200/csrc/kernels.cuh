@@ -121,9 +121,11 @@ inline bool band_applies(const AttnProblem& p) {
     return p.causal && p.window >= 1 && p.window <= kBlockN;
 }
 
-// tcgen05 attention over a band work list (same tensor maps as launch_attn_tc).
+// tcgen05 attention over a band work list (same tensor maps as launch_attn_tc, plus tm_o: a map
+// over o like tm_q but with a 64 x 32 box, for the epilogue's stores).
 cudaError_t launch_attn_band(const AttnProblem& p, const CUtensorMap& tm_q,
-                             const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int4* items,
-                             WorkspaceHeader* hdr, cudaStream_t stream);
+                             const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const CUtensorMap& tm_o, const int4* items, WorkspaceHeader* hdr,
+                             cudaStream_t stream);
 
 }  // namespace pha

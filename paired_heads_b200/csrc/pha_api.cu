@@ -28,13 +28,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 
-// 2-D bf16 map over [rows][width] elements, box 64 x 128, 128-byte swizzle, zero fill outside.
-bool encode_slot_map(CUtensorMap* map, const void* base, uint64_t width, uint64_t rows) {
+// 2-D bf16 map over [rows][width] elements, box 64 x box_rows, 128-byte swizzle, zero fill
+// outside.
+bool encode_slot_map(CUtensorMap* map, const void* base, uint64_t width, uint64_t rows,
+                     uint32_t box_rows = 128) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
     if (!encode) return false;
     cuuint64_t dims[2] = {width, rows};
     cuuint64_t strides[1] = {width * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -329,7 +331,11 @@ pha_status attn_fwd_impl(const void* q, const void* k, const void* v, const void
         !encode_slot_map(&tk, k, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
         !encode_slot_map(&tv, v, static_cast<uint64_t>(p.kv_heads) * head_dim, rows))
         return PHA_ERR_CUDA;
-    const cudaError_t e = band ? launch_attn_band(p, tq, tk, tv, items, hdr, stream)
+    // the band kernel stores O with one 32-row box per warp
+    CUtensorMap to;
+    if (band && !encode_slot_map(&to, o, static_cast<uint64_t>(p.heads) * head_dim, rows, 32))
+        return PHA_ERR_CUDA;
+    const cudaError_t e = band ? launch_attn_band(p, tq, tk, tv, to, items, hdr, stream)
                                : launch_attn_tc(p, tq, tk, tv, items, hdr, stream);
     return e == cudaSuccess ? PHA_OK : PHA_ERR_CUDA;
 }
