@@ -87,13 +87,14 @@ cudaError_t launch_attn_bwd_zero_outside(const AttnProblem& p, void* dq, void* d
                                          cudaStream_t stream);
 
 // Backward of the band attention on the tensor cores (bf16, band_applies, head_dim 64 / 128) over
-// a band work list: the dQ kernel, then the dK / dV kernel. tm_do is a map over dout like tm_q.
-// Writes the rows inside the documents only.
+// a band work list: the dQ kernel, then the dK / dV kernel. tm_do is a map over dout like tm_q;
+// tm_dq a map over dq like tm_q with a 64 x 32 box (the dQ kernel's TMA stores). Writes the rows
+// inside the documents only.
 cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
                                const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                               const CUtensorMap& tm_do, const float* dsum, void* dq, void* dk,
-                               void* dv, const int4* items, WorkspaceHeader* hdr,
-                               cudaStream_t stream);
+                               const CUtensorMap& tm_do, const CUtensorMap& tm_dq,
+                               const float* dsum, void* dq, void* dk, void* dv, const int4* items,
+                               WorkspaceHeader* hdr, cudaStream_t stream);
 
 // RoPE preceded by the QK RMS-norm of every head row (weights may be NULL = ones).
 cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
