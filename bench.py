@@ -313,7 +313,10 @@ def main():
                            "(tcgen05)" if tc_bwd else
                            "pha_attn_bwd: D = dO.O, then dq and dk/dv on CUDA cores") +
                           "; then pha_rope_bwd",
-               "flop_count": "2.5 x the forward's causal-counted FLOPs (S, dP, dV, dK, dQ)"}
+               "flop_count": "2.5 x the forward's causal-counted FLOPs (S, dP, dV, dK, dQ)",
+               "traffic_per_launch": {"dq_kernel": load_traffic(w, "attn_bwd_dq"),
+                                      "dkdv_kernel": load_traffic(w, "attn_bwd_dkdv")}
+               if tc_bwd else None}
 
     # ---- end to end through the public API with host buffers. Documents are independent, so the
     # step is issued in chunks of whole documents on two streams: the host->device copy of one
