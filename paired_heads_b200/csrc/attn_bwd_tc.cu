@@ -54,10 +54,13 @@ struct BwdLayout {
     static constexpr int kYStages = 2;
     static constexpr int kOffX = 0;                                  // X0, X1
     static constexpr int kOffY = kOffX + 2 * kTile;                  // [stage] Y0, Y1
-    // key-major: [stage] lse2[128], D[128]; query-major: the dQ tile staged for its TMA stores
+    // key-major: [stage] lse2[128], D[128], then per warp a 16-row x 64-column staging box (2 KB)
+    // for the dK / dV TMA stores; query-major: the dQ tile staged for its TMA stores
     static constexpr int kOffVec = kOffY + kYStages * 2 * kTile;
-    static constexpr int kVecBytes = KEYMAJOR ? kYStages * 2 * 128 * 4 : kTile;
-    static constexpr int kOffBar = kOffVec + kVecBytes;
+    static constexpr int kVecBytes = KEYMAJOR ? kYStages * 2 * 128 * 4 : 0;
+    static constexpr int kOffStg = kOffVec + kVecBytes;
+    static constexpr int kStgBytes = KEYMAJOR ? 8 * 2048 : kTile;
+    static constexpr int kOffBar = kOffStg + kStgBytes;
     static constexpr int kBarBytes = 256;
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + slack to align to 1024
     static constexpr uint32_t kTmemCols = 512;
@@ -160,12 +163,14 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_st, const AttnProblem p,
+                       const __grid_constant__ CUtensorMap tm_st,
+                       const __grid_constant__ CUtensorMap tm_st2, const AttnProblem p,
                        const float* __restrict__ dsum, __nv_bfloat16* __restrict__ out_a,
                        __nv_bfloat16* __restrict__ out_b, const int4* __restrict__ items,
                        WorkspaceHeader* hdr) {
     // out_a: dQ (query-major) or dK (key-major); out_b: dV (key-major); tm_st: a map over dQ with
-    // a 64 x 32 box (query-major)
+    // a 64 x 32 box (query-major) or over dK with a 64 x 16 box (key-major); tm_st2: over dV with a
+    // 64 x 16 box (key-major)
     using L = BwdLayout<HD, KEYMAJOR>;
     static_assert(sizeof(BwdBars) <= L::kBarBytes, "barrier block");
     extern __shared__ uint8_t smem_raw[];
@@ -490,12 +495,57 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 const int out_heads = KEYMAJOR ? Hkv : H;
                 const int out_head = KEYMAJOR ? it.head / G : it.head;
                 const int64_t base = (static_cast<int64_t>(slot) * out_heads + out_head) * HD;
+                // key-major with hd 128, a warp whose 32 rows all lie inside the document: its
+                // rows of dK (times scale), then of dV (this warpgroup's 64 columns) go out
+                // through its 2 KB staging box, 16 rows (one TMA store) at a time
+                const bool tma_km = KEYMAJOR && HD == 128 && o.row0 + r0 + 31 < it.doc_end;
+                if (tma_km) {
+                    uint8_t* stg = smem + L::kOffStg + warp * 2048;
+#pragma unroll 1
+                    for (int a = 0; a < 2; ++a) {
+                        const uint32_t col0 = L::kTmAcc + (a == 0 ? HD : 0);
+                        const float mul = a == 0 ? p.scale : 1.f;
+                        uint4 w8[8];
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            uint32_t v[32];
+                            tmem_ld32(tm_lane + col0 + 32 * (2 * h + cc), v);
+                            tmem_wait_ld();
+                            regs_after_wait(v);
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                w8[4 * cc + q4] = make_uint4(
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * mul, __uint_as_float(v[8 * q4 + 1]) * mul),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * mul, __uint_as_float(v[8 * q4 + 3]) * mul),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * mul, __uint_as_float(v[8 * q4 + 5]) * mul),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * mul, __uint_as_float(v[8 * q4 + 7]) * mul));
+                        }
+#pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {
+                            if ((lane >> 4) == half) {
+                                const int r = lane & 15;  // row of the 16-row box
+#pragma unroll
+                                for (int u = 0; u < 8; ++u)
+                                    *reinterpret_cast<uint4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) = w8[u];
+                            }
+                            fence_proxy_async_smem();  // the rows are read by the async proxy (TMA)
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d(a == 0 ? &tm_st : &tm_st2, (it.head / G) * HD + 64 * h,
+                                             o.row0 + r0 + 16 * half, stg);
+                                tma_store_commit();
+                                tma_store_wait_read();  // the box is rewritten next
+                            }
+                            __syncwarp();
+                        }
+                    }
+                }
                 // query-major with hd 128 (warpgroup h owns the 64-column chunk h), a warp whose 32
                 // rows all lie inside the document: its dQ rows are staged in the TMA box layout
                 // and written by one TMA store; otherwise every thread stores its own row
                 const bool tma_rows = !KEYMAJOR && HD == 128 && o.row0 + r0 + 31 < it.doc_end;
 #pragma unroll 1
-                for (int a = 0; a < (KEYMAJOR ? 2 : 1); ++a) {
+                for (int a = 0; !tma_km && a < (KEYMAJOR ? 2 : 1); ++a) {
                     // a = 0: the dS product (dQ or dK, times scale); a = 1: dV
                     const uint32_t col0 = L::kTmAcc + (KEYMAJOR && a == 0 ? HD : 0);
                     const float mul = a == 0 ? p.scale : 1.f;
@@ -515,7 +565,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                 pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * mul, __uint_as_float(v[8 * q4 + 7]) * mul));
                             if (tma_rows) {
                                 const int u = 4 * c + q4;  // 16-byte unit of the row
-                                *reinterpret_cast<uint4*>(smem + L::kOffVec + (u >> 3) * L::kChunk +
+                                *reinterpret_cast<uint4*>(smem + L::kOffStg + (u >> 3) * L::kChunk +
                                                           row * 128 + (((u & 7) ^ (row & 7)) << 4)) = w4;
                             } else if (valid) {
                                 *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q4) = w4;
@@ -528,7 +578,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     __syncwarp();
                     if (lane == 0) {
                         tma_store_2d(&tm_st, it.head * HD + 64 * h, o.row0 + r0,
-                                     smem + L::kOffVec + h * L::kChunk + r0 * 128);
+                                     smem + L::kOffStg + h * L::kChunk + r0 * 128);
                         tma_store_commit();
                         tma_store_wait_read();  // the staging area is rewritten by the next tile
                     }
@@ -541,7 +591,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     }
 
     // ---------------------------------------------------------------- teardown
-    if (!KEYMAJOR && warp < 8 && lane == 0) tma_store_wait_all();  // dQ stores have completed
+    if (warp < 8 && lane == 0) tma_store_wait_all();  // the epilogue's TMA stores have completed
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -551,7 +601,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 template <int HD, bool KEYMAJOR>
 cudaError_t launch_bwd_tc_one(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
                               const CUtensorMap& tv, const CUtensorMap& tdo,
-                              const CUtensorMap& tst, const float* dsum,
+                              const CUtensorMap& tst, const CUtensorMap& tst2, const float* dsum,
                               __nv_bfloat16* out_a, __nv_bfloat16* out_b, const int4* items,
                               WorkspaceHeader* hdr, int sms, cudaStream_t stream) {
     using L = BwdLayout<HD, KEYMAJOR>;
@@ -559,14 +609,15 @@ cudaError_t launch_bwd_tc_one(const AttnProblem& p, const CUtensorMap& tq, const
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     attn_bwd_tc_kernel<HD, KEYMAJOR><<<sms, kBwdTcThreads, L::kSmemBytes, stream>>>(
-        tq, tk, tv, tdo, tst, p, dsum, out_a, out_b, items, hdr);
+        tq, tk, tv, tdo, tst, tst2, p, dsum, out_a, out_b, items, hdr);
     return cudaGetLastError();
 }
 
 template <int HD>
 cudaError_t launch_bwd_tc_hd(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, const CUtensorMap& tdo,
-                             const CUtensorMap& tdq, const float* dsum,
+                             const CUtensorMap& tdq, const CUtensorMap& tdk,
+                             const CUtensorMap& tdv, const float* dsum,
                              void* dq, void* dk, void* dv, const int4* items, WorkspaceHeader* hdr,
                              cudaStream_t stream) {
     int dev = 0, sms = 0;
@@ -574,10 +625,10 @@ cudaError_t launch_bwd_tc_hd(const AttnProblem& p, const CUtensorMap& tq, const 
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    if ((e = launch_bwd_tc_one<HD, false>(p, tq, tk, tv, tdo, tdq, dsum, static_cast<__nv_bfloat16*>(dq),
+    if ((e = launch_bwd_tc_one<HD, false>(p, tq, tk, tv, tdo, tdq, tdq, dsum, static_cast<__nv_bfloat16*>(dq),
                                           nullptr, items, hdr, sms, stream)) != cudaSuccess)
         return e;
-    return launch_bwd_tc_one<HD, true>(p, tq, tk, tv, tdo, tdq, dsum, static_cast<__nv_bfloat16*>(dk),
+    return launch_bwd_tc_one<HD, true>(p, tq, tk, tv, tdo, tdk, tdv, dsum, static_cast<__nv_bfloat16*>(dk),
                                        static_cast<__nv_bfloat16*>(dv), items, hdr, sms, stream);
 }
 
@@ -586,14 +637,15 @@ cudaError_t launch_bwd_tc_hd(const AttnProblem& p, const CUtensorMap& tq, const 
 cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
                                const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                const CUtensorMap& tm_do, const CUtensorMap& tm_dq,
+                               const CUtensorMap& tm_dk, const CUtensorMap& tm_dv,
                                const float* dsum, void* dq, void* dk, void* dv, const int4* items,
                                WorkspaceHeader* hdr, cudaStream_t stream) {
     if (!band_applies(p)) return cudaErrorInvalidValue;
     if (p.head_dim == 128)
-        return launch_bwd_tc_hd<128>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, dsum, dq, dk, dv, items, hdr,
+        return launch_bwd_tc_hd<128>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq, dk, dv, items, hdr,
                                      stream);
     if (p.head_dim == 64)
-        return launch_bwd_tc_hd<64>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, dsum, dq, dk, dv, items, hdr,
+        return launch_bwd_tc_hd<64>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq, dk, dv, items, hdr,
                                     stream);
     return cudaErrorInvalidValue;
 }

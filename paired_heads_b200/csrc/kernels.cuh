@@ -88,11 +88,12 @@ cudaError_t launch_attn_bwd_zero_outside(const AttnProblem& p, void* dq, void* d
 
 // Backward of the band attention on the tensor cores (bf16, band_applies, head_dim 64 / 128) over
 // a band work list: the dQ kernel, then the dK / dV kernel. tm_do is a map over dout like tm_q;
-// tm_dq a map over dq like tm_q with a 64 x 32 box (the dQ kernel's TMA stores). Writes the rows
-// inside the documents only.
+// tm_dq a map over dq like tm_q with a 64 x 32 box, tm_dk / tm_dv maps over dk / dv like tm_k
+// with a 64 x 16 box (the epilogues' TMA stores). Writes the rows inside the documents only.
 cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
                                const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                const CUtensorMap& tm_do, const CUtensorMap& tm_dq,
+                               const CUtensorMap& tm_dk, const CUtensorMap& tm_dv,
                                const float* dsum, void* dq, void* dk, void* dv, const int4* items,
                                WorkspaceHeader* hdr, cudaStream_t stream);
 

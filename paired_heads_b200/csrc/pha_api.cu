@@ -236,15 +236,18 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void*
                    ? PHA_OK
                    : PHA_ERR_CUDA;
     const uint64_t rows = static_cast<uint64_t>(total_tokens) * p.slot_mult;
-    CUtensorMap tq, tk, tv, tdo, tdq;
+    CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
     if (!encode_slot_map(&tq, q, static_cast<uint64_t>(p.heads) * head_dim, rows) ||
         !encode_slot_map(&tk, k, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
         !encode_slot_map(&tv, v, static_cast<uint64_t>(p.kv_heads) * head_dim, rows) ||
         !encode_slot_map(&tdo, dout, static_cast<uint64_t>(p.heads) * head_dim, rows) ||
-        !encode_slot_map(&tdq, dq, static_cast<uint64_t>(p.heads) * head_dim, rows, 32))
+        !encode_slot_map(&tdq, dq, static_cast<uint64_t>(p.heads) * head_dim, rows, 32) ||
+        !encode_slot_map(&tdk, dk, static_cast<uint64_t>(p.kv_heads) * head_dim, rows, 16) ||
+        !encode_slot_map(&tdv, dv, static_cast<uint64_t>(p.kv_heads) * head_dim, rows, 16))
         return PHA_ERR_CUDA;
     if (launch_attn_bwd_zero_outside(p, dq, dk, dv, stream) != cudaSuccess ||
-        launch_attn_bwd_tc(p, tq, tk, tv, tdo, tdq, dsum, dq, dk, dv, items, hdr, stream) !=
+        launch_attn_bwd_tc(p, tq, tk, tv, tdo, tdq, tdk, tdv, dsum, dq, dk, dv, items, hdr,
+                           stream) !=
             cudaSuccess)
         return PHA_ERR_CUDA;
     return PHA_OK;
