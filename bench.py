@@ -467,7 +467,7 @@ def main():
 
 def load_traffic(w, kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it matches this workload and
-    the current kernel sources; else None."""
+    the kernel's current sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -479,7 +479,9 @@ def load_traffic(w, kernel: str):
         return None
     from paired_heads_b200 import build as b
 
-    if ent.get("sources_sha") != b.sources_sha():
+    # valid while the files that define this kernel's device code are those that were captured
+    now = b.files_sha(ent["sources"]) if "sources" in ent else b.sources_sha()
+    if ent.get("sources_sha") != now:
         return None
     return ent.get("bytes_per_launch")
 

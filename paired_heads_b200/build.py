@@ -57,6 +57,17 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
 
 
 
+def files_sha(rel_paths) -> str:
+    """sha256 over the given repository files (paths relative to the repository root)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in rel_paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(os.path.basename(rel).encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
 def sources_sha() -> str:
     """sha256 over the kernel sources and the ABI header (identifies a kernel build)."""
     import hashlib
