@@ -10,10 +10,11 @@ a difference of large terms, so a tolerance scaled by the tensor's maximum does 
 error. bf16 gradients are therefore bounded per element, from the rounding steps of the
 tensor-core path (u = 2^-8, the unit roundoff of bf16's 8 significant bits); the CUDA-core path's
 rounding steps are a subset of these:
-  O (stored bf16, from bf16 P):  |dO_e| <= 2u sum_j P_ij |v_je|
-  so D = dO . O:                 |dD_i| <= 2u A_i,  A_i = sum_j P_ij (|dO_i| . |v_j|)
-  dS (bf16 of P (dP - D)):       |ddS_ij| <= u |dS_ij| + P_ij |dD_i|
-  dq = scale dS K, dk = scale dS^T Q:  scale sum |ddS| |k| (|q|), + u |result| (stored bf16)
+(err(x) is the error of the computed x; dO, dP, dS are gradients)
+  O (stored bf16, from bf16 P):  err(O_ie) <= 2u sum_j P_ij |v_je|
+  so D = dO . O:                 err(D_i) <= 2u A_i,  A_i = sum_j P_ij (|dO_i| . |v_j|)
+  dS (bf16 of P (dP - D)):       err(dS_ij) <= u |dS_ij| + P_ij err(D_i)
+  dq = scale dS K, dk = scale dS^T Q:  scale sum err(dS) |k| (|q|), + u |result| (stored bf16)
   dv = P^T dO with P in bf16:    u sum_i P_ij |dO_ie| + u |dv|
 each evaluated in float64 from the inputs and the exact P, dS, and allowed 1.25 times (the float32
 sums, the exponentials and the lse add relative errors near 1e-6 of the same terms). f32
