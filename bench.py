@@ -328,7 +328,7 @@ def main():
     o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
     lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
     cu_h = host["cu_seqlens"].tolist()
-    n_chunks = max(1, min(4, w.batch))
+    n_chunks = max(1, min(8, w.batch))
     chunks = []  # (first doc, last doc + 1): contiguous groups of about equal token counts
     d0 = 0
     for c in range(n_chunks):
