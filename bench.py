@@ -53,6 +53,28 @@ def visible_pairs(w) -> int:
     return total * heads
 
 
+def doc_chunks(cu, n_chunks: int):
+    """Split documents 0 .. len(cu) - 2 (token offsets cu) into at most n_chunks contiguous groups
+    of about equal token counts: a list of (first doc, last doc + 1), covering every document once,
+    each group holding at least one document."""
+    batch = len(cu) - 1
+    chunks = []
+    d0 = 0
+    for c in range(n_chunks):
+        target = cu[-1] * (c + 1) / n_chunks
+        d1 = d0 + 1
+        while d1 < batch and (cu[d1] < target or d1 == d0) and c < n_chunks - 1:
+            d1 += 1
+        if c == n_chunks - 1:
+            d1 = batch
+        if d1 > d0:
+            chunks.append((d0, d1))
+        d0 = d1
+        if d0 >= batch:
+            break
+    return chunks
+
+
 def attn_flops(w) -> float:
     return 4.0 * w.head_dim * visible_pairs(w)
 
@@ -328,21 +350,7 @@ def main():
     o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
     lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
     cu_h = host["cu_seqlens"].tolist()
-    n_chunks = max(1, min(8, w.batch))
-    chunks = []  # (first doc, last doc + 1): contiguous groups of about equal token counts
-    d0 = 0
-    for c in range(n_chunks):
-        target = cu_h[-1] * (c + 1) / n_chunks
-        d1 = d0 + 1
-        while d1 < w.batch and (cu_h[d1] < target or d1 == d0) and c < n_chunks - 1:
-            d1 += 1
-        if c == n_chunks - 1:
-            d1 = w.batch
-        if d1 > d0:
-            chunks.append((d0, d1))
-        d0 = d1
-        if d0 >= w.batch:
-            break
+    chunks = doc_chunks(cu_h, max(1, min(8, w.batch)))
     streams = [torch.cuda.Stream(dev) for _ in range(2)]
     parts = []
     for (a0, a1) in chunks:

@@ -1,0 +1,88 @@
+"""Host logic of bench.py (no GPU): the algorithmic counters against brute force, the e2e leg's
+partition of documents into chunks, and the validity check of the committed ncu traffic."""
+import importlib.util
+import json
+import os
+
+import numpy as np
+import pytest
+
+from paired_heads_b200 import build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("lens,H,causal,window,paired", [
+    ((5, 1, 12), 4, True, 0, False),
+    ((5, 1, 12), 4, True, 3, False),
+    ((7, 9), 2, False, 0, False),
+    ((7, 9, 1), 6, True, 4, True),
+    ((130,), 2, True, 128, True),
+])
+def test_visible_pairs_brute_force(bench, lens, H, causal, window, paired):
+    w = synth.Workload("t", lens, H, H, 16, "bf16", causal=causal, window=window, paired=paired)
+    m = 2 if paired else 1
+    want = 0
+    for n in lens:
+        L = n * m
+        i, j = np.arange(L)[:, None], np.arange(L)[None, :]
+        vis = np.ones((L, L), dtype=bool)
+        if causal:
+            vis &= j <= i
+            if window > 0:
+                vis &= i - j < window
+        want += int(vis.sum())
+    want *= H // m
+    assert bench.visible_pairs(w) == want
+    assert bench.attn_flops(w) == 4.0 * 16 * want
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("n_chunks", [1, 2, 4, 8])
+def test_doc_chunks_partition(bench, seed, n_chunks):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, 300, rng.integers(1, 40))   # zero-length documents included
+    cu = [0] + np.cumsum(lens).tolist()
+    chunks = bench.doc_chunks(cu, n_chunks)
+    assert 1 <= len(chunks) <= n_chunks
+    assert chunks[0][0] == 0 and chunks[-1][1] == len(lens)
+    for (a0, a1), (b0, _) in zip(chunks, chunks[1:]):
+        assert a1 == b0                                 # contiguous, each document once
+    assert all(a1 > a0 for a0, a1 in chunks)            # no empty group
+
+
+def test_load_traffic_follows_the_sources(bench, tmp_path, monkeypatch):
+    w = synth.workload("paired_varlen")
+    srcs = ["paired_heads_b200/csrc/rope.cu", "paired_heads_b200/csrc/ptx.cuh"]
+    key = f"{w.name}:w{w.window}:p{int(w.paired)}:rope"
+    (tmp_path / "profiles").mkdir()
+
+    def write(entry):
+        (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({key: entry}))
+
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    write({"bytes_per_launch": 123, "sources": srcs, "sources_sha": build.files_sha(srcs)})
+    assert bench.load_traffic(w, "rope") == 123
+    write({"bytes_per_launch": 123, "sources": srcs, "sources_sha": "0" * 16})
+    assert bench.load_traffic(w, "rope") is None       # a kernel source changed since the capture
+    assert bench.load_traffic(w, "attention") is None  # no entry
+    assert bench.load_traffic(synth.workload("gpt2"), "rope") is None
+
+
+def test_committed_traffic_entries_name_existing_sources():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    for key, ent in d.items():
+        if key.startswith("_"):
+            continue
+        assert ent["bytes_per_launch"] == ent["read"] + ent["write"]
+        for rel in ent["sources"]:
+            assert os.path.exists(os.path.join(ROOT, rel)), rel
