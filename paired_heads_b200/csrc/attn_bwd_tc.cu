@@ -22,6 +22,9 @@
 // 256 + hd (dK).
 // A tile loaded for the K-major S / dP product (rows = slots, [64-column chunks] 128-byte
 // swizzled) is the MN-major B operand of the second product as it stands.
+// Epilogue (hd 128): a warp whose 32 rows lie inside the document stages them in shared memory in
+// the TMA box layout and writes them with TMA stores (dQ: a 32 KB tile, one 64 x 32 box per warp;
+// dK, dV: a private 2 KB box per warp, 16 rows per store); other warps store row by row.
 //
 // CTA = 10 warps, persistent, one per SM, band items in snake order:
 //   warps 0-7  elementwise, two warpgroups: warpgroup h takes half h of every inner step (row =
