@@ -404,6 +404,31 @@ def test_round_bf16_matches_torch_on_float32_values():
     np.testing.assert_array_equal(oracle.round_bf16(x.astype(np.float64)), ref)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("paired,stagger", [(False, False), (True, False), (True, True)])
+def test_rope_stored_is_the_rotation_rounded_once(dtype, paired, stagger):
+    # The stored RoPE output is a value of the buffer's dtype within half a unit in its last
+    # place of the unrounded rotation (float32 table values), and position 0 (phase 0: cos 1,
+    # sin 0) leaves an input that is already in the dtype unchanged.
+    torch = pytest.importorskip("torch")
+    tdt, bits = (torch.bfloat16, 8) if dtype == "bf16" else (torch.float32, 24)
+    rng = np.random.default_rng(31)
+    x = torch.from_numpy(rng.standard_normal((64, 4, 32)).astype(np.float32)).to(tdt)
+    x = x.to(torch.float64).numpy()
+    pos = rng.integers(0, 5000, 64).astype(np.int32)
+    pos[:4] = 0
+    y = oracle.rope_stored(x, pos, dtype, paired, stagger)
+    # values of the dtype
+    np.testing.assert_array_equal(torch.from_numpy(y).to(tdt).to(torch.float64).numpy(), y)
+    # within half an ulp of the unrounded rotation
+    u = oracle.rope(x, pos, paired, stagger, table_f32=True)
+    half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(u), 2.0 ** -120))) - bits)
+    assert np.all(np.abs(y - u) <= half_ulp)
+    # phase 0: tokens at position 0 (every head unless the odd heads are staggered)
+    heads = slice(None) if not stagger else slice(0, None, 2)
+    np.testing.assert_array_equal(y[:4, heads], x[:4, heads])
+
+
 def test_float32_tables_only_perturb_by_float32_rounding():
     # Rounding cos / sin to float32 changes each rotated element by at most
     # 2^-24 (|x_2i| + |x_2i+1|) (one float32 half-ulp on each factor of magnitude <= 1).
