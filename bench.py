@@ -218,12 +218,29 @@ def main():
     ap.add_argument("--aux-v", action="store_true",
                     help="add a value embedding to v inside attention (pha_attn_fwd_aux_v)")
     ap.add_argument("--oracle-tokens", type=int, default=16384)
+    ap.add_argument("--no-suite", action="store_true",
+                    help="skip the per-workload timings of the other page-shaped workloads")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="start the ranks, join a gloo group, print each rank's id and exit "
+                         "(tests the multi-process launch without a GPU)")
     args = ap.parse_args()
     w = pick_workload(args)
 
     from paired_heads_b200 import dist as pdist
 
     rank, world, local_rank = pdist.env()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit(launch_ranks(args.gpus))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks were launched")
+
+    if args.launch_check:
+        d = pdist.init("gloo", timeout_s=60)
+        ranks = pdist.gather_ints(d, rank)
+        if rank == 0:
+            print(json.dumps({"launch_check": True, "world": world, "ranks": ranks}))
+        pdist.finalize(d)
+        return
 
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
@@ -461,6 +478,8 @@ def main():
     }
     if bwd is not None:
         line["backward"] = bwd
+    if not args.no_suite and args.workload == "paired_varlen" and not (args.qk_norm or args.aux_v):
+        line["configs"] = time_suite(max(3, min(args.steps, 20)), args.warmup, dev, peaks, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, s, thr = time_oracle(w, args.oracle_tokens, args.qk_norm)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
@@ -471,6 +490,97 @@ def main():
     if rank == 0:
         print(json.dumps(line))
     pdist.finalize(dist)
+
+
+# The other workloads of the page-shaped suite, timed after the headline in the default run:
+# (label, workload, overrides). The mixed-window workload runs at each window, paired or not.
+SUITE = (
+    ("gpt2", "gpt2", {}),
+    ("mixed_window_w128", "mixed_window", {"window": 128}),
+    ("mixed_window_w128_paired", "mixed_window", {"window": 128, "paired": True, "stagger": True}),
+    ("mixed_window_w1024", "mixed_window", {"window": 1024}),
+    ("mixed_window_w1024_paired", "mixed_window", {"window": 1024, "paired": True, "stagger": True}),
+    ("mixed_window_full", "mixed_window", {"window": 0}),
+    ("mixed_window_full_paired", "mixed_window", {"window": 0, "paired": True, "stagger": True}),
+    ("gqa_long", "gqa_long", {}),
+)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def time_suite(steps: int, warmup: int, dev, peaks, rank: int = 0):
+    """RoPE + attention on each workload of SUITE, timed per call with CUDA events on the launching
+    stream. Workloads whose inputs fit in L2 get a 256 MiB buffer written before every step (outside
+    the events). Returns {label: {...}}."""
+    import torch
+
+    from paired_heads_b200.runner import AttentionStep, StepShape
+
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {}
+    for label, name, kw in SUITE:
+        w = synth.workload(name, **kw)
+        inp = synth.make_inputs(w, rank=rank)
+        q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+        cu, pos = inp["cu_seqlens"].to(dev), inp["positions"].to(dev)
+        step = AttentionStep(StepShape.of(w, int(inp["positions"].max()) + 1), dev)
+        tab_width = (2 if w.paired else 1) * w.head_dim
+        in_l2 = attn_bytes(w) + rope_bytes(w, tab_width) < L2_BYTES
+        for _ in range(max(warmup, 3)):
+            step.rope(q, k, pos)
+            step.attn(q, k, v, cu)
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        sampler = ClockSampler(dev.index if dev.index is not None else 0)
+        sampler.start()
+        time.sleep(0.2)
+        for s in range(steps):
+            if in_l2:
+                flush.fill_(s & 0xFF)
+            ev[s][0].record(stream)
+            step.rope(q, k, pos)
+            ev[s][1].record(stream)
+            step.attn(q, k, v, cu)
+            ev[s][2].record(stream)
+        torch.cuda.synchronize(dev)
+        clk = sampler.stop()
+        status, _ = step.status()
+        if status != 0:
+            raise SystemExit(f"{label}: device status {status}")
+        rope_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        flops, ab = attn_flops(w), attn_bytes(w)
+        tflops = flops / (attn_ms * 1e-3) / 1e12
+        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        bound = "hbm" if flops / ab < ridge else "tensor"
+        roof_tflops = min(peaks["bf16_tflops"], flops / ab * peaks["hbm_gbs"] * 1e9 / 1e12)
+        out[label] = {
+            "tokens": w.total, "n_heads": w.n_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "window": w.window, "paired": w.paired,
+            "kernel": "band" if (w.causal and 1 <= w.window <= 128) else "block",
+            "attn_ms": attn_ms, "attn_tflops": tflops,
+            "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+            "bound": bound, "frac_of_roofline": tflops / roof_tflops,
+            "attn_gbs": ab / (attn_ms * 1e-3) / 1e9,
+            "rope_ms": rope_ms, "rope_gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9,
+            "step_ms": rope_ms + attn_ms,
+            "tokens_per_s": w.total / ((rope_ms + attn_ms) * 1e-3),
+            "l2": "flushed (256 MiB write) before each step" if in_l2 else "inputs larger than L2",
+            "steps": steps, "sm_mhz": clk.get("sm_mhz"), "clock_reasons": clk.get("reasons"),
+        }
+        del q, k, v, cu, pos, step, inp
+        torch.cuda.empty_cache()
+    return out
+
+
+def launch_ranks(n: int) -> int:
+    """Re-run this command as n processes on one node (one per GPU) under torch.distributed.run.
+    Returns the launcher's exit code."""
+    port = int(os.environ.get("MASTER_PORT", "29517"))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def load_traffic(w, kernel: str):

@@ -248,10 +248,14 @@ pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha
  *   scratch is a 1 MiB array inside the library, one per GPU, held by every GPU that loads the
  *   library until the process exits. The call itself allocates nothing.
  *   Limit: problems whose pha_attn_workspace_bytes(...) exceeds 1 MiB are rejected with
- *   PHA_ERR_WORKSPACE before any launch (PHA_F32 uses no scratch and has no such limit).
- *   Set-up: the first call on a device looks up the array's device address, with the calling
- *   thread's current device; that device must be the one `stream` belongs to. Make that first
- *   call before any stream capture.
+ *   PHA_ERR_WORKSPACE before any launch, after the argument checks of pha_attn_fwd (PHA_F32 uses
+ *   no scratch and has no such limit).
+ *   Set-up: the first call in a CUDA context on a device looks up the array's device address,
+ *   with the calling thread's current device; that device must be the one `stream` belongs to.
+ *   Make that first call before any stream capture. A new context on the device (after
+ *   cudaDeviceReset, or after the primary context was released and created again) loads the
+ *   library's device code afresh; the next call notices the new context and looks the address
+ *   up again, so that first call should also come before any capture.
  *   Sharing: every call uses the same array, which keeps the last call's contents. Nothing in it
  *   needs to start at zero (each call rewrites what it reads). Calls whose kernels can run at the
  *   same time on one GPU (unordered streams, several host threads) race on the array; order them

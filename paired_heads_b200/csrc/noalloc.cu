@@ -9,6 +9,7 @@
 //
 // The array is kNoAllocScratchBytes (1 MiB) per GPU and is held by every GPU that loads the
 // library until the process exits. Problems whose work list needs more than that are rejected.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -25,23 +26,51 @@ constexpr int kMaxDevices = 64;
 // comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// Per device: the CUDA context in which the address was looked up, and the address. A new
+// context on the device (after cudaDeviceReset, or once the primary context has been released
+// and created again) loads the module afresh, so the address is looked up again.
+struct ScratchSlot {
+    CUcontext ctx;
+    void* addr;
+};
 std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch per device, once set up
+ScratchSlot g_scratch[kMaxDevices];
 
-// Device address of the scratch array on the calling thread's current device. The first call
-// on a device resolves it (with that device current) and remembers it.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn get_ctx_fn() {
+    // Resolved through the runtime so that the library does not link libcuda directly.
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(fn);
+}
+
+// Device address of the scratch array in the calling thread's current device and context.
+// The first call in a context resolves it (with that device current) and remembers it.
 pha_status scratch_on_current_device(void** addr) {
+    static CtxGetCurrentFn ctx_get = get_ctx_fn();
+    if (!ctx_get) return PHA_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PHA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return PHA_ERR_UNSUPPORTED;
+    CUcontext ctx = nullptr;  // NULL while no context is current on this thread yet
+    if (ctx_get(&ctx) != CUDA_SUCCESS) return PHA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchSlot& slot = g_scratch[dev];
+    if (ctx == nullptr || slot.addr == nullptr || slot.ctx != ctx) {
+        // the lookup makes the device's primary context current when none is
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
             return PHA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        if (ctx == nullptr && (ctx_get(&ctx) != CUDA_SUCCESS || ctx == nullptr))
+            return PHA_ERR_CUDA;
+        slot.ctx = ctx;
+        slot.addr = p;
     }
-    *addr = g_scratch_addr[dev];
+    *addr = slot.addr;
     return PHA_OK;
 }
 
@@ -53,16 +82,13 @@ extern "C" pha_status pha_attn_fwd_noalloc(const void* q, const void* k, const v
                                            int head_dim, pha_dtype dtype, int causal, int window,
                                            int paired, float scale, void* o, float* lse,
                                            pha_stream_t stream) {
-    if (dtype == PHA_BF16) {
-        const size_t need = pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired);
-        if (need == 0) return PHA_ERR_INVALID;
-        if (need > kNoAllocScratchBytes) return PHA_ERR_WORKSPACE;  // beyond the built-in 1 MiB
-    }
     void* scratch = nullptr;
     const pha_status st = scratch_on_current_device(&scratch);
     if (st != PHA_OK) return st;
-    // Nothing in the scratch has to start at zero: the scheduler kernel writes the header, the
-    // per-document offsets and every work item the attention kernel then reads.
+    // pha_attn_fwd checks the arguments first, then rejects a work list larger than the array
+    // with PHA_ERR_WORKSPACE, before any launch. Nothing in the scratch has to start at zero:
+    // the scheduler kernel writes the header, the per-document offsets and every work item the
+    // attention kernel then reads.
     return pha_attn_fwd(q, k, v, cu_seqlens, batch, max_len, total_tokens, n_heads, n_kv_heads,
                         head_dim, dtype, causal, window, paired, scale, o, lse, scratch,
                         kNoAllocScratchBytes, stream);

@@ -42,6 +42,18 @@ def max_over_ranks(dist, value: float, device=None) -> float:
     return float(t.item())
 
 
+def gather_ints(dist, value: int) -> list:
+    """Every rank's integer, in rank order (a one-element list for a single process)."""
+    if dist is None:
+        return [int(value)]
+    import torch
+
+    t = torch.tensor([int(value)], dtype=torch.int64)
+    out = [torch.zeros_like(t) for _ in range(dist.get_world_size())]
+    dist.all_gather(out, t)
+    return [int(x.item()) for x in out]
+
+
 def barrier(dist):
     if dist is not None:
         dist.barrier()

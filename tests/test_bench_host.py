@@ -86,3 +86,25 @@ def test_committed_traffic_entries_name_existing_sources():
         assert ent["bytes_per_launch"] == ent["read"] + ent["write"]
         for rel in ent["sources"]:
             assert os.path.exists(os.path.join(ROOT, rel)), rel
+
+
+def test_gpus_two_starts_two_ranks():
+    """`bench.py --gpus 2` run without a launcher re-runs itself as two processes under
+    torch.distributed.run; --launch-check makes each rank join a gloo group and report its id."""
+    import socket
+    import subprocess
+    import sys
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["MASTER_PORT"] = str(port)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--launch-check"], capture_output=True, text=True, timeout=240, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["world"] == 2 and d["ranks"] == [0, 1]
