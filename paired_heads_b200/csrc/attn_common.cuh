@@ -41,7 +41,14 @@ struct TcBars {
     int abort;
 };
 
-constexpr int kTcThreads = 320;
+// Block kernel (attn_tc.cu): two softmax warpgroups, then a third warpgroup whose warps 8 and 9 are
+// the TMA producer and the MMA issuer (10 and 11 only give the register split a whole warpgroup).
+constexpr int kTcThreads = 384;
+// Register split of the block kernel, per thread: the softmax warpgroups hold a whole 128-column
+// score row in registers. 8 warps x 200 + 4 warps x 88 = 1952 <= 12 warps x 168 (the launch
+// allocation), so the increase never waits for registers that cannot be freed.
+constexpr int kTcRegsSoftmax = 200;
+constexpr int kTcRegsOther = 88;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -131,6 +138,47 @@ __device__ __forceinline__ uint64_t row_exp64(const uint32_t* v, int base, int c
         pk[e >> 1] = pack_bf16x2(pa, pb);
     }
     return sum2;
+}
+
+// Row routines over a whole 32-column chunk held in registers, with independent accumulator
+// chains (the max and the sum are associative up to rounding of the sum, which the softmax's
+// float32 accumulation already allows).
+
+// Max of the visible scores among 32 columns starting at `base` (-inf if none is visible).
+template <int MODE>
+__device__ __forceinline__ float chunk_max(const uint32_t* v, int base, int c_lo, int c_hi) {
+    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            m[j] = fmax3(m[j], mask_col<MODE>(__uint_as_float(v[e + 2 * j]), base + e + 2 * j, c_lo, c_hi),
+                         mask_col<MODE>(__uint_as_float(v[e + 2 * j + 1]), base + e + 2 * j + 1, c_lo, c_hi));
+    }
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p = 2^(s * scale_log2 - m) for 32 columns (0 where masked), packed into 16 bf16 pairs; the
+// values are added into two packed partial sums.
+template <int MODE>
+__device__ __forceinline__ void chunk_exp(const uint32_t* v, int base, int c_lo, int c_hi,
+                                          uint64_t scale2, uint64_t negm2, uint64_t& sum_a,
+                                          uint64_t& sum_b, uint32_t* pk) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+        const float a0 = mask_col<MODE>(__uint_as_float(v[e]), base + e, c_lo, c_hi);
+        const float a1 = mask_col<MODE>(__uint_as_float(v[e + 1]), base + e + 1, c_lo, c_hi);
+        const float a2 = mask_col<MODE>(__uint_as_float(v[e + 2]), base + e + 2, c_lo, c_hi);
+        const float a3 = mask_col<MODE>(__uint_as_float(v[e + 3]), base + e + 3, c_lo, c_hi);
+        float x0, x1, x2, x3;
+        f32x2_split(fma_f32x2(f32x2(a0, a1), scale2, negm2), x0, x1);
+        f32x2_split(fma_f32x2(f32x2(a2, a3), scale2, negm2), x2, x3);
+        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+        sum_a = add_f32x2(sum_a, f32x2(p0, p1));
+        sum_b = add_f32x2(sum_b, f32x2(p2, p3));
+        pk[e >> 1] = pack_bf16x2(p0, p1);
+        pk[(e >> 1) + 1] = pack_bf16x2(p2, p3);
+    }
 }
 
 // Band work item (see kernels.cuh), decoded.

@@ -9,30 +9,37 @@
 // forward pass" and "sequence length and window handling").
 //
 // A work item is a block of up to 256 query slots split into two 128-row sub-tiles r = 0, 1 that
-// share one stream of 128-key K / V tiles. CTA = 10 warps, persistent (one CTA per SM, static
-// round-robin over the longest-first work list):
+// share one stream of 128-key K / V tiles. CTA = 12 warps, persistent (one CTA per SM; the
+// longest-first work list is dealt out in snake order); the softmax warpgroups run with 200
+// registers per thread, the third warpgroup with 88:
 //   warps 0-3   softmax of sub-tile 0      warps 4-7   softmax of sub-tile 1
-//               thread = query row = TMEM lane. Two passes over the S row in TMEM (row max with
-//               three-input max, then exponentials with packed f32x2 arithmetic). Masks are
-//               applied only on tiles that straddle a causal / window / document edge, and only
-//               the bound(s) that tile needs. P (bf16) goes back into the first 64 columns of its
-//               own S buffer; O is rescaled in TMEM only when the running max grew by more than
-//               2^8. At the end the row is normalised and O and the LSE are stored.
+//               thread = query row = TMEM lane. The whole 128-column S row is loaded from TMEM
+//               with one wait, its max and its exponentials are taken from registers with
+//               independent accumulator chains, and P (bf16) is written back to TMEM. Masks are
+//               applied only on tiles that straddle a causal / window / document edge, per
+//               32-column chunk and only where some row of the warp needs them. O is rescaled in
+//               TMEM only when the running max grew by more than 2^8. At the end the row is
+//               normalised and O and the LSE are stored.
 //   warp 8      TMA producer: Q sub-tiles into a ring of 3 slots (so the next item's Q arrives
 //               while the current item computes), K and V tiles into their rings (64-column x
 //               128-row boxes, 128-byte swizzle).
-//   warp 9      MMA issuer (one thread) and TMEM owner (512 columns):
+//   warp 9      MMA issuer (one thread) and TMEM owner (512 columns); warps 10 and 11 idle:
 //               S_r = Q_r K^T   tcgen05.mma kind::f16, A and B from shared memory, M=128 N=128
 //               O_r += P_r V    tcgen05.mma kind::f16, A (P) from TMEM, B (V) from shared memory
-//               Per key tile: S_0, S_1, then (when P_r is ready) O_0 += P_0 V, O_1 += P_1 V, so
-//               the tensor core works on one sub-tile while the other runs its softmax. A
-//               sub-tile skips the key tiles that lie wholly outside its own causal / window
-//               range.
-// TMEM columns: S_r at 128 r (P_r aliases its first 64 columns), O_r at 256 + hd r.
-// Ordering: before S_r of a new tile is issued the MMA thread waits until O_r += P_r V of the
-// previous tile has completed (pv_done[r]), because S_r overwrites the TMEM columns holding P_r.
-// The commit that signals S_r (s_full[r]) therefore also covers that P.V, so the softmax may
-// then overwrite P_r and rescale O_r.
+//               The issue order is software-pipelined per sub-tile: once P_r of key tile g-1 is
+//               ready, O_r += P_r V_{g-1} is issued and then at once S_r of key tile g, so sub-tile
+//               r's next softmax starts while the other sub-tile's softmax is still running and
+//               the tensor core alternates between the two. A sub-tile skips the key tiles that
+//               lie wholly outside its own causal / window range.
+// TMEM columns: S_r at 128 r, O_r at 256 + hd r. P_r: hd 64 -- columns 384 + 64 r, apart from S_r,
+// so S_r of the next tile never waits for the P.V that reads P_r; hd 128 -- the first 64 columns
+// of S_r (all 512 columns are taken), so before S_r of the next tile is issued the MMA thread
+// waits until that P.V has completed.
+// Ordering: the commit that signals S_r of a tile (s_full[r]) follows the previous tile's
+// O_r += P_r V, so when the softmax sees S_r, that P.V is complete: P_r may be overwritten and O_r
+// rescaled. At a work item's first key tile the P.V products that end the previous item's
+// sub-tiles are issued before anything of the new item is awaited (their epilogues free the Q
+// slots the producer waits for).
 // Every wait is bounded (1 s); on expiry the CTA records a status, drains its own in-flight
 // copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -85,6 +92,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __grid_constant__ CUtensorMap tm_v, const AttnProblem p,
                    const int4* __restrict__ items, WorkspaceHeader* hdr) {
     using L = TcLayout<HD>;
+    // P_r apart from S_r where TMEM has room for it (hd 64), else in the first 64 columns of S_r.
+    constexpr bool kSepP = HD == 64;
+    constexpr uint32_t kTmP = kSepP ? L::kTmO + 2 * HD : 0;
+    static_assert(!kSepP || kTmP + 128 <= L::kTmemCols, "TMEM columns");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -134,16 +145,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads;
     const int G = p.heads / p.kv_heads;
+    static_assert(8 * kTcRegsSoftmax + 4 * kTcRegsOther <= 12 * 168, "register split");
 
-    if (warp == 8) {
+    if (warp >= 8) regs_decrease<kTcRegsOther>();  // the whole third warpgroup, then its roles
+    if (warp >= 10) {
+        // ------------------------------------------------------------ idle (register split only)
+    } else if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t qc = 0, kc = 0, vc = 0;
             bool ok = true;
-            int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
-            for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
-                const Item it = decode_item(next, p);
-                if (idx + gridDim.x < n_items) next = __ldg(items + idx + gridDim.x);  // prefetch
+            ItemWalk wk;
+            for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+                if (!wk.has()) continue;
+                const Item it = decode_item(wk.cur, p);
                 const int g = it.head / G;
                 for (int r = 0; r < it.n_sub; ++r) {
                     const uint32_t sq = qc % L::kQSlots;
@@ -200,36 +215,87 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, HD, 0, 1);
-            uint32_t qc = 0, kc = 0, vc = 0;
-            uint32_t p_cnt[2] = {0, 0};
+            uint32_t qc = 0;    // Q sub-tiles of the items before the current one
+            uint32_t g = 0;     // global index of the current key tile (the K / V ring position)
+            uint32_t p_cnt[2] = {0, 0};         // P.V products issued per sub-tile
+            bool pv_open[2] = {false, false};   // hd 128: the last P.V of r not yet seen complete
+            // the key tile g - 1 as sub-tile r used it: its S was issued, its P.V not yet
+            bool pend[2] = {false, false}, pend_first[2] = {false, false}, pend_last[2] = {false, false};
             bool ok = true;
-            int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
-            for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
-                const Item it = decode_item(next, p);
-                if (idx + gridDim.x < n_items) next = __ldg(items + idx + gridDim.x);  // prefetch
+
+            // O_r += P_r V_{g-1} for a pending sub-tile (V_{g-1} has landed)
+            auto issue_pv = [&](int r) -> bool {
+                if (!mbar_wait(&bars->p_full[r], p_cnt[r] & 1, abort_flag, dev_status)) return false;
+                tc_fence_after();
+                const uint32_t v_tile = sbase + L::kOffV + ((g - 1) % L::kVStages) * L::kKV;
+                const uint32_t a_p = tmem + (kSepP ? kTmP + 64 * r : 128 * r);
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                    umma_f16_ts(tmem + L::kTmO + HD * r, a_p + 8 * kk, desc_v(v_tile, kk), idesc_pv,
+                                (!pend_first[r] || kk > 0) ? 1u : 0u);
+                if (!kSepP) umma_commit(&bars->pv_done[r]);
+                if (pend_last[r]) umma_commit(&bars->o_ready[r]);
+                ++p_cnt[r];
+                pv_open[r] = !kSepP;
+                pend[r] = false;
+                return true;
+            };
+            auto wait_v_prev = [&]() -> bool {
+                const uint32_t n = g - 1;
+                if (!mbar_wait(&bars->v_full[n % L::kVStages], (n / L::kVStages) & 1, abort_flag,
+                               dev_status))
+                    return false;
+                return true;
+            };
+
+            ItemWalk wk;
+            for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+                if (!wk.has()) continue;
+                const Item it = decode_item(wk.cur, p);
                 uint32_t q_slot[2], q_par[2];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     q_slot[r] = (qc + r) % L::kQSlots;
                     q_par[r] = ((qc + r) / L::kQSlots) & 1;
                 }
-                for (int t = 0; t < it.n_kv && ok; ++t) {
-                    const uint32_t sk = kc % L::kKStages;
-                    if (!mbar_wait(&bars->k_full[sk], (kc / L::kKStages) & 1, abort_flag, dev_status)) {
+                for (int t = 0; t < it.n_kv && ok; ++t, ++g) {
+                    // every key tile has a user (the two sub-tiles' ranges are contiguous and
+                    // cover the item's), so V_{g-1} is awaited and released once, in order
+                    if (g > 0 && !wait_v_prev()) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
+                    // the previous item's last P.V products first: their epilogues free the Q slots
+                    // the producer may be waiting for before it loads this tile
+                    if (t == 0) {
+                        for (int r = 0; r < 2 && ok; ++r)
+                            if (pend[r]) ok = issue_pv(r);
+                        if (!ok) break;
+                    }
+                    const uint32_t sk = g % L::kKStages;
+                    if (!mbar_wait(&bars->k_full[sk], (g / L::kKStages) & 1, abort_flag, dev_status)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t k_tile = sbase + L::kOffK + sk * L::kKV;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
+                        if (pend[r] && !issue_pv(r)) {
+                            ok = false;
+                            break;
+                        }
                         if (t < it.t_first[r] || t > it.t_last[r]) continue;
-                        // Q_r must have landed (first tile of the sub-tile), and S_r reuses the
-                        // columns of P_r: the last P_r . V must have finished.
-                        if ((t == it.t_first[r] &&
-                             !mbar_wait(&bars->q_full[q_slot[r]], q_par[r], abort_flag, dev_status)) ||
-                            (p_cnt[r] > 0 && !mbar_wait(&bars->pv_done[r], (p_cnt[r] - 1) & 1,
-                                                        abort_flag, dev_status))) {
+                        // S_r overwrites the columns that P_r of hd 128 shares with it
+                        if (pv_open[r]) {
+                            if (!mbar_wait(&bars->pv_done[r], (p_cnt[r] - 1) & 1, abort_flag,
+                                           dev_status)) {
+                                ok = false;
+                                break;
+                            }
+                            pv_open[r] = false;
+                        }
+                        if (t == it.t_first[r] &&
+                            !mbar_wait(&bars->q_full[q_slot[r]], q_par[r], abort_flag, dev_status)) {
                             ok = false;
                             break;
                         }
@@ -241,39 +307,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                         idesc_qk, kk == 0 ? 0u : 1u);
                         umma_commit(&bars->s_full[r]);
                         if (t == it.t_last[r]) umma_commit(&bars->q_empty[q_slot[r]]);
+                        pend[r] = true;
+                        pend_first[r] = t == it.t_first[r];
+                        pend_last[r] = t == it.t_last[r];
                     }
                     if (!ok) break;
+                    if (g > 0) umma_commit(&bars->v_empty[(g - 1) % L::kVStages]);
                     umma_commit(&bars->k_empty[sk]);
-                    ++kc;
-                    const uint32_t sv = vc % L::kVStages;
-                    if (!mbar_wait(&bars->v_full[sv], (vc / L::kVStages) & 1, abort_flag, dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t v_tile = sbase + L::kOffV + sv * L::kKV;
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        if (t < it.t_first[r] || t > it.t_last[r]) continue;
-                        if (!mbar_wait(&bars->p_full[r], p_cnt[r] & 1, abort_flag, dev_status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < kBlockN / 16; ++kk)
-                            umma_f16_ts(tmem + L::kTmO + HD * r, tmem + 128 * r + 8 * kk,
-                                        desc_v(v_tile, kk), idesc_pv,
-                                        (t > it.t_first[r] || kk > 0) ? 1u : 0u);
-                        umma_commit(&bars->pv_done[r]);
-                        if (t == it.t_last[r]) umma_commit(&bars->o_ready[r]);
-                        ++p_cnt[r];
-                    }
-                    if (!ok) break;
-                    umma_commit(&bars->v_empty[sv]);
-                    ++vc;
                 }
                 qc += it.n_sub;
+            }
+            // the last key tile's P.V products
+            if (ok && g > 0) {
+                ok = wait_v_prev();
+                for (int r = 0; r < 2 && ok; ++r)
+                    if (pend[r]) ok = issue_pv(r);
+                if (ok) umma_commit(&bars->v_empty[(g - 1) % L::kVStages]);
             }
             // Wait (bounded) until every MMA this thread issued has finished.
             umma_commit(&bars->drain);
@@ -282,10 +331,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax, sub-tile r
+        regs_increase<kTcRegsSoftmax>();
         const int r = warp >> 2;
         const int row = threadIdx.x & 127;  // query row in the sub-tile == TMEM lane
-        const uint32_t tm_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const int r0 = (warp & 3) * 32;     // first row of this warp
+        const uint32_t tm_lane = tmem + (static_cast<uint32_t>(r0) << 16);
         const uint32_t tm_s = tm_lane + 128 * r;
+        const uint32_t tm_p = kSepP ? tm_lane + kTmP + 64 * r : tm_s;
         const uint32_t tm_o = tm_lane + L::kTmO + HD * r;
         const float scale_log2 = p.scale * kLog2e;
         const uint64_t scale2 = f32x2(scale_log2, scale_log2);
@@ -293,10 +345,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t s_cnt = 0, o_cnt = 0;
         uint32_t q_seq = 0;  // index of the current item's first Q sub-tile in this CTA's stream
         bool ok = true;
-        int4 next = blockIdx.x < n_items ? __ldg(items + blockIdx.x) : make_int4(0, 0, 0, 0);
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
-            const Item it = decode_item(next, p);
-            if (idx + gridDim.x < n_items) next = __ldg(items + idx + gridDim.x);  // prefetch
+        ItemWalk wk;
+        for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+            if (!wk.has()) continue;
+            const Item it = decode_item(wk.cur, p);
             // per-sub-tile fields by select (r is not a compile-time index here)
             const int nr = r ? it.nr[1] : it.nr[0];
             const int t_first = r ? it.t_first[1] : it.t_first[0];
@@ -321,54 +373,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ok) break;
                 ++s_cnt;
                 tc_fence_after();
+                // the whole S row, one wait
+                uint32_t v[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tm_s + 32 * c, v + 32 * c);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) regs_after_wait(v + 32 * c);
                 const int c_lo = j_min - kv0, c_hi = j_max - kv0;
                 // Masked tiles are processed in 32-column chunks classed uniformly over this
                 // warp's 32 rows [r0, r0 + 31]: the row bounds c_lo(row), c_hi(row) grow with the
                 // row, so a chunk is skipped when it lies below the first row's c_lo or above the
-                // last row's c_hi, needs no lower (upper) mask when it lies wholly at or above the
-                // last row's c_lo (at or below the first row's c_hi), and is masked on the needed
-                // side(s) otherwise. Skipped chunks cost no loads, no exponentials, and P = 0.
+                // last row's c_hi, needs no mask when it lies wholly inside [last row's c_lo,
+                // first row's c_hi], and is masked otherwise. Skipped chunks cost no exponentials
+                // and give P = 0.
                 const bool full_tile = (tile_jmin <= kv0) && (kv0 + kBlockN - 1 <= tile_jmax);
-                const int r0 = (warp & 3) * 32;
                 const int lo_first = window > 0 ? qr0 + r0 - window + 1 - kv0 : INT32_MIN / 2;
                 const int lo_last = window > 0 ? lo_first + 31 : INT32_MIN / 2;
                 const int hi_first = (p.causal ? min(qr0 + r0, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
                 const int hi_last = (p.causal ? min(qr0 + r0 + 31, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
-                auto chunk_class = [&](int c) -> int {  // 4 = skip, else mask mode bits
+                int cls[4];  // 0 = skip, 1 = no mask, 2 = masked
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
                     const int lo = 32 * c, hi = lo + 31;
-                    if (hi < lo_first || lo > hi_last) return 4;
-                    return (lo < lo_last ? kMaskLo : 0) | (hi > hi_first ? kMaskHi : 0);
-                };
-                // pass 1: row max over the visible columns
+                    cls[c] = full_tile ? 1
+                             : (hi < lo_first || lo > hi_last) ? 0
+                             : (lo >= lo_last && hi <= hi_first) ? 1 : 2;
+                }
+                // row max over the visible columns
                 float mx = -INFINITY;
-                if (full_tile) {
-                    // unmasked tile: two 64-column halves, one wait each
-#pragma unroll 1
-                    for (int hlf = 0; hlf < 2; ++hlf) {
-                        uint32_t v[64];
-                        tmem_ld32(tm_s + 64 * hlf, v);
-                        tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
-                        tmem_wait_ld();
-                        regs_after_wait(v);
-                        regs_after_wait(v + 32);
-                        mx = row_max64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, mx);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        const int cls = chunk_class(c);
-                        if (cls == 4) continue;
-                        uint32_t v[32];
-                        tmem_ld32(tm_s + 32 * c, v);
-                        tmem_wait_ld();
-                        regs_after_wait(v);
-                        switch (cls) {
-                            case kMaskNone: mx = row_max32<kMaskNone>(v, 32 * c, c_lo, c_hi, mx); break;
-                            case kMaskLo: mx = row_max32<kMaskLo>(v, 32 * c, c_lo, c_hi, mx); break;
-                            case kMaskHi: mx = row_max32<kMaskHi>(v, 32 * c, c_lo, c_hi, mx); break;
-                            default: mx = row_max32<kMaskBoth>(v, 32 * c, c_lo, c_hi, mx); break;
-                        }
-                    }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (cls[c] == 1)
+                        mx = fmaxf(mx, chunk_max<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi));
+                    else if (cls[c] == 2)
+                        mx = fmaxf(mx, chunk_max<kMaskBoth>(v + 32 * c, 32 * c, c_lo, c_hi));
                 }
                 const float m_new = fmaxf(m, mx * scale_log2);
                 // Keep the reference max until the row max grows by more than 8 (a factor 256):
@@ -378,58 +417,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (rescale) m = m_new;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const uint64_t negm2 = f32x2(neg_m, neg_m);
-                // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first half of S (packed
-                // words of 32 columns go to 16 columns, all of them already read in this pass)
-                uint64_t sum2 = f32x2(0.f, 0.f);
-                if (full_tile) {
-#pragma unroll 1
-                    for (int hlf = 0; hlf < 2; ++hlf) {
-                        uint32_t v[64];
-                        tmem_ld32(tm_s + 64 * hlf, v);
-                        tmem_ld32(tm_s + 64 * hlf + 32, v + 32);
-                        tmem_wait_ld();
-                        regs_after_wait(v);
-                        regs_after_wait(v + 32);
-                        uint32_t pk[32];
-                        sum2 = row_exp64<kMaskNone>(v, 64 * hlf, c_lo, c_hi, scale2, negm2, sum2, pk);
-                        tmem_st32(tm_s + 32 * hlf, pk);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        const int cls = chunk_class(c);
-                        uint32_t pk[16];
-                        if (cls == 4) {
+                // P = 2^(s * scale * log2e - m) as bf16 (written after the whole row was read, so
+                // it may share the columns of S)
+                uint64_t sum_a = f32x2(0.f, 0.f), sum_b = f32x2(0.f, 0.f);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                        } else {
-                            uint32_t v[32];
-                            tmem_ld32(tm_s + 32 * c, v);
-                            tmem_wait_ld();
-                            regs_after_wait(v);
-                            switch (cls) {
-                                case kMaskNone: sum2 = row_exp32<kMaskNone>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                                case kMaskLo: sum2 = row_exp32<kMaskLo>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                                case kMaskHi: sum2 = row_exp32<kMaskHi>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                                default: sum2 = row_exp32<kMaskBoth>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                            }
-                        }
-                        tmem_st16(tm_s + 16 * c, pk);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+                    if (cls[c] == 1) {
+                        chunk_exp<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
+                    } else if (cls[c] == 2) {
+                        chunk_exp<kMaskBoth>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
                     }
+                    tmem_st16(tm_p + 16 * c, pk);
                 }
+                const uint64_t sum2 = add_f32x2(sum_a, sum_b);
                 float s_lo, s_hi;
                 f32x2_split(sum2, s_lo, s_hi);
                 l = l * alpha + (s_lo + s_hi);
                 if (t > t_first && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-                    for (int c = 0; c < HD / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(tm_o + 32 * c, v);
-                        tmem_wait_ld();
-                        regs_after_wait(v);
+                    uint32_t ov[HD];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                        tmem_st32(tm_o + 32 * c, v);
+                    for (int c = 0; c < HD / 32; ++c) tmem_ld32(tm_o + 32 * c, ov + 32 * c);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        regs_after_wait(ov + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            ov[32 * c + e] = __float_as_uint(__uint_as_float(ov[32 * c + e]) * alpha);
+                        tmem_st32(tm_o + 32 * c, ov + 32 * c);
                     }
                 }
                 tmem_wait_st();
@@ -452,32 +471,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr int kChunks = HD / 8;  // 16-byte chunks per row
             uint8_t* stage = smem + L::kOffQ + (my_q % L::kQSlots) * L::kQSub + (warp & 3) * 32 * (HD * 2);
             const int wrow = row & 31;
-#pragma unroll 1
-            for (int c = 0; c < HD / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tm_o + 32 * c, v);
-                tmem_wait_ld();
-                regs_after_wait(v);
+            {
+                uint32_t ov[HD];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint4 w4 = make_uint4(
-                        pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv_l, __uint_as_float(v[8 * q4 + 1]) * inv_l),
-                        pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv_l, __uint_as_float(v[8 * q4 + 3]) * inv_l),
-                        pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv_l, __uint_as_float(v[8 * q4 + 5]) * inv_l),
-                        pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv_l, __uint_as_float(v[8 * q4 + 7]) * inv_l));
-                    const int chunk = 4 * c + q4;
-                    *reinterpret_cast<uint4*>(stage + wrow * (HD * 2) + ((chunk ^ (wrow & (kChunks - 1))) << 4)) = w4;
+                for (int c = 0; c < HD / 32; ++c) tmem_ld32(tm_o + 32 * c, ov + 32 * c);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    regs_after_wait(ov + 32 * c);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint32_t* w8 = ov + 32 * c + 8 * q4;
+                        const uint4 w4 = make_uint4(
+                            pack_bf16x2(__uint_as_float(w8[0]) * inv_l, __uint_as_float(w8[1]) * inv_l),
+                            pack_bf16x2(__uint_as_float(w8[2]) * inv_l, __uint_as_float(w8[3]) * inv_l),
+                            pack_bf16x2(__uint_as_float(w8[4]) * inv_l, __uint_as_float(w8[5]) * inv_l),
+                            pack_bf16x2(__uint_as_float(w8[6]) * inv_l, __uint_as_float(w8[7]) * inv_l));
+                        const int chunk = 4 * c + q4;
+                        *reinterpret_cast<uint4*>(stage + wrow * (HD * 2) + ((chunk ^ (wrow & (kChunks - 1))) << 4)) = w4;
+                    }
                 }
             }
             __syncwarp();
             {
-                const int row0 = qr0 + (warp & 3) * 32;  // first slot of this warp's rows
+                const int row0 = qr0 + r0;  // first slot of this warp's rows
                 constexpr int kRowsPerIter = 32 / kChunks;
 #pragma unroll 4
                 for (int j = 0; j < 32 / kRowsPerIter; ++j) {
                     const int rl = j * kRowsPerIter + lane / kChunks;
                     const int chunk = lane % kChunks;
-                    if ((warp & 3) * 32 + rl < nr) {
+                    if (r0 + rl < nr) {
                         const uint4 w4 = *reinterpret_cast<const uint4*>(
                             stage + rl * (HD * 2) + ((chunk ^ (rl & (kChunks - 1))) << 4));
                         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) +
