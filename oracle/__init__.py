@@ -27,6 +27,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
 _i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
 _c = ctypes.c_int
 _l = ctypes.c_int64
 _d = ctypes.c_double
@@ -63,6 +64,10 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [_f64p, _f64p, _f64p, _f64p, _i32p, _c, _c, _c, _c, _c, _c,
                                         _c, _d, _f64p, _f64p, _f64p]
         lib.oracle_rope_bwd.argtypes = [_f64p, _i32p, _l, _c, _c, _c, _c, _d, _c]
+        lib.oracle_decode_e4m3.argtypes = [_u8p, _f64p, _l]
+        lib.oracle_encode_e4m3.argtypes = [_f64p, _u8p, _l]
+        lib.oracle_decode_e4m3.restype = ctypes.c_int
+        lib.oracle_encode_e4m3.restype = ctypes.c_int
         lib.oracle_attn_bwd.restype = ctypes.c_int
         lib.oracle_rope_bwd.restype = ctypes.c_int
         for f in ("oracle_rms_norm", "oracle_rope", "oracle_round_bf16", "oracle_interleave", "oracle_deinterleave", "oracle_attention",
@@ -200,6 +205,34 @@ def attn_fwd(q, k, v, cu_seqlens, causal=True, window=0, paired=False, scale=Non
     _check(_load().oracle_attn_fwd(q, k, v, cu, len(cu) - 1, H, Hkv, hd, int(causal),
                                    int(window), int(paired), scale, o, lse), "attn_fwd")
     return o, lse
+
+
+def decode_e4m3(codes):
+    """float64 value of every e4m3 code (uint8 array of the same shape); see oracle.c."""
+    b = np.ascontiguousarray(codes, dtype=np.uint8)
+    y = np.empty(b.shape, dtype=np.float64)
+    _check(_load().oracle_decode_e4m3(b.reshape(-1), y.reshape(-1), b.size), "decode_e4m3")
+    return y
+
+
+def encode_e4m3(x):
+    """Nearest e4m3 code of every element (ties to even; NaN past 448), as uint8."""
+    y = _f64(x)
+    b = np.empty(y.shape, dtype=np.uint8)
+    _check(_load().oracle_encode_e4m3(y.reshape(-1), b.reshape(-1), y.size), "encode_e4m3")
+    return b
+
+
+def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, cu_seqlens, causal=True, window=0,
+                 paired=False, scale=None):
+    """Attention over FP8 inputs: q = q_scale * value(q8), k = k_scale * value(k8),
+    v = v_scale * value(v8) (e4m3 codes, per-tensor float32 scales), then attn_fwd on those
+    exact float64 values. Returns (o, lse) like attn_fwd; the softmax scale defaults to
+    1/sqrt(head_dim)."""
+    q = decode_e4m3(q8) * float(np.float32(q_scale))
+    k = decode_e4m3(k8) * float(np.float32(k_scale))
+    v = decode_e4m3(v8) * float(np.float32(v_scale))
+    return attn_fwd(q, k, v, cu_seqlens, causal, window, paired, scale)
 
 
 def attn_rows(q, k, v, cu_seqlens, rows, causal=True, window=0, paired=False, scale=None):

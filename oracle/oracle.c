@@ -131,6 +131,61 @@ int oracle_round_bf16(double* x, int64_t n)
     return ORACLE_OK;
 }
 
+/* ---- e4m3 ("float8_e4m3fn"): the 8-bit floating point format of the packed FP8 Q/K/V path
+ * ([PHA] "5. interactions with other mechanisms": on paired layers the FP8 QKV projection is
+ * issued as separate column-slice GEMMs, so attention may receive Q, K, V in FP8).
+ * Format (the OCP FP8 E4M3 definition, the one torch.float8_e4m3fn implements): 1 sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits. Exponent field 0 holds the subnormals
+ * m/8 * 2^-6 = m * 2^-9; exponent field E in 1..15 holds (1 + m/8) * 2^(E-7); the two codes with
+ * all exponent and mantissa bits set are NaN; there is no infinity, and the largest finite value
+ * is 1.75 * 2^8 = 448. A tensor of codes b with per-tensor float32 scale s stands for s * value(b). */
+static double decode_e4m3(uint8_t b)
+{
+    const int sign = b >> 7, E = (b >> 3) & 15, m = b & 7;
+    if (E == 15 && m == 7) return NAN;
+    const double v = E == 0 ? ldexp((double)m, -9) : ldexp(8.0 + (double)m, E - 10);
+    return sign ? -v : v;
+}
+
+int oracle_decode_e4m3(const uint8_t* b, double* y, int64_t n)
+{
+    if ((!b || !y) && n > 0) return ORACLE_EINVAL;
+    for (int64_t i = 0; i < n; ++i) y[i] = decode_e4m3(b[i]);
+    return ORACLE_OK;
+}
+
+/* Nearest e4m3 code of x, ties to even (the mantissa code with its low bit clear). A magnitude
+ * that rounds past 448 (above the midpoint 464 between 448 and the next step, 480), an infinity
+ * or a NaN gives NaN: the format cannot hold it (torch's float8_e4m3fn cast behaves the same). */
+static uint8_t encode_e4m3(double x)
+{
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    if (isinf(a)) return sign | 0x7F;
+    if (a < ldexp(1.0, -6)) {                       /* subnormal grid, step 2^-9 */
+        const double q = nearbyint(a * 512.0);      /* 0 .. 8; 8 is the smallest normal 2^-6 */
+        return sign | (uint8_t)q;
+    }
+    int e;
+    frexp(a, &e);                                   /* a in [2^(e-1), 2^e) */
+    int E = e - 1;
+    double q = nearbyint(ldexp(a, 3 - E));          /* 8 .. 16 significand steps of 2^(E-3) */
+    if (q == 16.0) {
+        E += 1;
+        q = 8.0;
+    }
+    if (E > 8 || (E == 8 && q > 14.0)) return sign | 0x7F; /* past 448 */
+    return sign | (uint8_t)(((E + 7) << 3) | ((int)q - 8));
+}
+
+int oracle_encode_e4m3(const double* x, uint8_t* b, int64_t n)
+{
+    if ((!b || !x) && n > 0) return ORACLE_EINVAL;
+    for (int64_t i = 0; i < n; ++i) b[i] = encode_e4m3(x[i]);
+    return ORACLE_OK;
+}
+
 /* Explicit paired interleave ([PHA] "core idea", "4. interleave index"): token t, head h of
  * x[T][H][d] moves to slot 2t + h/(H/2), head h % (H/2) of y[2T][H/2][d]. A copy loop, not a view. */
 int oracle_interleave(const double* x, double* y, int64_t T, int H, int d)

@@ -623,3 +623,75 @@ def test_rope_backward_is_adjoint_and_inverse(paired, stagger):
     bty = oracle.rope_bwd(y, pos, paired, stagger)
     assert abs(float((rx * y).sum() - (x * bty).sum())) < 1e-11   # <R x, y> = <x, R^T y>
     np.testing.assert_allclose(oracle.rope_bwd(rx, pos, paired, stagger), x, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------- e4m3 (FP8)
+# The FP8 path consumes e4m3 codes with per-tensor float32 scales ("modded-nanogpt Paired Head
+# Attention record", section "5. interactions with other mechanisms": the packed FP8 QKV
+# projection). The oracle's decode and encode are pinned to torch's float8_e4m3fn (an independent
+# implementation of the same OCP format), to closed-form codes, and to invariants of the scales.
+
+def test_decode_e4m3_all_codes_match_torch():
+    import torch
+
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.decode_e4m3(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+
+
+def test_decode_e4m3_closed_forms():
+    cases = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+             0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    got = oracle.decode_e4m3(np.array(list(cases), dtype=np.uint8))
+    np.testing.assert_array_equal(got, np.array(list(cases.values())))
+    assert np.isnan(oracle.decode_e4m3(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def test_encode_e4m3_matches_torch_on_float32_values():
+    import torch
+
+    rng = np.random.default_rng(5)
+    x = np.concatenate([
+        rng.standard_normal(50000) * 100.0,                 # normals, some past 448
+        rng.standard_normal(20000) * 2.0 ** -8,             # subnormal range
+        rng.uniform(440.0, 500.0, 5000),                    # around the largest finite value
+    ]).astype(np.float32)
+    # exact ties: midpoints between neighbouring finite codes (both even and odd lower codes)
+    vals = oracle.decode_e4m3(np.arange(0, 126, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, np.float32([464.0, -464.0, 0.0, -0.0])])
+    got = oracle.encode_e4m3(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+
+
+def test_encode_e4m3_round_trips_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert np.array_equal(oracle.encode_e4m3(oracle.decode_e4m3(codes)), codes)
+
+
+def test_attn_fwd_fp8_scales_enter_as_the_definition_says():
+    rng = np.random.default_rng(9)
+    T, H, hd = 40, 2, 16
+    q8, k8, v8 = (oracle.encode_e4m3(rng.standard_normal((T, H, hd)) * 3.0) for _ in range(3))
+    cu = np.array([0, 17, 40], dtype=np.int32)
+    o1, l1 = oracle.attn_fwd_fp8(q8, k8, v8, 1.0, 1.0, 1.0, cu, True, 5, False, 0.25)
+    # v's scale multiplies O and leaves the LSE alone
+    o2, l2 = oracle.attn_fwd_fp8(q8, k8, v8, 1.0, 1.0, 2.5, cu, True, 5, False, 0.25)
+    np.testing.assert_allclose(o2, 2.5 * o1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-13)
+    # q's and k's scales multiply the logits: the same as folding them into the softmax scale
+    o3, l3 = oracle.attn_fwd_fp8(q8, k8, v8, 0.5, 3.0, 1.0, cu, True, 5, False, 0.25)
+    o4, l4 = oracle.attn_fwd(oracle.decode_e4m3(q8), oracle.decode_e4m3(k8),
+                             oracle.decode_e4m3(v8), cu, True, 5, False, 0.25 * 1.5)
+    np.testing.assert_allclose(o3, o4, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(l3, l4, rtol=1e-12, atol=1e-12)
+    # and with unit scales the values are the decoded codes themselves
+    o5, l5 = oracle.attn_fwd(oracle.decode_e4m3(q8), oracle.decode_e4m3(k8),
+                             oracle.decode_e4m3(v8), cu, True, 5, False, 0.25)
+    np.testing.assert_array_equal(o1, o5)
+    np.testing.assert_array_equal(l1, l5)
