@@ -269,7 +269,7 @@ def main():
     aux = None
     if args.aux_v:
         if not step.aux_v_supported:
-            raise SystemExit("--aux-v needs the band kernel (bf16, causal, window <= 128)")
+            raise SystemExit("--aux-v needs the bf16 tensor-core path (head_dim 64 or 128)")
         g = torch.Generator().manual_seed(7 + 1000 * rank)
         aux = torch.randn(tuple(v.shape), generator=g).to(v.dtype).to(dev)
 
@@ -480,6 +480,7 @@ def main():
         line["backward"] = bwd
     if not args.no_suite and args.workload == "paired_varlen" and not (args.qk_norm or args.aux_v):
         line["configs"] = time_suite(max(3, min(args.steps, 20)), args.warmup, dev, peaks, rank)
+        line["fp8"] = time_fp8(max(3, min(args.steps, 20)), args.warmup, dev, peaks, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, s, thr = time_oracle(w, args.oracle_tokens, args.qk_norm)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
@@ -569,6 +570,67 @@ def time_suite(steps: int, warmup: int, dev, peaks, rank: int = 0):
             "steps": steps, "sm_mhz": clk.get("sm_mhz"), "clock_reasons": clk.get("reasons"),
         }
         del q, k, v, cu, pos, step, inp
+        torch.cuda.empty_cache()
+    return out
+
+
+FP8_SUITE = (("paired_varlen", "paired_varlen", {}),
+             ("mixed_window_full", "mixed_window", {"window": 0}),
+             ("gqa_long", "gqa_long", {}))
+
+
+def time_fp8(steps: int, warmup: int, dev, peaks, rank: int = 0):
+    """pha_attn_fwd_fp8 on e4m3 copies of the workloads' q, k, v (per-tensor scales), timed per
+    call with CUDA events. S = Q K^T runs in kind::f8f6f4 (twice the bf16 rate, nominally), P V in
+    kind::f16, so the applicable tensor peak is 4/3 of the bf16 one (half the FLOPs at each rate)."""
+    import torch
+
+    from paired_heads_b200 import pha
+
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {}
+    for label, name, kw in FP8_SUITE:
+        w = synth.workload(name, **kw)
+        inp = synth.make_fp8_inputs(w, rank=rank)
+        q8, k8, v8 = (inp[n].to(dev) for n in ("q8", "k8", "v8"))
+        cu = inp["cu_seqlens"].to(dev)
+        o = torch.empty(w.total, w.n_heads, w.head_dim, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(w.total, w.n_heads, device=dev)
+        ws = torch.empty(pha.pha_attn_workspace_bytes(w.batch, w.max_len, w.n_heads, w.head_dim,
+                                                      w.paired), dtype=torch.uint8, device=dev)
+        sc = (inp["q_scale"], inp["k_scale"], inp["v_scale"])
+
+        def call():
+            pha.pha_attn_fwd_fp8(q8, k8, v8, *sc, cu, w.max_len, o, lse, ws, causal=w.causal,
+                                 window=w.window, paired=w.paired, scale=w.scale)
+
+        for _ in range(max(warmup, 3)):
+            call()
+        torch.cuda.synchronize(dev)
+        fbytes = float(w.total * w.head_dim * (w.n_heads + 2 * w.n_kv_heads)
+                       + 2 * w.total * w.n_heads * w.head_dim + 4 * w.total * w.n_heads)
+        in_l2 = fbytes < L2_BYTES
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for s_ in range(steps):
+            if in_l2:
+                flush.fill_(s_ & 0xFF)
+            ev[s_][0].record(stream)
+            call()
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize(dev)
+        status, _ = pha.pha_attn_status(ws)
+        if status != 0:
+            raise SystemExit(f"fp8 {label}: device status {status}")
+        ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        flops = attn_flops(w)
+        tf = flops / (ms * 1e-3) / 1e12
+        out[label] = {"attn_ms": ms, "attn_tflops": tf,
+                      "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                      "frac_of_mixed_peak": tf / (peaks["bf16_tflops"] * 4.0 / 3.0),
+                      "bytes": fbytes, "gbs": fbytes / (ms * 1e-3) / 1e9,
+                      "frac_of_hbm": fbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "steps": steps}
+        del q8, k8, v8, o, lse, ws, inp
         torch.cuda.empty_cache()
     return out
 

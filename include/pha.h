@@ -163,9 +163,9 @@ pha_status pha_attn_fwd(const void* q, const void* k, const void* v, const int32
  *   shape, dtype and layout ([total_tokens][n_kv_heads][head_dim], 16-byte aligned); neither v nor
  *   aux_v is modified (the sum is formed tile by tile in shared memory).
  *   Other arguments, results and errors: as pha_attn_fwd.
- *   Supported: bf16, causal, 1 <= window <= 128 (the band kernel), head_dim in {64, 128};
- *      anything else returns PHA_ERR_UNSUPPORTED before any launch. aux_v NULL with
- *      total_tokens > 0: PHA_ERR_INVALID.
+ *   Supported: bf16 with head_dim in {64, 128}, every window and causal setting (the band kernel
+ *      for causal windows <= 128, the block kernel otherwise); f32 returns PHA_ERR_UNSUPPORTED
+ *      before any launch. aux_v NULL with total_tokens > 0: PHA_ERR_INVALID.
  */
 pha_status pha_attn_fwd_aux_v(const void* q, const void* k, const void* v, const void* aux_v,
                               const int32_t* cu_seqlens, int batch, int max_len,
@@ -173,6 +173,36 @@ pha_status pha_attn_fwd_aux_v(const void* q, const void* k, const void* v, const
                               pha_dtype dtype, int causal, int window, int paired, float scale,
                               void* o, float* lse, void* workspace, size_t workspace_bytes,
                               pha_stream_t stream);
+
+/*
+ * pha_attn_fwd_fp8 -- pha_attn_fwd over FP8 (e4m3) q, k, v with per-tensor scales.
+ *   The packed FP8 QKV projection of the record page produces Q, K and V in 8-bit floating point
+ *   ("modded-nanogpt Paired Head Attention record", section "5. interactions with other
+ *   mechanisms"); this entry point consumes them without widening them in HBM.
+ *   q8: [total_tokens][n_heads][head_dim], k8, v8: [total_tokens][n_kv_heads][head_dim], one byte
+ *      per element in the OCP FP8 E4M3 format (torch.float8_e4m3fn: bias 7, no infinities, NaN
+ *      codes 0x7F / 0xFF, largest finite 448); 16-byte aligned; read only. The paired slot view,
+ *      cu_seqlens, masks, GQA mapping and errors are those of pha_attn_fwd.
+ *   q_scale, k_scale, v_scale: positive finite float32; the tensors stand for
+ *      q = q_scale * value(q8), k = k_scale * value(k8), v = v_scale * value(v8).
+ *   Result: O and LSE of attention over those q, k, v, exactly as pha_attn_fwd defines them
+ *      (scale <= 0 selects 1/sqrt(head_dim)); o is bf16 ([total_tokens][n_heads][head_dim]),
+ *      lse float32 [total_tokens][n_heads] (may be NULL).
+ *   Arithmetic: S = Q K^T on the tensor cores in kind::f8f6f4 (products of e4m3 values are exact
+ *      in the float32 accumulator), scaled by scale * q_scale * k_scale; P rounded to f16; V
+ *      widened exactly to f16 in shared memory; O += P V in kind::f16 with float32 accumulation;
+ *      O multiplied by v_scale / l; bf16 output.
+ *   Supported: head_dim 64 or 128, any causal window or none, causal or not (block kernel).
+ *   workspace: as pha_attn_fwd (pha_attn_workspace_bytes with the same arguments).
+ *   Errors: as pha_attn_fwd; PHA_ERR_INVALID also for a scale that is not positive and finite;
+ *      PHA_ERR_UNSUPPORTED for head_dim other than 64 / 128.
+ */
+pha_status pha_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale,
+                            float k_scale, float v_scale, const int32_t* cu_seqlens, int batch,
+                            int max_len, int total_tokens, int n_heads, int n_kv_heads,
+                            int head_dim, int causal, int window, int paired, float scale, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes,
+                            pha_stream_t stream);
 
 /*
  * pha_rope_bwd -- backward of pha_rope: the gradients with respect to the unrotated q and k, from
@@ -237,6 +267,25 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void*
  * PHA_ERR_CUDA if the copy fails.
  */
 pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream);
+
+/*
+ * pha_test_attn_fwd_stalled -- failure-detection test hook; not for production use.
+ *   Runs pha_attn_fwd (same arguments, same checks) with one change in the band kernel: its
+ *   softmax warps first wait up to stall_us microseconds on a barrier that nothing signals. The
+ *   wait runs out, the kernel records device status 3 (read it with pha_attn_status), every role
+ *   of each CTA winds down (the producer waits for its copies in flight, the MMA thread for its
+ *   MMAs, tensor memory is freed) and no output row is written. The GPU context stays usable: a
+ *   later call on the same workspace and stream runs normally. This is how a kernel wait that
+ *   gives up is exercised without faulting or hanging a GPU.
+ *   stall_us: 1 .. 100000, else PHA_ERR_INVALID. Only the band kernel has the hook (bf16, causal,
+ *   1 <= window <= 128); other shapes return PHA_ERR_UNSUPPORTED.
+ */
+pha_status pha_test_attn_fwd_stalled(const void* q, const void* k, const void* v,
+                                     const int32_t* cu_seqlens, int batch, int max_len,
+                                     int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                                     pha_dtype dtype, int causal, int window, int paired,
+                                     float scale, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, int stall_us, pha_stream_t stream);
 
 /*
  * pha_attn_fwd_noalloc -- pha_attn_fwd without a caller-provided workspace.

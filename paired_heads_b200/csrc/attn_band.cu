@@ -42,48 +42,10 @@ struct BandBars {
     uint64_t v_add[4];  // value embedding: the landed V tile has had aux_v added
     uint64_t s_full[2], p_full[2], pv_done[2], o_ready[2];
     uint64_t drain[2];
+    uint64_t stall;  // never signalled: the failure-detection test hook waits on it
     uint32_t tmem_base;
     int abort;
 };
-
-// Adder warpgroup (value embedding): adds rows [row0, row0 + 128) of aux_v (head hs of the slot
-// view, heads_slot heads per slot row, the same layout as v) to the landed V tile in shared memory,
-// rounding each sum to bf16 as a bf16 tensor addition does. Rows past the tensor are left as they
-// are. Thread t of the 128 takes 16-byte unit t % (hd / 8) of every (1024 / hd)-th row; all of its
-// global loads are issued before the first add.
-template <int HD>
-__device__ __forceinline__ void add_aux_tile(uint8_t* tile, const __nv_bfloat16* aux, int row0, int hs,
-                                             int heads_slot, int64_t slots, int at) {
-    constexpr int kUnits = HD / 8;
-    constexpr int kRowsPerPass = 128 / kUnits;
-    constexpr int kPasses = kBlockN / kRowsPerPass;
-    const int unit = at % kUnits;
-    uint4 a[kPasses];
-#pragma unroll
-    for (int k = 0; k < kPasses; ++k) {
-        const int r = at / kUnits + k * kRowsPerPass;
-        const int64_t slot = static_cast<int64_t>(row0) + r;
-        a[k] = slot < slots ? __ldg(reinterpret_cast<const uint4*>(
-                                  aux + (slot * heads_slot + hs) * HD + unit * 8))
-                            : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int k = 0; k < kPasses; ++k) {
-        const int r = at / kUnits + k * kRowsPerPass;
-        if (static_cast<int64_t>(row0) + r >= slots) break;
-        // unit u of row r in the 128-byte-swizzled [128 rows][64 bf16] chunks of the tile
-        uint4* addr = reinterpret_cast<uint4*>(tile + (unit >> 3) * (kBlockN * 128) + r * 128 +
-                                               (((unit & 7) ^ (r & 7)) << 4));
-        const uint4 v = *addr;
-        const uint32_t vw[4] = {v.x, v.y, v.z, v.w}, aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)  // bf16 + bf16 is exact in float32; one rounding to bf16
-            o[e] = pack_bf16x2(__uint_as_float(vw[e] << 16) + __uint_as_float(aw[e] << 16),
-                               __uint_as_float(vw[e] & 0xFFFF0000u) + __uint_as_float(aw[e] & 0xFFFF0000u));
-        *addr = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-}
 
 template <int HD, bool AUXV>
 __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
@@ -128,6 +90,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
             mbar_init(&bars->o_ready[w], 1);
             mbar_init(&bars->drain[w], 1);
         }
+        mbar_init(&bars->stall, 1);
         bars->abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
@@ -234,8 +197,9 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[sv], (vc / S) & 1, abort_flag,
                                                        dev_status));
                 if (!ok) break;
-                add_aux_tile<HD>(smem + L::kOffV + sv * L::kKV, aux, kv_first + s * kBlockN, gk,
-                                 p.kv_heads, slots, at);
+                add_aux_tile<HD, 128, 128 / (1024 / HD)>(smem + L::kOffV + sv * L::kKV, aux,
+                                                          kv_first + s * kBlockN, gk, p.kv_heads,
+                                                          slots, at);
                 fence_proxy_async_smem();  // the tensor cores read the tile next
                 mbar_arrive(&bars->v_add[sv]);
                 ++vc;
@@ -345,6 +309,9 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
         const int window = p.window;
         uint32_t s_cnt = 0, o_cnt = 0, qn = 0;
         bool ok = true;
+        if (p.test_stall_us > 0)  // the wait runs out: status 3, and every role winds down
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->stall, 0, abort_flag, dev_status,
+                                                   1000ull * static_cast<uint64_t>(p.test_stall_us)));
         ItemWalk wk;
         for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
             if (!wk.has()) continue;

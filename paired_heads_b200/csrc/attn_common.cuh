@@ -36,6 +36,8 @@ struct TcBars {
     uint64_t q_full[3], q_empty[3];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2], pv_done[2], o_ready[2];
+    uint64_t v8_full[2], v8_empty[2];  // FP8: the e4m3 V staging ring
+    uint64_t v_add[4];                 // value embedding: aux_v added to the landed V tile
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -158,9 +160,9 @@ __device__ __forceinline__ float chunk_max(const uint32_t* v, int base, int c_lo
     return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// p = 2^(s * scale_log2 - m) for 32 columns (0 where masked), packed into 16 bf16 pairs; the
-// values are added into two packed partial sums.
-template <int MODE>
+// p = 2^(s * scale_log2 - m) for 32 columns (0 where masked), packed into 16 bf16 pairs (f16
+// pairs when F16P); the values are added into two packed partial sums.
+template <int MODE, bool F16P = false>
 __device__ __forceinline__ void chunk_exp(const uint32_t* v, int base, int c_lo, int c_hi,
                                           uint64_t scale2, uint64_t negm2, uint64_t& sum_a,
                                           uint64_t& sum_b, uint32_t* pk) {
@@ -176,8 +178,51 @@ __device__ __forceinline__ void chunk_exp(const uint32_t* v, int base, int c_lo,
         const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
         sum_a = add_f32x2(sum_a, f32x2(p0, p1));
         sum_b = add_f32x2(sum_b, f32x2(p2, p3));
-        pk[e >> 1] = pack_bf16x2(p0, p1);
-        pk[(e >> 1) + 1] = pack_bf16x2(p2, p3);
+        pk[e >> 1] = F16P ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+        pk[(e >> 1) + 1] = F16P ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
+    }
+}
+
+// Adder threads (value embedding): add rows [row0, row0 + 128) of aux_v (head hs of the slot
+// view, heads_slot heads per slot row, the same layout as v) to the landed bf16 V tile in shared
+// memory, rounding each sum to bf16 as a bf16 tensor addition does. Rows past the tensor are left
+// as they are. Thread t of the NT takes 16-byte unit t % (hd / 8) of every (8 NT / hd)-th row;
+// its global loads are issued BATCH rows at a time, all before the adds of those rows.
+template <int HD, int NT, int BATCH>
+__device__ __forceinline__ void add_aux_tile(uint8_t* tile, const __nv_bfloat16* aux, int row0, int hs,
+                                             int heads_slot, int64_t slots, int at) {
+    constexpr int kUnits = HD / 8;
+    constexpr int kRowsPerPass = NT / kUnits;
+    constexpr int kPasses = kBlockN / kRowsPerPass;
+    static_assert(kPasses % BATCH == 0, "batches of passes");
+    const int unit = at % kUnits;
+#pragma unroll 1
+    for (int k0 = 0; k0 < kPasses; k0 += BATCH) {
+        uint4 a[BATCH];
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int r = at / kUnits + (k0 + k) * kRowsPerPass;
+            const int64_t slot = static_cast<int64_t>(row0) + r;
+            a[k] = slot < slots ? __ldg(reinterpret_cast<const uint4*>(
+                                      aux + (slot * heads_slot + hs) * HD + unit * 8))
+                                : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int r = at / kUnits + (k0 + k) * kRowsPerPass;
+            if (static_cast<int64_t>(row0) + r >= slots) break;
+            // unit u of row r in the 128-byte-swizzled [128 rows][64 bf16] chunks of the tile
+            uint4* addr = reinterpret_cast<uint4*>(tile + (unit >> 3) * (kBlockN * 128) + r * 128 +
+                                                   (((unit & 7) ^ (r & 7)) << 4));
+            const uint4 v = *addr;
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w}, aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)  // bf16 + bf16 is exact in float32; one rounding to bf16
+                o[e] = pack_bf16x2(__uint_as_float(vw[e] << 16) + __uint_as_float(aw[e] << 16),
+                                   __uint_as_float(vw[e] & 0xFFFF0000u) + __uint_as_float(aw[e] & 0xFFFF0000u));
+            *addr = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
 }
 

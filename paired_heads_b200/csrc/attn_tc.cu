@@ -22,10 +22,16 @@
 //               normalised and O and the LSE are stored.
 //   warp 8      TMA producer: Q sub-tiles into a ring of 3 slots (so the next item's Q arrives
 //               while the current item computes), K and V tiles into their rings (64-column x
-//               128-row boxes, 128-byte swizzle).
-//   warp 9      MMA issuer (one thread) and TMEM owner (512 columns); warps 10 and 11 idle:
-//               S_r = Q_r K^T   tcgen05.mma kind::f16, A and B from shared memory, M=128 N=128
-//               O_r += P_r V    tcgen05.mma kind::f16, A (P) from TMEM, B (V) from shared memory
+//               128-row boxes, 128-byte swizzle; FP8: one hd-byte x 128-row box per tile, V into
+//               an unswizzled staging ring).
+//   warp 9      MMA issuer (one thread) and TMEM owner (512 columns)
+//   warps 10-11 FP8: widen each landed e4m3 V tile to f16; value embedding: add aux_v's rows to
+//               each landed V tile (rounded to bf16 as a bf16 tensor addition); otherwise idle
+//   S and P.V, per sub-tile:
+//               S_r = Q_r K^T   tcgen05.mma kind::f16 (FP8: kind::f8f6f4 on e4m3 tiles), A and B
+//                               from shared memory, M=128 N=128
+//               O_r += P_r V    tcgen05.mma kind::f16 (bf16; FP8: f16 P and V), A (P) from TMEM,
+//                               B (V) from shared memory
 //               The issue order is software-pipelined per sub-tile: once P_r of key tile g-1 is
 //               ready, O_r += P_r V_{g-1} is issued and then at once S_r of key tile g, so sub-tile
 //               r's next softmax starts while the other sub-tile's softmax is still running and
@@ -86,12 +92,75 @@ __device__ __forceinline__ Item decode_item(int4 w, const AttnProblem& p) {
     return it;
 }
 
+// Shared memory of the block kernel. bf16: Q slots, K and V rings of [hd / 64][128 rows][128 B]
+// chunks. FP8: Q and K tiles hold e4m3 ([128 rows][hd B], one swizzled box), V arrives as e4m3
+// in a staging ring ([128 rows][hd B], unswizzled) and is widened to f16 into the V ring, which
+// has the bf16 layout.
+template <int HD, bool F8>
+struct BlockLayout {
+    static constexpr int kChunk = 128 * 128;  // one [128 rows][64 x 16-bit] swizzled chunk
+    static constexpr int kQSub = kBlockM * HD * (F8 ? 1 : 2);
+    static constexpr int kK = kBlockN * HD * (F8 ? 1 : 2);
+    static constexpr int kV = kBlockN * HD * 2;
+    static constexpr int kV8 = F8 ? kBlockN * HD : 0;
+    static constexpr int kQSlots = 3;
+    static constexpr int kKStages = (F8 || HD == 64) ? 4 : 2;
+    static constexpr int kVStages = (!F8 && HD == 64) ? 4 : 2;
+    static constexpr int kV8Stages = F8 ? 2 : 1;  // (kV8 = 0 without FP8: no space)
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQSlots * kQSub;
+    static constexpr int kOffV = kOffK + kKStages * kK;
+    static constexpr int kOffV8 = kOffV + kVStages * kV;
+    static constexpr int kOffBar = kOffV8 + kV8Stages * kV8;
+    static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + slack to align to 1024
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kTmO = 256;
+    // rows of a warp staged at a time in the epilogue (O as bf16 through the Q slot)
+    static constexpr int kStageRows = kQSub / (4 * HD * 2) < 32 ? kQSub / (4 * HD * 2) : 32;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(sizeof(TcBars) <= 512, "barrier block");
+    static_assert(kStageRows == 16 || kStageRows == 32, "epilogue staging");
+};
+
+// Converter warps (FP8): e4m3 V tile [128 rows][HD B] -> f16 in the V ring's layout; thread t of
+// 64 takes 16-byte units t, t + 64, ... (16 values of one row each).
 template <int HD>
+__device__ __forceinline__ void widen_v_tile(const uint8_t* v8, uint8_t* vh, int t) {
+    constexpr int kUnitsPerRow = HD / 16;
+    constexpr int kUnits = kBlockN * kUnitsPerRow;
+#pragma unroll 4
+    for (int u = t; u < kUnits; u += 64) {
+        const int r = u / kUnitsPerRow, j = u % kUnitsPerRow;
+        const uint4 w = *reinterpret_cast<const uint4*>(v8 + r * HD + 16 * j);
+        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            h[2 * e] = e4m3x2_to_f16x2(static_cast<uint16_t>(in[e] & 0xFFFFu));
+            h[2 * e + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(in[e] >> 16));
+        }
+        // values 16j .. 16j + 15 = 16-byte units 2(j % 4), 2(j % 4) + 1 of chunk j / 4 of row r
+        uint8_t* row = vh + (j >> 2) * (kBlockN * 128) + r * 128;
+        const int u0 = 2 * (j & 3);
+        *reinterpret_cast<uint4*>(row + ((u0 ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(row + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+}
+
+// K-major descriptor of an e4m3 Q / K tile, k-step kk of 32 values (32 bytes).
+template <int HD>
+__device__ __forceinline__ uint64_t desc_kmajor_e4m3(uint32_t tile, int kk) {
+    return HD == 128 ? smem_desc_sw128(tile + kk * 32, 16, 1024)
+                     : smem_desc_sw64(tile + kk * 32, 16, 512);
+}
+
+template <int HD, bool F8, bool AUXV>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnProblem p,
                    const int4* __restrict__ items, WorkspaceHeader* hdr) {
-    using L = TcLayout<HD>;
+    using L = BlockLayout<HD, F8>;
+    static_assert(!(F8 && AUXV), "the value embedding is a bf16 path");
     // P_r apart from S_r where TMEM has room for it (hd 64), else in the first 64 columns of S_r.
     constexpr bool kSepP = HD == 64;
     constexpr uint32_t kTmP = kSepP ? L::kTmO + 2 * HD : 0;
@@ -117,14 +186,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
-            mbar_init(&bars->v_full[s], 1);
+            // FP8: filled by the 64 converter threads; bf16: by the producer's TMA
+            mbar_init(&bars->v_full[s], F8 ? 64 : 1);
             mbar_init(&bars->v_empty[s], 1);
+            mbar_init(&bars->v_add[s], 64);
         }
         for (int r = 0; r < 2; ++r) {
             mbar_init(&bars->s_full[r], 1);
             mbar_init(&bars->p_full[r], 128);
             mbar_init(&bars->pv_done[r], 1);
             mbar_init(&bars->o_ready[r], 1);
+            mbar_init(&bars->v8_full[r], 1);
+            mbar_init(&bars->v8_empty[r], 64);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -149,7 +222,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp >= 8) regs_decrease<kTcRegsOther>();  // the whole third warpgroup, then its roles
     if (warp >= 10) {
-        // ------------------------------------------------------------ idle (register split only)
+        // ------------------------------------------------- FP8: V converter; aux_v: adder; else idle
+        if (AUXV) {
+            // V tiles in the producer's order: once one has landed, aux_v's matching rows are
+            // added in place and the tile is published to the MMA issuer (v_add)
+            const int at = threadIdx.x - 320;  // 0 .. 63
+            const int64_t slots = static_cast<int64_t>(p.total_tokens) * p.slot_mult;
+            const __nv_bfloat16* aux = static_cast<const __nv_bfloat16*>(p.v_aux);
+            uint32_t vc = 0;
+            bool ok = true;
+            ItemWalk wk;
+            for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+                if (!wk.has()) continue;
+                const Item it = decode_item(wk.cur, p);
+                for (int t = 0; ok && t < it.n_kv; ++t, ++vc) {
+                    const uint32_t sv = vc % L::kVStages;
+                    ok = mbar_wait(&bars->v_full[sv], (vc / L::kVStages) & 1, abort_flag, dev_status);
+                    if (!ok) break;
+                    add_aux_tile<HD, 64, 8>(smem + L::kOffV + sv * L::kV, aux, it.kv_lo + t * kBlockN,
+                                            it.head / G, p.kv_heads, slots, at);
+                    fence_proxy_async_smem();  // the tensor cores read the tile next
+                    mbar_arrive(&bars->v_add[sv]);
+                }
+            }
+        }
+        if (F8) {
+            const int ct = threadIdx.x - 320;  // 0 .. 63
+            uint32_t vc = 0;
+            bool ok = true;
+            ItemWalk wk;
+            for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+                if (!wk.has()) continue;
+                const Item it = decode_item(wk.cur, p);
+                for (int t = 0; ok && t < it.n_kv; ++t, ++vc) {
+                    const uint32_t s8 = vc % L::kV8Stages, sv = vc % L::kVStages;
+                    ok = mbar_wait(&bars->v8_full[s8], (vc / L::kV8Stages) & 1, abort_flag, dev_status) &&
+                         mbar_wait(&bars->v_empty[sv], ((vc / L::kVStages) & 1) ^ 1, abort_flag, dev_status);
+                    if (!ok) break;
+                    widen_v_tile<HD>(smem + L::kOffV8 + s8 * L::kV8, smem + L::kOffV + sv * L::kV, ct);
+                    fence_proxy_async_smem();  // the tensor cores read the f16 tile next
+                    mbar_arrive(&bars->v_full[sv]);
+                    mbar_arrive(&bars->v8_empty[s8]);
+                }
+            }
+        }
     } else if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -168,9 +284,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&bars->q_full[sq], L::kQSub);
-                    for (int c = 0; c < HD / 64; ++c)
-                        tma_load_2d(smem + L::kOffQ + sq * L::kQSub + c * L::kChunk, &tm_q,
-                                    it.head * HD + 64 * c, it.q0 + kBlockM * r, &bars->q_full[sq]);
+                    if (F8)
+                        tma_load_2d(smem + L::kOffQ + sq * L::kQSub, &tm_q, it.head * HD,
+                                    it.q0 + kBlockM * r, &bars->q_full[sq]);
+                    else
+                        for (int c = 0; c < HD / 64; ++c)
+                            tma_load_2d(smem + L::kOffQ + sq * L::kQSub + c * L::kChunk, &tm_q,
+                                        it.head * HD + 64 * c, it.q0 + kBlockM * r, &bars->q_full[sq]);
                     ++qc;
                 }
                 for (int t = 0; ok && t < it.n_kv; ++t) {
@@ -181,21 +301,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars->k_full[sk], L::kKV);
-                    for (int c = 0; c < HD / 64; ++c)
-                        tma_load_2d(smem + L::kOffK + sk * L::kKV + c * L::kChunk, &tm_k,
-                                    g * HD + 64 * c, row, &bars->k_full[sk]);
+                    mbar_arrive_expect_tx(&bars->k_full[sk], L::kK);
+                    if (F8)
+                        tma_load_2d(smem + L::kOffK + sk * L::kK, &tm_k, g * HD, row, &bars->k_full[sk]);
+                    else
+                        for (int c = 0; c < HD / 64; ++c)
+                            tma_load_2d(smem + L::kOffK + sk * L::kK + c * L::kChunk, &tm_k,
+                                        g * HD + 64 * c, row, &bars->k_full[sk]);
                     ++kc;
-                    const uint32_t sv = vc % L::kVStages;
-                    if (!mbar_wait(&bars->v_empty[sv], ((vc / L::kVStages) & 1) ^ 1, abort_flag,
-                                   dev_status)) {
-                        ok = false;
-                        break;
+                    if (F8) {
+                        // e4m3 V into the staging ring; the converter widens it into the V ring
+                        const uint32_t s8 = vc % L::kV8Stages;
+                        if (!mbar_wait(&bars->v8_empty[s8], ((vc / L::kV8Stages) & 1) ^ 1, abort_flag,
+                                       dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bars->v8_full[s8], L::kV8);
+                        tma_load_2d(smem + L::kOffV8 + s8 * L::kV8, &tm_v, g * HD, row, &bars->v8_full[s8]);
+                    } else {
+                        const uint32_t sv = vc % L::kVStages;
+                        if (!mbar_wait(&bars->v_empty[sv], ((vc / L::kVStages) & 1) ^ 1, abort_flag,
+                                       dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bars->v_full[sv], L::kV);
+                        for (int c = 0; c < HD / 64; ++c)
+                            tma_load_2d(smem + L::kOffV + sv * L::kV + c * L::kChunk, &tm_v,
+                                        g * HD + 64 * c, row, &bars->v_full[sv]);
                     }
-                    mbar_arrive_expect_tx(&bars->v_full[sv], L::kKV);
-                    for (int c = 0; c < HD / 64; ++c)
-                        tma_load_2d(smem + L::kOffV + sv * L::kKV + c * L::kChunk, &tm_v,
-                                    g * HD + 64 * c, row, &bars->v_full[sv]);
                     ++vc;
                 }
             }
@@ -205,16 +340,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     drain_wait(&bars->q_full[n % L::kQSlots], (n / L::kQSlots) & 1);
                 for (uint32_t n = kc > L::kKStages ? kc - L::kKStages : 0; n < kc; ++n)
                     drain_wait(&bars->k_full[n % L::kKStages], (n / L::kKStages) & 1);
-                for (uint32_t n = vc > L::kVStages ? vc - L::kVStages : 0; n < vc; ++n)
-                    drain_wait(&bars->v_full[n % L::kVStages], (n / L::kVStages) & 1);
+                if (F8) {
+                    for (uint32_t n = vc > L::kV8Stages ? vc - L::kV8Stages : 0; n < vc; ++n)
+                        drain_wait(&bars->v8_full[n % L::kV8Stages], (n / L::kV8Stages) & 1);
+                } else {
+                    for (uint32_t n = vc > L::kVStages ? vc - L::kVStages : 0; n < vc; ++n)
+                        drain_wait(&bars->v_full[n % L::kVStages], (n / L::kVStages) & 1);
+                }
             }
         }
         __syncwarp();
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, HD, 0, 1);
+            constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(kBlockM, kBlockN)
+                                             : idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+            constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(kBlockM, HD, 0, 1)
+                                             : idesc_bf16_f32(kBlockM, HD, 0, 1);
             uint32_t qc = 0;    // Q sub-tiles of the items before the current one
             uint32_t g = 0;     // global index of the current key tile (the K / V ring position)
             uint32_t p_cnt[2] = {0, 0};         // P.V products issued per sub-tile
@@ -227,7 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             auto issue_pv = [&](int r) -> bool {
                 if (!mbar_wait(&bars->p_full[r], p_cnt[r] & 1, abort_flag, dev_status)) return false;
                 tc_fence_after();
-                const uint32_t v_tile = sbase + L::kOffV + ((g - 1) % L::kVStages) * L::kKV;
+                const uint32_t v_tile = sbase + L::kOffV + ((g - 1) % L::kVStages) * L::kV;
                 const uint32_t a_p = tmem + (kSepP ? kTmP + 64 * r : 128 * r);
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk)
@@ -242,8 +384,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             };
             auto wait_v_prev = [&]() -> bool {
                 const uint32_t n = g - 1;
-                if (!mbar_wait(&bars->v_full[n % L::kVStages], (n / L::kVStages) & 1, abort_flag,
-                               dev_status))
+                uint64_t* bar = AUXV ? &bars->v_add[n % L::kVStages] : &bars->v_full[n % L::kVStages];
+                if (!mbar_wait(bar, (n / L::kVStages) & 1, abort_flag, dev_status))
                     return false;
                 return true;
             };
@@ -277,7 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         ok = false;
                         break;
                     }
-                    const uint32_t k_tile = sbase + L::kOffK + sk * L::kKV;
+                    const uint32_t k_tile = sbase + L::kOffK + sk * L::kK;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         if (pend[r] && !issue_pv(r)) {
@@ -301,10 +443,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                         tc_fence_after();
                         const uint32_t q_tile = sbase + L::kOffQ + q_slot[r] * L::kQSub;
+                        if (F8) {
 #pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk)
-                            umma_f16_ss(tmem + 128 * r, desc_kmajor(q_tile, kk), desc_kmajor(k_tile, kk),
-                                        idesc_qk, kk == 0 ? 0u : 1u);
+                            for (int kk = 0; kk < HD / 32; ++kk)
+                                umma_f8_ss(tmem + 128 * r, desc_kmajor_e4m3<HD>(q_tile, kk),
+                                           desc_kmajor_e4m3<HD>(k_tile, kk), idesc_qk, kk == 0 ? 0u : 1u);
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                umma_f16_ss(tmem + 128 * r, desc_kmajor(q_tile, kk),
+                                            desc_kmajor(k_tile, kk), idesc_qk, kk == 0 ? 0u : 1u);
+                        }
                         umma_commit(&bars->s_full[r]);
                         if (t == it.t_last[r]) umma_commit(&bars->q_empty[q_slot[r]]);
                         pend[r] = true;
@@ -339,7 +488,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t tm_s = tm_lane + 128 * r;
         const uint32_t tm_p = kSepP ? tm_lane + kTmP + 64 * r : tm_s;
         const uint32_t tm_o = tm_lane + L::kTmO + HD * r;
-        const float scale_log2 = p.scale * kLog2e;
+        const float scale_log2 = p.scale * (F8 ? p.qk_scale : 1.0f) * kLog2e;
         const uint64_t scale2 = f32x2(scale_log2, scale_log2);
         const int window = p.window;
         uint32_t s_cnt = 0, o_cnt = 0;
@@ -424,9 +573,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
                     if (cls[c] == 1) {
-                        chunk_exp<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
+                        chunk_exp<kMaskNone, F8>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
                     } else if (cls[c] == 2) {
-                        chunk_exp<kMaskBoth>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
+                        chunk_exp<kMaskBoth, F8>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = 0u;
@@ -463,44 +612,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ++o_cnt;
             tc_fence_after();
             const bool valid = row < nr;
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float inv_l = l > 0.f ? (F8 ? p.v_scale : 1.f) / l : 0.f;
             // O / l -> bf16, staged through this sub-tile's Q slot (its last S has completed):
-            // each warp writes its 32 rows with an XOR swizzle of the 16-byte chunks, then copies
-            // them out two rows per instruction, so every global store of the warp covers 512
-            // contiguous bytes. Rows past the end of the document are not written.
+            // each warp writes kStageRows of its rows at a time (all 32 when the slot holds them,
+            // 16 for the narrower e4m3 slot) with an XOR swizzle of the 16-byte chunks, then copies
+            // them out two rows per instruction at hd 128, so every global store of the warp covers
+            // 512 contiguous bytes. Rows past the end of the document are not written.
             constexpr int kChunks = HD / 8;  // 16-byte chunks per row
-            uint8_t* stage = smem + L::kOffQ + (my_q % L::kQSlots) * L::kQSub + (warp & 3) * 32 * (HD * 2);
-            const int wrow = row & 31;
-            {
-                uint32_t ov[HD];
+            constexpr int kSR = L::kStageRows;
+            uint8_t* stage = smem + L::kOffQ + (my_q % L::kQSlots) * L::kQSub + (warp & 3) * kSR * (HD * 2);
+            uint32_t ov[HD];
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) tmem_ld32(tm_o + 32 * c, ov + 32 * c);
-                tmem_wait_ld();
+            for (int c = 0; c < HD / 32; ++c) tmem_ld32(tm_o + 32 * c, ov + 32 * c);
+            tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
-                    regs_after_wait(ov + 32 * c);
+            for (int c = 0; c < HD / 32; ++c) regs_after_wait(ov + 32 * c);
+#pragma unroll 1
+            for (int ps = 0; ps < 32 / kSR; ++ps) {
+                if ((lane / kSR) == ps) {
+                    const int wrow = lane % kSR;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint32_t* w8 = ov + 32 * c + 8 * q4;
-                        const uint4 w4 = make_uint4(
-                            pack_bf16x2(__uint_as_float(w8[0]) * inv_l, __uint_as_float(w8[1]) * inv_l),
-                            pack_bf16x2(__uint_as_float(w8[2]) * inv_l, __uint_as_float(w8[3]) * inv_l),
-                            pack_bf16x2(__uint_as_float(w8[4]) * inv_l, __uint_as_float(w8[5]) * inv_l),
-                            pack_bf16x2(__uint_as_float(w8[6]) * inv_l, __uint_as_float(w8[7]) * inv_l));
-                        const int chunk = 4 * c + q4;
-                        *reinterpret_cast<uint4*>(stage + wrow * (HD * 2) + ((chunk ^ (wrow & (kChunks - 1))) << 4)) = w4;
+                    for (int c = 0; c < HD / 32; ++c) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint32_t* w8 = ov + 32 * c + 8 * q4;
+                            const uint4 w4 = make_uint4(
+                                pack_bf16x2(__uint_as_float(w8[0]) * inv_l, __uint_as_float(w8[1]) * inv_l),
+                                pack_bf16x2(__uint_as_float(w8[2]) * inv_l, __uint_as_float(w8[3]) * inv_l),
+                                pack_bf16x2(__uint_as_float(w8[4]) * inv_l, __uint_as_float(w8[5]) * inv_l),
+                                pack_bf16x2(__uint_as_float(w8[6]) * inv_l, __uint_as_float(w8[7]) * inv_l));
+                            const int chunk = 4 * c + q4;
+                            *reinterpret_cast<uint4*>(stage + wrow * (HD * 2) +
+                                                      ((chunk ^ (wrow & (kChunks - 1))) << 4)) = w4;
+                        }
                     }
                 }
-            }
-            __syncwarp();
-            {
-                const int row0 = qr0 + r0;  // first slot of this warp's rows
+                __syncwarp();
+                const int row0 = qr0 + r0 + ps * kSR;  // first slot of the staged rows
                 constexpr int kRowsPerIter = 32 / kChunks;
 #pragma unroll 4
-                for (int j = 0; j < 32 / kRowsPerIter; ++j) {
+                for (int j = 0; j < kSR / kRowsPerIter; ++j) {
                     const int rl = j * kRowsPerIter + lane / kChunks;
                     const int chunk = lane % kChunks;
-                    if (r0 + rl < nr) {
+                    if (r0 + ps * kSR + rl < nr) {
                         const uint4 w4 = *reinterpret_cast<const uint4*>(
                             stage + rl * (HD * 2) + ((chunk ^ (rl & (kChunks - 1))) << 4));
                         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) +
@@ -508,6 +662,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         *reinterpret_cast<uint4*>(dst) = w4;
                     }
                 }
+                __syncwarp();
             }
             __syncwarp();
             fence_proxy_async_smem();  // the slot's next fill is written by the async proxy (TMA)
@@ -524,27 +679,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 9) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-template <int HD>
+template <int HD, bool F8, bool AUXV>
 static cudaError_t launch_tc_hd(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const int4* items, WorkspaceHeader* hdr,
                                 cudaStream_t stream) {
-    using L = TcLayout<HD>;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD>,
+    using L = BlockLayout<HD, F8>;
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, F8, AUXV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    attn_tc_kernel<HD><<<sms, kTcThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p, items, hdr);
+    attn_tc_kernel<HD, F8, AUXV><<<sms, kTcThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p, items, hdr);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_tc(const AttnProblem& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const int4* items, WorkspaceHeader* hdr,
-                           cudaStream_t stream) {
-    if (p.head_dim == 128) return launch_tc_hd<128>(p, tm_q, tm_k, tm_v, items, hdr, stream);
-    if (p.head_dim == 64) return launch_tc_hd<64>(p, tm_q, tm_k, tm_v, items, hdr, stream);
+                           cudaStream_t stream, bool fp8) {
+    const bool aux = p.v_aux != nullptr;
+    if (fp8 && aux) return cudaErrorInvalidValue;
+    if (p.head_dim == 128)
+        return fp8 ? launch_tc_hd<128, true, false>(p, tm_q, tm_k, tm_v, items, hdr, stream)
+               : aux ? launch_tc_hd<128, false, true>(p, tm_q, tm_k, tm_v, items, hdr, stream)
+                     : launch_tc_hd<128, false, false>(p, tm_q, tm_k, tm_v, items, hdr, stream);
+    if (p.head_dim == 64)
+        return fp8 ? launch_tc_hd<64, true, false>(p, tm_q, tm_k, tm_v, items, hdr, stream)
+               : aux ? launch_tc_hd<64, false, true>(p, tm_q, tm_k, tm_v, items, hdr, stream)
+                     : launch_tc_hd<64, false, false>(p, tm_q, tm_k, tm_v, items, hdr, stream);
     return cudaErrorInvalidValue;
 }
 

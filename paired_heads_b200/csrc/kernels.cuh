@@ -56,6 +56,14 @@ struct AttnProblem {
     // Value embedding (pha_attn_fwd_aux_v): added to v, with v's layout, before attention;
     // nullptr: none.
     const void* v_aux;
+    // Failure-detection test hook (band kernel): > 0 makes the softmax warps first wait up to this
+    // many microseconds on a barrier that nothing signals; 0 in every normal call.
+    int test_stall_us;
+    // FP8 inputs (pha_attn_fwd_fp8): q, k, v hold e4m3 codes standing for qk / v scale times
+    // their values; the block kernel folds qk_scale (= q_scale * k_scale) into the logit scale
+    // and v_scale into the epilogue. 1 / 1 otherwise.
+    float qk_scale;
+    float v_scale;
 };
 
 cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
@@ -114,9 +122,11 @@ cudaError_t launch_schedule(const AttnProblem& p, bool band, int capacity, int* 
 // tcgen05 attention over a scheduled work list. tm_q / tm_k / tm_v are 2-D bf16 tensor maps
 // over the slot view ([slots][heads * head_dim] and [slots][kv_heads * head_dim]) with a
 // 64 x 128 box and 128-byte swizzle.
+// fp8: q, k, v are e4m3; tm_q / tm_k are 2-D uint8 maps with a head_dim x 128 box (128-byte
+// swizzle at head_dim 128, 64-byte at 64) and tm_v the same box without swizzle.
 cudaError_t launch_attn_tc(const AttnProblem& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const int4* items, WorkspaceHeader* hdr,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool fp8 = false);
 
 // True when the band kernel covers the problem: causal, 1 <= window <= kBlockN.
 inline bool band_applies(const AttnProblem& p) {

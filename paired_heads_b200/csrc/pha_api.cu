@@ -45,6 +45,25 @@ bool encode_slot_map(CUtensorMap* map, const void* base, uint64_t width, uint64_
     return r == CUDA_SUCCESS;
 }
 
+// 2-D uint8 map over [rows][width] bytes for e4m3 tiles: box box_inner x 128, swizzled to match
+// the box width (128-byte rows: 128-byte swizzle; 64-byte rows: 64-byte swizzle) or unswizzled.
+bool encode_u8_map(CUtensorMap* map, const void* base, uint64_t width, uint64_t rows,
+                   uint32_t box_inner, bool swizzle) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {width, rows};
+    cuuint64_t strides[1] = {width};
+    cuuint32_t box[2] = {box_inner, 128};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = !swizzle ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                  : box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                     : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int64_t div_up(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 int64_t max_work_items(int batch, int max_len, int n_heads, int paired) {
@@ -268,7 +287,7 @@ pha_status attn_fwd_impl(const void* q, const void* k, const void* v, const void
                          const int32_t* cu_seqlens, int batch, int max_len, int total_tokens,
                          int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype, int causal,
                          int window, int paired, float scale, void* o, float* lse, void* workspace,
-                         size_t workspace_bytes, pha_stream_t stream) {
+                         size_t workspace_bytes, pha_stream_t stream, int test_stall_us = 0) {
     if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
     // With no tokens the q / k / v / o / lse buffers may be empty (NULL); cu_seqlens is still read.
     const bool have = total_tokens > 0;
@@ -301,9 +320,17 @@ pha_status attn_fwd_impl(const void* q, const void* k, const void* v, const void
     p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
     p.o = o;
     p.lse = lse;
-    if (v_aux) {
-        // value embedding: the band kernel only (bf16, causal, 1 <= window <= 128)
+    p.qk_scale = 1.0f;
+    p.v_scale = 1.0f;
+    if (test_stall_us != 0) {
+        // the failure-detection hook exists in the band kernel only
         if (dtype != PHA_BF16 || !band_applies(p)) return PHA_ERR_UNSUPPORTED;
+        if (test_stall_us < 1 || test_stall_us > 100000) return PHA_ERR_INVALID;
+        p.test_stall_us = test_stall_us;
+    }
+    if (v_aux) {
+        // value embedding: the bf16 tensor-core kernels (band and block)
+        if (dtype != PHA_BF16) return PHA_ERR_UNSUPPORTED;
         if (!aligned16(v_aux)) return PHA_ERR_INVALID;
         p.v_aux = v_aux;
     }
@@ -369,6 +396,81 @@ pha_status pha_attn_fwd_aux_v(const void* q, const void* k, const void* v, const
     return attn_fwd_impl(q, k, v, total_tokens > 0 ? aux_v : nullptr, cu_seqlens, batch, max_len,
                          total_tokens, n_heads, n_kv_heads, head_dim, dtype, causal, window,
                          paired, scale, o, lse, workspace, workspace_bytes, stream);
+}
+
+pha_status pha_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale,
+                            float k_scale, float v_scale, const int32_t* cu_seqlens, int batch,
+                            int max_len, int total_tokens, int n_heads, int n_kv_heads,
+                            int head_dim, int causal, int window, int paired, float scale, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes,
+                            pha_stream_t stream) {
+    const bool have = total_tokens > 0;
+    if ((have && (!q8 || !k8 || !v8 || !o || !aligned16(q8) || !aligned16(k8) || !aligned16(v8) ||
+                  !aligned16(o))) ||
+        !cu_seqlens || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || batch <= 0 ||
+        max_len < 0 || total_tokens < 0 || total_tokens > (1 << 29) || n_heads <= 0 ||
+        n_kv_heads <= 0 || n_heads > 4096 || n_heads % n_kv_heads != 0 || head_dim <= 0 ||
+        (causal != 0 && causal != 1) || (paired != 0 && paired != 1) || !(scale == scale) ||
+        !(q_scale > 0.f) || !(k_scale > 0.f) || !(v_scale > 0.f) || !(q_scale < INFINITY) ||
+        !(k_scale < INFINITY) || !(v_scale < INFINITY))
+        return PHA_ERR_INVALID;
+    if (paired && ((n_heads & 1) || (n_kv_heads & 1))) return PHA_ERR_INVALID;
+    if (!causal && window > 0) return PHA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PHA_ERR_UNSUPPORTED;
+
+    AttnProblem p{};
+    p.q = q8;
+    p.k = k8;
+    p.v = v8;
+    p.cu_seqlens = cu_seqlens;
+    p.batch = batch;
+    p.max_len = max_len;
+    p.total_tokens = total_tokens;
+    p.slot_mult = paired ? 2 : 1;
+    p.heads = paired ? n_heads / 2 : n_heads;
+    p.kv_heads = paired ? n_kv_heads / 2 : n_kv_heads;
+    p.head_dim = head_dim;
+    p.causal = causal;
+    p.window = window > 0 ? window : 0;
+    p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
+    p.o = o;
+    p.lse = lse;
+    p.qk_scale = q_scale * k_scale;
+    p.v_scale = v_scale;
+
+    const size_t need = pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PHA_ERR_WORKSPACE;
+    const size_t fixed = kWorkspaceHeaderBytes + workspace_doc_bytes(batch);
+    const int64_t cap64 = static_cast<int64_t>((workspace_bytes - fixed) / sizeof(int4));
+    const int capacity = cap64 > 0x7FFFFFFF ? 0x7FFFFFFF : static_cast<int>(cap64);
+    auto* base = static_cast<uint8_t*>(workspace);
+    auto* hdr = reinterpret_cast<WorkspaceHeader*>(base);
+    auto* doc_blocks = reinterpret_cast<int*>(base + kWorkspaceHeaderBytes);
+    auto* items = reinterpret_cast<int4*>(base + fixed);
+    // every window runs on the block kernel (its FP8 variant)
+    if (launch_schedule(p, false, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+        return PHA_ERR_CUDA;
+    if (total_tokens == 0) return PHA_OK;
+    const uint64_t rows = static_cast<uint64_t>(total_tokens) * p.slot_mult;
+    CUtensorMap tq, tk, tv;
+    if (!encode_u8_map(&tq, q8, static_cast<uint64_t>(p.heads) * head_dim, rows, head_dim, true) ||
+        !encode_u8_map(&tk, k8, static_cast<uint64_t>(p.kv_heads) * head_dim, rows, head_dim, true) ||
+        !encode_u8_map(&tv, v8, static_cast<uint64_t>(p.kv_heads) * head_dim, rows, head_dim, false))
+        return PHA_ERR_CUDA;
+    return launch_attn_tc(p, tq, tk, tv, items, hdr, stream, true) == cudaSuccess ? PHA_OK
+                                                                                   : PHA_ERR_CUDA;
+}
+
+pha_status pha_test_attn_fwd_stalled(const void* q, const void* k, const void* v,
+                                     const int32_t* cu_seqlens, int batch, int max_len,
+                                     int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                                     pha_dtype dtype, int causal, int window, int paired,
+                                     float scale, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, int stall_us, pha_stream_t stream) {
+    if (stall_us == 0) return PHA_ERR_INVALID;
+    return attn_fwd_impl(q, k, v, nullptr, cu_seqlens, batch, max_len, total_tokens, n_heads,
+                         n_kv_heads, head_dim, dtype, causal, window, paired, scale, o, lse,
+                         workspace, workspace_bytes, stream, stall_us);
 }
 
 pha_status pha_attn_status(const void* workspace, int* status, int* n_items, pha_stream_t stream) {

@@ -74,14 +74,15 @@ __device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
 // CTA-wide abort flag and the device status) when the limit passes or another thread of the
 // CTA has already aborted. Never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag, int* dev_status) {
+                                          volatile int* abort_flag, int* dev_status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_test(bar, parity)) return true;
         if ((it & 63u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 if (dev_status) atomicExch(dev_status, DEV_TIMEOUT);
                 return false;
@@ -185,6 +186,18 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (8-bit float inputs, fp32 accumulate),
+// cta_group::1; one instruction covers K = 32 elements.
+__device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when all tcgen05 operations issued so far by this thread complete.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile(
@@ -203,6 +216,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     d |= 1ull << 46;  // descriptor version for sm_100
     d |= 2ull << 61;  // 128-byte swizzle
     return d;
+}
+
+// Shared-memory matrix descriptor for a 64-byte-swizzled tile whose base is 512-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;  // descriptor version for sm_100
+    d |= 4ull << 61;  // 64-byte swizzle
+    return d;
+}
+
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0), fp32 D, M x N, K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f16: f16 A and B (format code 0), fp32 D, operand majors.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4) | (static_cast<uint32_t>(a_mn_major) << 15) |
+           (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N, operand majors (0 = K-major).
@@ -361,6 +397,20 @@ __device__ __forceinline__ void ex2_poly2(float xa, float xb, float& ya, float& 
     f32x2_split(p2, pa, pb);
     ya = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ja) << 23));
     yb = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(jb) << 23));
+}
+
+// Two e4m3 values (low byte -> low half) to two f16 values, exactly (every e4m3 value is an f16
+// value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

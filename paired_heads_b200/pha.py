@@ -48,6 +48,11 @@ _lib.pha_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i
 _lib.pha_attn_status.argtypes = [_p, ctypes.POINTER(_i), ctypes.POINTER(_i), _p]
 _lib.pha_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                       ctypes.c_float, _p, _p, _p]
+_lib.pha_attn_fwd_fp8.argtypes = [_p, _p, _p, ctypes.c_float, ctypes.c_float, ctypes.c_float, _p,
+                                  _i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_float, _p, _p, _p,
+                                  _sz, _p]
+_lib.pha_test_attn_fwd_stalled.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                           _i, ctypes.c_float, _p, _p, _p, _sz, _i, _p]
 _lib.pha_attn_fwd_aux_v.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                     ctypes.c_float, _p, _p, _p, _sz, _p]
 _lib.pha_rope_bwd.argtypes = [_p, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _i, _p]
@@ -58,7 +63,7 @@ _lib.pha_attn_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i
 _lib.pha_qk_norm_rope.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _p, _i, _i, _p, _i, _i, _i,
                                   _i, _i, _i, _i, _p]
 for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status",
-           "pha_attn_fwd_noalloc", "pha_qk_norm_rope", "pha_attn_fwd_aux_v", "pha_rope_bwd",
+           "pha_attn_fwd_noalloc", "pha_test_attn_fwd_stalled", "pha_attn_fwd_fp8", "pha_qk_norm_rope", "pha_attn_fwd_aux_v", "pha_rope_bwd",
            "pha_attn_bwd"):
     getattr(_lib, _f).restype = _i
 
@@ -255,6 +260,37 @@ def pha_attn_fwd_noalloc(q, k, v, cu_seqlens, max_len: int, o, lse, *, causal: b
                                      total_tokens, n_heads, n_kv_heads, head_dim, dtype,
                                      int(causal), int(window), int(paired), float(scale), _ptr(o),
                                      _ptr(lse), _stream(stream, q)))
+
+
+def pha_attn_fwd_fp8(q8, k8, v8, q_scale: float, k_scale: float, v_scale: float, cu_seqlens,
+                     max_len: int, o, lse, workspace, *, causal: bool = True, window: int = 0,
+                     paired: bool = False, scale: float = 0.0, stream=None):
+    """Attention forward over e4m3 q8, k8, v8 (torch.float8_e4m3fn or uint8 tensors) with
+    per-tensor scales, into o (bf16, q's shape) and lse [T][H] float32 (or None)."""
+    total_tokens, n_heads, head_dim = q8.shape
+    _check("pha_attn_fwd_fp8",
+           _lib.pha_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_scale), float(k_scale),
+                                 float(v_scale), _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+                                 max_len, total_tokens, n_heads, k8.shape[1], head_dim,
+                                 int(causal), int(window), int(paired), float(scale), _ptr(o),
+                                 _ptr(lse), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream, q8)))
+
+
+def pha_test_attn_fwd_stalled(q, k, v, cu_seqlens, max_len: int, o, lse, workspace, stall_us: int,
+                              *, causal: bool = True, window: int = 0, paired: bool = False,
+                              scale: float = 0.0, stream=None):
+    """Failure-detection test hook: pha_attn_fwd whose band-kernel softmax first waits stall_us
+    microseconds on a barrier nothing signals (device status 3 afterwards, no output written)."""
+    total_tokens, n_heads, head_dim = q.shape
+    _check("pha_test_attn_fwd_stalled",
+           _lib.pha_test_attn_fwd_stalled(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                          cu_seqlens.shape[0] - 1, max_len, total_tokens, n_heads,
+                                          k.shape[1], head_dim, _dtype_code(q), int(causal),
+                                          int(window), int(paired), float(scale), _ptr(o),
+                                          _ptr(lse), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          int(stall_us), _stream(stream, q)))
 
 
 def pha_attn_status(workspace, stream=None):

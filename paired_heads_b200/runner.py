@@ -72,11 +72,10 @@ class AttentionStep:
 
     @property
     def aux_v_supported(self) -> bool:
-        """Whether pha_attn_fwd_aux_v covers this shape (the band kernel: bf16, causal,
-        1 <= window <= 128, head_dim 64 or 128)."""
+        """Whether pha_attn_fwd_aux_v covers this shape (the bf16 tensor-core kernels: head_dim
+        64 or 128)."""
         s = self.s
-        return (s.dtype == "bf16" and s.causal and 1 <= s.window <= 128
-                and s.head_dim in (64, 128))
+        return s.dtype == "bf16" and s.head_dim in (64, 128)
 
     def attn_aux_v(self, q, k, v, aux_v, cu_seqlens, stream=None):
         """Attention over (q, k, v + aux_v); v and aux_v are left unchanged."""

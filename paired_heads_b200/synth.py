@@ -137,6 +137,27 @@ def make_inputs(w: Workload, rank: int = 0, device: Optional[str] = None):
     return out
 
 
+def make_fp8_inputs(w: Workload, rank: int = 0, device: Optional[str] = None):
+    """FP8 versions of make_inputs' q, k, v: each float32 draw divided by its tensor's scale
+    s = max|x| / 448 (rounded to float32, so that the largest magnitude lands on e4m3's largest
+    finite value) and cast to torch.float8_e4m3fn. Returns a dict with q8, k8, v8 (float8 tensors),
+    q_scale, k_scale, v_scale (floats; x ~ scale * value(code)), cu_seqlens and positions."""
+    import torch
+
+    out = {}
+    for name, a in zip(("q", "k", "v"), qkv_float32(w, rank)):
+        amax = float(np.abs(a).max()) if a.size else 1.0
+        sc = float(np.float32(amax / 448.0)) if amax > 0 else 1.0
+        t = torch.from_numpy(a) / sc
+        out[name + "8"] = t.to(torch.float8_e4m3fn)
+        out[name + "_scale"] = sc
+    out["cu_seqlens"] = torch.from_numpy(cu_seqlens(w))
+    out["positions"] = torch.from_numpy(positions(w))
+    if device is not None:
+        out = {key: (t.to(device) if hasattr(t, "to") else t) for key, t in out.items()}
+    return out
+
+
 def to_f64(t) -> np.ndarray:
     """Exact float64 copy of a (bf16 / f32) torch tensor -- what the oracle receives."""
     import torch

@@ -28,9 +28,11 @@ def _declared():
 
 def test_header_declares_the_entry_points():
     assert _declared() == ["pha_attn_bwd", "pha_attn_bwd_workspace_bytes", "pha_attn_fwd",
-                           "pha_attn_fwd_aux_v", "pha_attn_fwd_noalloc", "pha_attn_status",
+                           "pha_attn_fwd_aux_v", "pha_attn_fwd_fp8", "pha_attn_fwd_noalloc",
+                           "pha_attn_status",
                            "pha_attn_workspace_bytes", "pha_qk_norm_rope", "pha_rope",
-                           "pha_rope_bwd", "pha_rope_tables", "pha_status_string"]
+                           "pha_rope_bwd", "pha_rope_tables", "pha_status_string",
+                           "pha_test_attn_fwd_stalled"]
 
 
 def test_library_exports_every_declared_symbol(pha):
@@ -103,6 +105,62 @@ def test_attn_argument_errors(pha, kw, code):
         assert _attn(pha, ws_bytes=10, **kw) == -3
         return
     assert _attn(pha, **kw) == code
+
+
+def _stalled(pha, stall_us, **kw):
+    args = dict(q=A, k=A, v=A, cu=A, batch=1, max_len=128, total=128, H=4, Hkv=4, hd=64,
+                dtype=pha.PHA_BF16, causal=1, window=128, paired=0, scale=0.0, o=A, lse=A, ws=A,
+                ws_bytes=10)
+    args.update(kw)
+    return pha.library().pha_test_attn_fwd_stalled(
+        args["q"], args["k"], args["v"], args["cu"], args["batch"], args["max_len"], args["total"],
+        args["H"], args["Hkv"], args["hd"], args["dtype"], args["causal"], args["window"],
+        args["paired"], ctypes.c_float(args["scale"]), args["o"], args["lse"], args["ws"],
+        args["ws_bytes"], stall_us, None)
+
+
+@pytest.mark.parametrize("stall_us,kw,code", [
+    (0, {}, -1),                               # the hook needs a stall
+    (-5, {}, -1),
+    (100001, {}, -1),
+    (1000, dict(window=0), -2),                # only the band kernel has the hook
+    (1000, dict(window=256), -2),
+    (1000, dict(dtype=1, hd=16), -2),
+    (1000, {}, -3),                            # otherwise the checks of pha_attn_fwd apply
+])
+def test_stall_hook_argument_errors(pha, stall_us, kw, code):
+    assert _stalled(pha, stall_us, **kw) == code
+
+
+def _fp8(pha, **kw):
+    args = dict(q=A, k=A, v=A, sq=1.0, sk=1.0, sv=1.0, cu=A, batch=1, max_len=128, total=128, H=4,
+                Hkv=4, hd=64, causal=1, window=0, paired=0, scale=0.0, o=A, lse=A, ws=A,
+                ws_bytes=1 << 20)
+    args.update(kw)
+    f = ctypes.c_float
+    return pha.library().pha_attn_fwd_fp8(
+        args["q"], args["k"], args["v"], f(args["sq"]), f(args["sk"]), f(args["sv"]), args["cu"],
+        args["batch"], args["max_len"], args["total"], args["H"], args["Hkv"], args["hd"],
+        args["causal"], args["window"], args["paired"], f(args["scale"]), args["o"], args["lse"],
+        args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(sq=0.0), -1),                        # scales must be positive and finite
+    (dict(sk=-1.0), -1),
+    (dict(sv=float("inf")), -1),
+    (dict(sq=float("nan")), -1),
+    (dict(H=6, Hkv=4), -1),
+    (dict(H=5, Hkv=5, paired=1), -1),
+    (dict(causal=0, window=16), -2),
+    (dict(hd=96), -2),                         # head_dim 64 / 128 only
+    (dict(q=MIS), -1),
+    (dict(v=None), -1),
+    (dict(ws=None), -3),
+    (dict(ws_bytes=100), -3),
+])
+def test_fp8_argument_errors(pha, kw, code):
+    assert _fp8(pha, **kw) == code
 
 
 def _rope(pha, **kw):

@@ -1,6 +1,7 @@
-"""Value embedding added to v inside the attention kernel (pha_attn_fwd_aux_v) on the GPU: bit for
+"""Value embedding added to v inside the attention kernels (pha_attn_fwd_aux_v) on the GPU: bit for
 bit the O and LSE of pha_attn_fwd on v + aux_v formed by a bf16 tensor addition, v and aux_v left
-unchanged, and within the parity bar of the oracle. Needs a B200."""
+unchanged, and within the parity bar of the oracle, on the band kernel (causal windows <= 128)
+and the block kernel (no window, longer windows). Needs a B200."""
 import numpy as np
 import pytest
 import torch
@@ -41,12 +42,17 @@ def _both(w, inp, aux):
 
 
 CASES = [
-    # doc lens, H, Hkv, hd, window, paired
+    # doc lens, H, Hkv, hd, window, paired -- windows <= 128 run on the band kernel, the others
+    # (0 = no window) on the block kernel
     ((700, 5, 260), 6, 6, 128, 128, True),
     ((512, 513, 64, 1, 2049), 4, 2, 128, 128, True),
     ((1024, 1025, 127, 129, 1), 4, 2, 64, 2, False),
     ((3000, 7), 8, 2, 128, 100, False),
     ((333, 64), 8, 4, 64, 37, True),
+    ((1500, 257, 1), 4, 4, 64, 0, False),
+    ((900, 300), 8, 2, 128, 0, True),
+    ((2100, 33), 4, 2, 64, 300, True),
+    ((1030,), 4, 4, 128, 1024, False),
 ]
 
 
