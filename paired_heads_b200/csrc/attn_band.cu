@@ -12,11 +12,18 @@
 // window tile it is. Consecutive query tiles alternate between the two softmax warpgroups, so
 // both warpgroups have one tile at every step and every K / V tile is read from HBM once per run.
 //
-// CTA = 11 warps, persistent, one per SM, items in snake order over the longest-first list:
-//   warps 0-3, 4-7   softmax warpgroups w = 0, 1: query tiles n (CTA-wide count) with n % 2 == w
+// CTA = 12 warps (16 with the value embedding), persistent, one per SM, items in snake order over
+// the longest-first list; the softmax warpgroups run with 200 registers per thread:
+//   warps 0-3, 4-7   softmax warpgroups w = 0, 1: query tiles n (CTA-wide count) with n % 2 == w.
+//                    The whole 128-column S row is loaded from TMEM with one wait; hidden scores
+//                    are set to -inf in registers (per-row bit masks, skipped for 32-column chunks
+//                    that are wholly visible or hidden for every row of the warp); max and
+//                    exponentials run on independent accumulator chains
 //   warp 8           TMA producer: Q tiles into a ring of 3 slots, K and V tiles into their rings
 //   warps 9, 10      MMA issuers, one per warpgroup (warp 9 also owns the 512 TMEM columns), so a
 //                    warpgroup's next S never waits behind the other warpgroup's softmax
+//   warp 11          idle (completes the third warpgroup for the register split)
+//   warps 12-15      value embedding only: add aux_v to each landed V tile
 // TMEM columns: S_w at 128 w (P_w aliases its first 64 columns), O_w at 256 + hd w.
 // A K / V stage is released when both issuers have arrived for its step: by a commit after
 // their MMAs on it, or by a plain arrive on a step their warpgroup does not use.
@@ -33,8 +40,16 @@
 
 namespace pha {
 
-constexpr int kBandThreads = 352;     // 8 softmax warps, producer, 2 MMA issuers
-constexpr int kBandAuxThreads = 480;  // + an adder warpgroup (value embedding)
+// 8 softmax warps; producer, 2 MMA issuers and an idle warp (a whole third warpgroup for the
+// register split); with the value embedding a fourth warpgroup of adders.
+constexpr int kBandThreads = 384;
+constexpr int kBandAuxThreads = 512;
+// Register split, per thread: the softmax warpgroups hold a whole 128-column score row. Without
+// the embedding 8 x 200 + 4 x 88 = 1952 <= 12 x 168 (the launch allocation of 384 threads); with
+// it 8 x 200 + 8 x 56 = 2048 <= 16 x 128 (512 threads).
+constexpr int kBandRegsSoftmax = 200;
+constexpr int kBandRegsOther = 88;
+constexpr int kBandRegsOtherAux = 56;
 
 struct BandBars {
     uint64_t q_full[3], q_empty[3];
@@ -110,8 +125,18 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads;
     const int G = p.heads / p.kv_heads;
+    static_assert(8 * kBandRegsSoftmax + 4 * kBandRegsOther <= 12 * 168, "register split");
+    static_assert(8 * kBandRegsSoftmax + 8 * kBandRegsOtherAux <= 16 * 128, "register split");
 
-    if (warp == 8) {
+    if (warp >= 8) {  // every warp of the third (and fourth) warpgroup, then their roles
+        if (AUXV)
+            regs_decrease<kBandRegsOtherAux>();
+        else
+            regs_decrease<kBandRegsOther>();
+    }
+    if (warp == 11) {
+        // ------------------------------------------------------------ idle (register split only)
+    } else if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t qc = 0, kc = 0, vc = 0;  // Q / K / V tiles issued so far
@@ -177,7 +202,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
             }
         }
         __syncwarp();
-    } else if (AUXV && warp >= 11) {
+    } else if (AUXV && warp >= 12) {
         // ------------------------------------------------------------ adder warpgroup
         // V tiles in the producer's order; each gets aux_v added once it has landed, then is
         // published to the MMA issuers.
@@ -197,15 +222,14 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[sv], (vc / S) & 1, abort_flag,
                                                        dev_status));
                 if (!ok) break;
-                add_aux_tile<HD, 128, 128 / (1024 / HD)>(smem + L::kOffV + sv * L::kKV, aux,
-                                                          kv_first + s * kBlockN, gk, p.kv_heads,
-                                                          slots, at);
+                add_aux_tile<HD, 128, 4>(smem + L::kOffV + sv * L::kKV, aux, kv_first + s * kBlockN,
+                                         gk, p.kv_heads, slots, at);
                 fence_proxy_async_smem();  // the tensor cores read the tile next
                 mbar_arrive(&bars->v_add[sv]);
                 ++vc;
             }
         }
-    } else if (warp >= 9) {
+    } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------ MMA issuer of warpgroup w
         const int w = warp - 9;
         if (lane == 0) {
@@ -296,8 +320,9 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
             drain_wait(&bars->drain[w], 0);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------------------ softmax of warpgroup w
+        regs_increase<kBandRegsSoftmax>();
         const int w = warp >> 2;
         const int row = threadIdx.x & 127;  // query row in the tile == TMEM lane
         const int r0 = (warp & 3) * 32;     // first row of this warp
@@ -334,34 +359,44 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                     tc_fence_after();
                     // visible columns of this row: [c_lo, c_hi] (keys i - window + 1 .. i)
                     const int c_lo = i - window + 1 - kv0, c_hi = i - kv0;
-                    // 32-column chunks classed uniformly over this warp's rows (bounds grow with
-                    // the row): skipped when below the first row's lower bound or above the last
-                    // row's upper bound, masked on a side only where some row of the warp needs
-                    // it. Skipped chunks cost no loads and no exponentials, and give P = 0.
-                    const int lo_first = q_start + r0 - window + 1 - kv0, lo_last = lo_first + 31;
-                    const int hi_first = q_start + r0 - kv0, hi_last = hi_first + 31;
-                    auto chunk_class = [&](int c) -> int {  // 4 = skip, else mask mode bits
-                        const int lo = 32 * c, hi = lo + 31;
-                        if (hi < lo_first || lo > hi_last) return 4;
-                        return (lo < lo_last ? kMaskLo : 0) | (hi > hi_first ? kMaskHi : 0);
-                    };
-                    // pass 1: row max over the visible columns
-                    float mx = -INFINITY;
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        const int cls = chunk_class(c);
-                        if (cls == 4) continue;
-                        uint32_t v[32];
-                        tmem_ld32(tm_s + 32 * c, v);
-                        tmem_wait_ld();
-                        regs_after_wait(v);
-                        switch (cls) {
-                            case kMaskNone: mx = row_max32<kMaskNone>(v, 32 * c, c_lo, c_hi, mx); break;
-                            case kMaskLo: mx = row_max32<kMaskLo>(v, 32 * c, c_lo, c_hi, mx); break;
-                            case kMaskHi: mx = row_max32<kMaskHi>(v, 32 * c, c_lo, c_hi, mx); break;
-                            default: mx = row_max32<kMaskBoth>(v, 32 * c, c_lo, c_hi, mx); break;
+                    // the whole S row, one wait
+                    uint32_t v[128];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) tmem_ld32(tm_s + 32 * c, v + 32 * c);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) regs_after_wait(v + 32 * c);
+                    // Hidden scores are set to -inf in place: bit e of vis[c] says whether column
+                    // 32 c + e is visible for this row. Chunks classed uniformly over this warp's
+                    // rows (the bounds grow with the row) skip the per-row test: wholly hidden
+                    // below the first row's lower bound or above the last row's upper bound, wholly
+                    // visible inside [last row's lower bound, first row's upper bound]. The max and
+                    // the exponentials then run unmasked (2^-inf = 0).
+                    {
+                        const int lo_first = q_start + r0 - window + 1 - kv0, lo_last = lo_first + 31;
+                        const int hi_first = q_start + r0 - kv0, hi_last = hi_first + 31;
+                        uint32_t vis[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int lo = 32 * c, hi = lo + 31;
+                            const int a = c_lo - lo, b = c_hi - lo;  // visible e in [a, b]
+                            const uint32_t below = a <= 0 ? 0u : (a >= 32 ? ~0u : (1u << a) - 1u);
+                            const uint32_t above = b >= 31 ? 0u : (b < 0 ? ~0u : ~((2u << b) - 1u));
+                            vis[c] = (hi < lo_first || lo > hi_last) ? 0u
+                                     : (lo >= lo_last && hi <= hi_first) ? ~0u : ~(below | above);
                         }
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                v[32 * c + e] = ((vis[c] >> e) & 1u) ? v[32 * c + e]
+                                                                     : __float_as_uint(-INFINITY);
                     }
+                    // row max over the visible columns
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        mx = fmaxf(mx, chunk_max<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi));
                     const float m_new = fmaxf(m, mx * scale_log2);
                     // Keep the reference max until the row max grows by more than 8 (a factor
                     // 256): O / l and the lse are exact for any reference value.
@@ -371,29 +406,16 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                     if (rescale) m = m_new;
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
                     const uint64_t negm2 = f32x2(neg_m, neg_m);
-                    // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first half of S
-                    uint64_t sum2 = f32x2(0.f, 0.f);
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        const int cls = chunk_class(c);
-                        uint32_t pk[16];
-                        if (cls == 4) {
+                    // P = 2^(s * scale * log2e - m) as bf16 into the first half of S (the whole
+                    // row is in registers already)
+                    uint64_t sum_a = f32x2(0.f, 0.f), sum_b = f32x2(0.f, 0.f);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                        } else {
-                            uint32_t v[32];
-                            tmem_ld32(tm_s + 32 * c, v);
-                            tmem_wait_ld();
-                            regs_after_wait(v);
-                            switch (cls) {
-                                case kMaskNone: sum2 = row_exp32<kMaskNone>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                                case kMaskLo: sum2 = row_exp32<kMaskLo>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                                case kMaskHi: sum2 = row_exp32<kMaskHi>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                                default: sum2 = row_exp32<kMaskBoth>(v, 32 * c, c_lo, c_hi, scale2, negm2, sum2, pk); break;
-                            }
-                        }
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pk[16];
+                        chunk_exp<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
                         tmem_st16(tm_s + 16 * c, pk);
                     }
+                    const uint64_t sum2 = add_f32x2(sum_a, sum_b);
                     float s_lo, s_hi;
                     f32x2_split(sum2, s_lo, s_hi);
                     l = l * alpha + (s_lo + s_hi);
@@ -432,20 +454,24 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                 auto unit_addr = [&](int r, int u) -> uint8_t* {
                     return slot_base + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4);
                 };
-#pragma unroll 1
-                for (int c = 0; c < HD / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tm_o + 32 * c, v);
-                    tmem_wait_ld();
-                    regs_after_wait(v);
+                {
+                    uint32_t ov[HD];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 w4 = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv_l, __uint_as_float(v[8 * q4 + 1]) * inv_l),
-                            pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv_l, __uint_as_float(v[8 * q4 + 3]) * inv_l),
-                            pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv_l, __uint_as_float(v[8 * q4 + 5]) * inv_l),
-                            pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv_l, __uint_as_float(v[8 * q4 + 7]) * inv_l));
-                        *reinterpret_cast<uint4*>(unit_addr(row, 4 * c + q4)) = w4;
+                    for (int c = 0; c < HD / 32; ++c) tmem_ld32(tm_o + 32 * c, ov + 32 * c);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        regs_after_wait(ov + 32 * c);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint32_t* w8 = ov + 32 * c + 8 * q4;
+                            const uint4 w4 = make_uint4(
+                                pack_bf16x2(__uint_as_float(w8[0]) * inv_l, __uint_as_float(w8[1]) * inv_l),
+                                pack_bf16x2(__uint_as_float(w8[2]) * inv_l, __uint_as_float(w8[3]) * inv_l),
+                                pack_bf16x2(__uint_as_float(w8[4]) * inv_l, __uint_as_float(w8[5]) * inv_l),
+                                pack_bf16x2(__uint_as_float(w8[6]) * inv_l, __uint_as_float(w8[7]) * inv_l));
+                            *reinterpret_cast<uint4*>(unit_addr(row, 4 * c + q4)) = w4;
+                        }
                     }
                 }
                 if (r0 + 31 < nr) {

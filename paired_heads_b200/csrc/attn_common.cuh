@@ -36,6 +36,7 @@ struct TcBars {
     uint64_t q_full[3], q_empty[3];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2], pv_done[2], o_ready[2];
+    uint64_t s_free[2];                // hd 64: the softmax has read S_r into registers
     uint64_t v8_full[2], v8_empty[2];  // FP8: the e4m3 V staging ring
     uint64_t v_add[4];                 // value embedding: aux_v added to the landed V tile
     uint64_t drain;

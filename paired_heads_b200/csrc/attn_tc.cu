@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&bars->o_ready[r], 1);
             mbar_init(&bars->v8_full[r], 1);
             mbar_init(&bars->v8_empty[r], 64);
+            mbar_init(&bars->s_free[r], 128);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -360,13 +361,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t qc = 0;    // Q sub-tiles of the items before the current one
             uint32_t g = 0;     // global index of the current key tile (the K / V ring position)
             uint32_t p_cnt[2] = {0, 0};         // P.V products issued per sub-tile
+            uint32_t s_cnt[2] = {0, 0};         // S products issued per sub-tile
             bool pv_open[2] = {false, false};   // hd 128: the last P.V of r not yet seen complete
             // the key tile g - 1 as sub-tile r used it: its S was issued, its P.V not yet
             bool pend[2] = {false, false}, pend_first[2] = {false, false}, pend_last[2] = {false, false};
             bool ok = true;
 
-            // O_r += P_r V_{g-1} for a pending sub-tile (V_{g-1} has landed)
-            auto issue_pv = [&](int r) -> bool {
+            // O_r += P_r V_{g-1} (V_{g-1} has landed); first: the sub-tile's first key tile of its
+            // item (O starts from zero), last: its last one (O is complete afterwards)
+            auto issue_pv = [&](int r, bool first, bool last) -> bool {
                 if (!mbar_wait(&bars->p_full[r], p_cnt[r] & 1, abort_flag, dev_status)) return false;
                 tc_fence_after();
                 const uint32_t v_tile = sbase + L::kOffV + ((g - 1) % L::kVStages) * L::kV;
@@ -374,12 +377,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk)
                     umma_f16_ts(tmem + L::kTmO + HD * r, a_p + 8 * kk, desc_v(v_tile, kk), idesc_pv,
-                                (!pend_first[r] || kk > 0) ? 1u : 0u);
-                if (!kSepP) umma_commit(&bars->pv_done[r]);
-                if (pend_last[r]) umma_commit(&bars->o_ready[r]);
+                                (!first || kk > 0) ? 1u : 0u);
+                umma_commit(&bars->pv_done[r]);
+                if (last) umma_commit(&bars->o_ready[r]);
                 ++p_cnt[r];
                 pv_open[r] = !kSepP;
-                pend[r] = false;
                 return true;
             };
             auto wait_v_prev = [&]() -> bool {
@@ -411,7 +413,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // the producer may be waiting for before it loads this tile
                     if (t == 0) {
                         for (int r = 0; r < 2 && ok; ++r)
-                            if (pend[r]) ok = issue_pv(r);
+                            if (pend[r]) {
+                                ok = issue_pv(r, pend_first[r], pend_last[r]);
+                                pend[r] = false;
+                            }
                         if (!ok) break;
                     }
                     const uint32_t sk = g % L::kKStages;
@@ -420,15 +425,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         break;
                     }
                     const uint32_t k_tile = sbase + L::kOffK + sk * L::kK;
+                    // the P.V products of tile g - 1 still to issue (hd 64: after both S of tile g)
+                    bool pv_now[2] = {false, false}, pv_first[2], pv_last[2];
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
-                        if (pend[r] && !issue_pv(r)) {
-                            ok = false;
-                            break;
+                        pv_now[r] = pend[r];
+                        pv_first[r] = pend_first[r];
+                        pv_last[r] = pend_last[r];
+                        pend[r] = false;
+                        if (!kSepP && pv_now[r]) {
+                            if (!issue_pv(r, pv_first[r], pv_last[r])) {
+                                ok = false;
+                                break;
+                            }
+                            pv_now[r] = false;
                         }
                         if (t < it.t_first[r] || t > it.t_last[r]) continue;
-                        // S_r overwrites the columns that P_r of hd 128 shares with it
-                        if (pv_open[r]) {
+                        if (kSepP) {
+                            // hd 64: S_r is free once the softmax has read its last tile
+                            if (s_cnt[r] > 0 && !mbar_wait(&bars->s_free[r], (s_cnt[r] - 1) & 1,
+                                                           abort_flag, dev_status)) {
+                                ok = false;
+                                break;
+                            }
+                        } else if (pv_open[r]) {
+                            // hd 128: S_r overwrites the columns that P_r shares with it
                             if (!mbar_wait(&bars->pv_done[r], (p_cnt[r] - 1) & 1, abort_flag,
                                            dev_status)) {
                                 ok = false;
@@ -456,11 +477,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                         umma_commit(&bars->s_full[r]);
                         if (t == it.t_last[r]) umma_commit(&bars->q_empty[q_slot[r]]);
+                        ++s_cnt[r];
                         pend[r] = true;
                         pend_first[r] = t == it.t_first[r];
                         pend_last[r] = t == it.t_last[r];
                     }
                     if (!ok) break;
+                    if (kSepP) {
+                        for (int r = 0; r < 2 && ok; ++r)
+                            if (pv_now[r]) ok = issue_pv(r, pv_first[r], pv_last[r]);
+                        if (!ok) break;
+                    }
                     if (g > 0) umma_commit(&bars->v_empty[(g - 1) % L::kVStages]);
                     umma_commit(&bars->k_empty[sk]);
                 }
@@ -470,7 +497,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (ok && g > 0) {
                 ok = wait_v_prev();
                 for (int r = 0; r < 2 && ok; ++r)
-                    if (pend[r]) ok = issue_pv(r);
+                    if (pend[r]) ok = issue_pv(r, pend_first[r], pend_last[r]);
                 if (ok) umma_commit(&bars->v_empty[(g - 1) % L::kVStages]);
             }
             // Wait (bounded) until every MMA this thread issued has finished.
@@ -492,6 +519,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint64_t scale2 = f32x2(scale_log2, scale_log2);
         const int window = p.window;
         uint32_t s_cnt = 0, o_cnt = 0;
+        uint32_t pv_seen = 0;  // hd 64: P.V completions of this sub-tile awaited so far
         uint32_t q_seq = 0;  // index of the current item's first Q sub-tile in this CTA's stream
         bool ok = true;
         ItemWalk wk;
@@ -529,35 +557,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) regs_after_wait(v + 32 * c);
+                if (kSepP) {
+                    // S_r may be overwritten by the next tile's product from here on
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free[r]);
+                }
                 const int c_lo = j_min - kv0, c_hi = j_max - kv0;
-                // Masked tiles are processed in 32-column chunks classed uniformly over this
-                // warp's 32 rows [r0, r0 + 31]: the row bounds c_lo(row), c_hi(row) grow with the
-                // row, so a chunk is skipped when it lies below the first row's c_lo or above the
-                // last row's c_hi, needs no mask when it lies wholly inside [last row's c_lo,
-                // first row's c_hi], and is masked otherwise. Skipped chunks cost no exponentials
-                // and give P = 0.
+                // Masked tiles: the hidden scores are set to -inf in place, per 32-column chunk
+                // classed uniformly over this warp's 32 rows [r0, r0 + 31]. The row bounds c_lo(row),
+                // c_hi(row) grow with the row, so a chunk is wholly hidden when it lies below the
+                // first row's c_lo or above the last row's c_hi, needs no mask when it lies wholly
+                // inside [last row's c_lo, first row's c_hi], and is masked element by element
+                // otherwise. The max and the exponentials then run unmasked (2^-inf = 0).
                 const bool full_tile = (tile_jmin <= kv0) && (kv0 + kBlockN - 1 <= tile_jmax);
-                const int lo_first = window > 0 ? qr0 + r0 - window + 1 - kv0 : INT32_MIN / 2;
-                const int lo_last = window > 0 ? lo_first + 31 : INT32_MIN / 2;
-                const int hi_first = (p.causal ? min(qr0 + r0, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
-                const int hi_last = (p.causal ? min(qr0 + r0 + 31, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
-                int cls[4];  // 0 = skip, 1 = no mask, 2 = masked
+                if (!full_tile) {
+                    // bit e of vis[c]: column 32 c + e visible for this row; chunks wholly visible or
+                    // wholly hidden for every row of the warp need no per-row test
+                    const int lo_first = window > 0 ? qr0 + r0 - window + 1 - kv0 : INT32_MIN / 2;
+                    const int lo_last = window > 0 ? lo_first + 31 : INT32_MIN / 2;
+                    const int hi_first = (p.causal ? min(qr0 + r0, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
+                    const int hi_last = (p.causal ? min(qr0 + r0 + 31, it.kv_hi - 1) : it.kv_hi - 1) - kv0;
+                    uint32_t vis[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int lo = 32 * c, hi = lo + 31;
-                    cls[c] = full_tile ? 1
-                             : (hi < lo_first || lo > hi_last) ? 0
-                             : (lo >= lo_last && hi <= hi_first) ? 1 : 2;
+                    for (int c = 0; c < 4; ++c) {
+                        const int lo = 32 * c, hi = lo + 31;
+                        const int a = c_lo - lo, b = c_hi - lo;  // visible e in [a, b]
+                        const uint32_t below = a <= 0 ? 0u : (a >= 32 ? ~0u : (1u << a) - 1u);
+                        const uint32_t above = b >= 31 ? 0u : (b < 0 ? ~0u : ~((2u << b) - 1u));
+                        vis[c] = (hi < lo_first || lo > hi_last) ? 0u
+                                 : (lo >= lo_last && hi <= hi_first) ? ~0u : ~(below | above);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            v[32 * c + e] = ((vis[c] >> e) & 1u) ? v[32 * c + e] : __float_as_uint(-INFINITY);
                 }
                 // row max over the visible columns
                 float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    if (cls[c] == 1)
-                        mx = fmaxf(mx, chunk_max<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi));
-                    else if (cls[c] == 2)
-                        mx = fmaxf(mx, chunk_max<kMaskBoth>(v + 32 * c, 32 * c, c_lo, c_hi));
-                }
+                for (int c = 0; c < 4; ++c)
+                    mx = fmaxf(mx, chunk_max<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi));
                 const float m_new = fmaxf(m, mx * scale_log2);
                 // Keep the reference max until the row max grows by more than 8 (a factor 256):
                 // O / l and the lse are exact for any reference value.
@@ -566,22 +606,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (rescale) m = m_new;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const uint64_t negm2 = f32x2(neg_m, neg_m);
-                // P = 2^(s * scale * log2e - m) as bf16 (written after the whole row was read, so
-                // it may share the columns of S)
+                // P = 2^(s * scale * log2e - m) (written after the whole row was read, so it may
+                // share the columns of S)
                 uint64_t sum_a = f32x2(0.f, 0.f), sum_b = f32x2(0.f, 0.f);
+                uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
-                    if (cls[c] == 1) {
-                        chunk_exp<kMaskNone, F8>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
-                    } else if (cls[c] == 2) {
-                        chunk_exp<kMaskBoth, F8>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    chunk_exp<kMaskNone, F8>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b,
+                                             pk + 16 * (c & 1));
+                    if (c == 1 && kSepP && pv_seen < s_cnt - 1) {
+                        // hd 64: the last P.V of this sub-tile reads P_r and adds into O_r; it must be
+                        // complete before P_r is overwritten and O_r rescaled
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done[r], pv_seen & 1,
+                                                               abort_flag, dev_status));
+                        ++pv_seen;
+                        tc_fence_after();
                     }
-                    tmem_st16(tm_p + 16 * c, pk);
+                    if (c & 1) {
+                        tmem_st16(tm_p + 16 * (c - 1), pk);
+                        tmem_st16(tm_p + 16 * c, pk + 16);
+                    }
                 }
+                if (!ok) break;
                 const uint64_t sum2 = add_f32x2(sum_a, sum_b);
                 float s_lo, s_hi;
                 f32x2_split(sum2, s_lo, s_hi);

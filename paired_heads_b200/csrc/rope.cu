@@ -168,8 +168,8 @@ struct Chunk16<float> {
 // One warp per token. The token's q row (n_heads * head_dim contiguous elements) followed by its
 // k row is cut into 16-byte chunks; lane l takes chunks l, l + 32, ... in batches of kBatch, so
 // every load instruction of the warp reads 512 contiguous bytes and each lane keeps kBatch x 16
-// bytes of HBM reads in flight. All heads of the token share its table row, which is read from
-// HBM once and then served from L1.
+// bytes of HBM reads in flight; the first batch is issued before the position is known. All heads
+// of the token share its table row, which is read from HBM once and then served from L1.
 constexpr int kRopeBatch = 4;
 
 // NORM: each head row is first RMS-normalised over head_dim in float32 ("Training an LLM from
@@ -203,10 +203,18 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
     const int64_t warp0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t t = warp0; t < total_tokens; t += n_warps) {
-        const int pos = __ldg(positions + t);
-        const bool in_range = pos >= 0 && pos < tab_rows;
         uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
         uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
+        // the first batch of the token's q / k chunks does not depend on its position: its loads
+        // go out before the position and table loads, so the two latencies overlap
+        uint4 raw[kRopeBatch];
+#pragma unroll
+        for (int j = 0; j < kRopeBatch; ++j) {
+            const int i = 32 * j + lane;
+            if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
+        }
+        const int pos = __ldg(positions + t);
+        const bool in_range = pos >= 0 && pos < tab_rows;
         const float* crow = cos_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
         const float* srow = sin_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
         // When cph divides 32 (and, paired, 32/cph is even so the head parity is fixed too), every
@@ -241,11 +249,12 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
             }
         }
         for (int base = 0; base < n_chunks; base += 32 * kRopeBatch) {
-            uint4 raw[kRopeBatch];
+            if (base > 0) {
 #pragma unroll
-            for (int j = 0; j < kRopeBatch; ++j) {
-                const int i = base + 32 * j + lane;
-                if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
+                for (int j = 0; j < kRopeBatch; ++j) {
+                    const int i = base + 32 * j + lane;
+                    if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
+                }
             }
             float inv[kRopeBatch];
             if (NORM) {
