@@ -377,28 +377,6 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
     return d;
 }
 
-// Two base-2 exponentials on the FMA pipe (no special-function unit): x = n + f with
-// n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low mantissa bits), f in [-0.5, 0.5];
-// 2^f from a degree-3 polynomial fitted to 2^f on [-0.5, 0.5] in relative error (coefficients from
-// exp2_poly_fit.py; max relative error 7.5e-5), and n added to the exponent field. Inputs below
-// -126 (including -inf) are clamped there, giving a value < 2^-125 in place of 0.
-__device__ __forceinline__ void ex2_poly2(float xa, float xb, float& ya, float& yb) {
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    const uint64_t x2 = f32x2(fmaxf(xa, -126.0f), fmaxf(xb, -126.0f));
-    const uint64_t j2 = add_f32x2(x2, f32x2(kShift, kShift));
-    const uint64_t n2 = add_f32x2(j2, f32x2(-kShift, -kShift));
-    const uint64_t f2 = fma_f32x2(n2, f32x2(-1.0f, -1.0f), x2);
-    uint64_t p2 = fma_f32x2(f2, f32x2(0.055170975625514984f, 0.055170975625514984f),
-                            f32x2(0.24260970950126648f, 0.24260970950126648f));
-    p2 = fma_f32x2(p2, f2, f32x2(0.6932609677314758f, 0.6932609677314758f));
-    p2 = fma_f32x2(p2, f2, f32x2(0.9999281764030457f, 0.9999281764030457f));
-    float ja, jb, pa, pb;
-    f32x2_split(j2, ja, jb);
-    f32x2_split(p2, pa, pb);
-    ya = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ja) << 23));
-    yb = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(jb) << 23));
-}
-
 // Two e4m3 values (low byte -> low half) to two f16 values, exactly (every e4m3 value is an f16
 // value).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
