@@ -334,6 +334,18 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
         const int window = p.window;
         uint32_t s_cnt = 0, o_cnt = 0, qn = 0;
         bool ok = true;
+        // Q slot whose rows this warp's TMA stores are still reading (-1: none); released once
+        // the stores have read it, at the warpgroup's next tile or at the end
+        int pending_slot = -1;
+        auto release_pending = [&]() {
+            if (pending_slot < 0) return;
+            if (lane == 0) {
+                tma_store_wait_read();
+                mbar_arrive(&bars->q_empty[pending_slot]);
+            }
+            __syncwarp();
+            pending_slot = -1;
+        };
         if (p.test_stall_us > 0)  // the wait runs out: status 3, and every role winds down
             ok = __all_sync(0xffffffffu, mbar_wait(&bars->stall, 0, abort_flag, dev_status,
                                                    1000ull * static_cast<uint64_t>(p.test_stall_us)));
@@ -344,6 +356,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
             const uint32_t qn_item = qn;
             qn += it.n_qt;
             for (int u = static_cast<int>((qn_item ^ w) & 1); u < it.n_qt; u += 2) {
+                release_pending();
                 const uint32_t n = qn_item + u;
                 const int q_start = it.q0 + kBlockM * u;
                 const int nr = min(kBlockM, it.doc_end - q_start);
@@ -482,9 +495,10 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                             tma_store_2d(&tm_out, it.head * HD + 64 * c, q_start + r0,
                                          slot_base + c * L::kChunk + r0 * 128);
                         tma_store_commit();
-                        tma_store_wait_read();  // the slot may be refilled once the rows are read
                     }
-                    __syncwarp();
+                    // the slot may be refilled once the stores have read the rows: released at
+                    // this warpgroup's next tile, off this tile's critical path
+                    pending_slot = static_cast<int>(n % L::kQSlots);
                 } else {
                     __syncwarp();
                     constexpr int kChunks = HD / 8;  // 16-byte units per row
@@ -503,13 +517,14 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                     }
                     __syncwarp();
                     fence_proxy_async_smem();  // the slot's next fill is written by the async proxy
+                    if (lane == 0) mbar_arrive(&bars->q_empty[n % L::kQSlots]);
                 }
-                if (lane == 0) mbar_arrive(&bars->q_empty[n % L::kQSlots]);
                 tc_fence_before();
                 if (row < nr && p.lse)
                     p.lse[static_cast<int64_t>(i) * H + it.head] = (m + log2f(l)) * kLn2;
             }
         }
+        if (ok) release_pending();
     }
 
     // ---------------------------------------------------------------- teardown
