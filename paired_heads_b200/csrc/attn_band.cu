@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
+    grid_dep_wait();  // the work list (written by the scheduler kernel) is complete from here on
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads;
     const int G = p.heads / p.kv_heads;
@@ -548,9 +549,18 @@ static cudaError_t launch_band_hd(const AttnProblem& p, const CUtensorMap& tq,
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    attn_band_kernel<HD, AUXV><<<sms, AUXV ? kBandAuxThreads : kBandThreads, L::kSmemBytes, stream>>>(
-        tq, tk, tv, to, p, items, hdr);
-    return cudaGetLastError();
+    // programmatic stream serialization: the prologue overlaps the scheduler kernel before it
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(AUXV ? kBandAuxThreads : kBandThreads);
+    cfg.dynamicSmemBytes = L::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_band_kernel<HD, AUXV>, tq, tk, tv, to, p, items, hdr);
 }
 
 cudaError_t launch_attn_band(const AttnProblem& p, const CUtensorMap& tm_q,

@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
+    grid_dep_wait();  // the work list (written by the scheduler kernel) is complete from here on
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads;
     const int G = p.heads / p.kv_heads;
@@ -737,8 +738,18 @@ static cudaError_t launch_tc_hd(const AttnProblem& p, const CUtensorMap& tq, con
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    attn_tc_kernel<HD, F8, AUXV><<<sms, kTcThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p, items, hdr);
-    return cudaGetLastError();
+    // programmatic stream serialization: the prologue overlaps the scheduler kernel before it
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = L::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel<HD, F8, AUXV>, tq, tk, tv, p, items, hdr);
 }
 
 cudaError_t launch_attn_tc(const AttnProblem& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,

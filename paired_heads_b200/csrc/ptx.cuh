@@ -324,6 +324,19 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Wait until the grids this one depends on (launched before it on the stream) have completed and
+// their memory is visible. A no-op when the kernel was launched without the programmatic
+// stream-serialization attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel on the stream, if launched with programmatic stream serialization, start
+// its launch now (it waits in grid_dep_wait for this grid's completion before using its results).
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ register split
 
 // Raise / lower this warpgroup's per-thread register allocation (all 128 threads execute it).

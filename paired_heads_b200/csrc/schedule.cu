@@ -102,6 +102,9 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     __shared__ int hist[kMaxCostBuckets];
     __shared__ int warp_sums[kSchedThreads / 32];
     __shared__ int bad;
+    // the attention kernel may start its prologue (barriers, tensor memory, descriptor prefetch)
+    // now; it waits for this grid's completion before it reads the work list
+    grid_dep_launch();
     const int tid = threadIdx.x;
     const int64_t mult = p.slot_mult;
     const int rows = band ? kBandRows : kItemRows;
