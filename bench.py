@@ -431,10 +431,15 @@ def main():
     ab = attn_bytes(w) + (float(w.total * w.n_kv_heads * w.head_dim * 2) if args.aux_v else 0.0)
     kernels = {
         rname: {"ms": rope_ms, "bytes": rope_bytes(w, tab_width),
-                 "gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9},
+                 "gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9,
+                 "frac_of_hbm": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                 "traffic": load_traffic(w, rname)},
         "attention": {"ms": attn_ms, "flops": flops, "bytes": ab,
                       "tflops": attn_tflops,
-                      "gbs": ab / (attn_ms * 1e-3) / 1e9},
+                      "gbs": ab / (attn_ms * 1e-3) / 1e9,
+                      "frac_of_hbm": ab / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "frac_of_bf16_peak": attn_tflops / peaks["bf16_tflops"],
+                      "traffic": load_traffic(w, "attention")},
     }
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     attn_bound = "hbm" if flops / ab < ridge else "tensor"
