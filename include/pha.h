@@ -219,10 +219,11 @@ pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* s
                         int stagger_offset, pha_stream_t stream);
 
 /*
- * pha_attn_bwd_workspace_bytes -- device scratch pha_attn_bwd needs: the forward's scheduling
- *   area (pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired), rounded up to 256
- *   bytes; its header is what pha_attn_status reads) followed by float[total_tokens][n_heads]
- *   (the row sums D_i), rounded up to 256 bytes. 0 for invalid arguments.
+ * pha_attn_bwd_workspace_bytes -- device scratch pha_attn_bwd needs: a scheduling area (a 256-byte
+ *   header, which pha_attn_status reads, int32[batch + 1] padded to 16 bytes, and 16 bytes for
+ *   each of at most batch * ceil(L/128) * H' (128-slot tile, head) work items, L and H' as for
+ *   pha_attn_workspace_bytes; rounded up to 256 bytes) followed by float[total_tokens][n_heads]
+ *   (the row sums D_i), rounded up to 256 bytes. head_dim does not enter. 0 for invalid arguments.
  */
 size_t pha_attn_bwd_workspace_bytes(int batch, int max_len, int total_tokens, int n_heads,
                                     int head_dim, int paired);
@@ -242,10 +243,10 @@ size_t pha_attn_bwd_workspace_bytes(int batch, int max_len, int total_tokens, in
  *   document get zeros). workspace: at least pha_attn_bwd_workspace_bytes(...), 16-byte aligned;
  *   pha_attn_status(workspace) reports the device status afterwards (malformed cu_seqlens, a
  *   kernel wait that gave up).
- *   Arithmetic: bf16 with causal 1 <= window <= 128 and head_dim 64 or 128 (the band case): the
- *   tensor cores (tcgen05, bf16 operands with P and dS rounded to bf16, float32 accumulation in
- *   TMEM), one kernel for dq and one for dk, dv; otherwise float32 on CUDA cores (dtype bf16 or
- *   f32, head_dim <= 128). No atomics on either path.
+ *   Arithmetic: bf16 with head_dim 64 or 128: the tensor cores (tcgen05, bf16 operands with P and
+ *   dS rounded to bf16, float32 accumulation in TMEM), one kernel for dq and one for dk, dv (band
+ *   work lists for causal windows <= 128, per-tile work lists otherwise); other head_dims and f32
+ *   run in float32 on CUDA cores (head_dim <= 128). No atomics on any path.
  *   Errors: as pha_attn_fwd (PHA_ERR_INVALID, PHA_ERR_UNSUPPORTED for head_dim > 128 and for
  *   non-causal windows, PHA_ERR_WORKSPACE); o or lse NULL with total_tokens > 0: PHA_ERR_INVALID.
  *   With total_tokens == 0 the call returns PHA_OK after checking its arguments, launching nothing.

@@ -80,17 +80,49 @@ struct BwdBars {
     int abort;
 };
 
-// The steps of one outer tile (u-th tile of a band item).
+// The steps of one outer tile (u-th tile of a band item, or the tile of a tile item).
 struct OuterTile {
     int row0;     // first slot of the outer tile
     int n_sub;    // inner steps
-    int nq;       // key-major: query tiles per head (1 or 2)
+    int nq;       // key-major: query tiles per head (band: 1 or 2)
+    int first;    // GEN: document tile index of the first inner step's Y tile
 };
 
-template <bool KEYMAJOR>
-__device__ __forceinline__ OuterTile outer_tile(const BandItem& it, int u, int G) {
+// GEN (tile items, any causal / window setting): query-major, the key tiles the query tile sees;
+// key-major, the query tiles that see the key tile, for every query head of its group. Tiles are
+// the document's 128-slot tiles counted from its start.
+template <bool KEYMAJOR, bool GEN>
+__device__ __forceinline__ OuterTile outer_tile(const BandItem& it, int u, int G,
+                                                const AttnProblem& p) {
     OuterTile o;
     o.row0 = it.q0 + kBlockM * u;
+    o.first = 0;
+    if (GEN) {
+        const int a = it.doc_start, b = it.doc_end;
+        const int j = (o.row0 - a) / kBlockN, last = (b - a - 1) / kBlockN;
+        int lo = 0, hi = last;
+        if (!KEYMAJOR) {
+            if (p.causal) {
+                hi = j;
+                if (p.window > 0 && o.row0 - p.window + 1 > a) lo = (o.row0 - p.window + 1 - a) / kBlockN;
+            }
+            o.nq = 0;
+            o.n_sub = hi - lo + 1;
+        } else {
+            if (p.causal) {
+                lo = j;
+                if (p.window > 0) {
+                    const int n_rows = min(kBlockM, b - o.row0);
+                    const int q_last = o.row0 + n_rows - 1 + p.window - 1;
+                    hi = ((q_last < b ? q_last : b - 1) - a) / kBlockN;
+                }
+            }
+            o.nq = hi - lo + 1;
+            o.n_sub = G * o.nq;
+        }
+        o.first = lo;
+        return o;
+    }
     if (KEYMAJOR) {
         o.nq = o.row0 + kBlockM < it.doc_end ? 2 : 1;  // the diagonal query tile, then the next
         o.n_sub = G * o.nq;
@@ -102,9 +134,19 @@ __device__ __forceinline__ OuterTile outer_tile(const BandItem& it, int u, int G
 }
 
 // Inner step s of an outer tile: the head and first slot of its Y tiles.
-template <bool KEYMAJOR>
+template <bool KEYMAJOR, bool GEN>
 __device__ __forceinline__ void inner_step(const BandItem& it, const OuterTile& o, int s, int G,
                                            int& y_head, int& y_row) {
+    if (GEN) {
+        if (KEYMAJOR) {
+            y_head = (it.head / G) * G + s / o.nq;
+            y_row = it.doc_start + kBlockN * (o.first + s % o.nq);
+        } else {
+            y_head = it.head / G;
+            y_row = it.doc_start + kBlockN * (o.first + s);
+        }
+        return;
+    }
     if (KEYMAJOR) {
         const int g = it.head / G;
         y_head = g * G + s / o.nq;
@@ -160,7 +202,7 @@ struct FillTrack {
     }
 };
 
-template <int HD, bool KEYMAJOR>
+template <int HD, bool KEYMAJOR, bool GEN>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -222,7 +264,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads, Hkv = p.kv_heads, G = H / Hkv;
-    const bool reuse = !KEYMAJOR || G == 1;
+    const bool reuse = !GEN && (!KEYMAJOR || G == 1);
     // X = (K, V) and Y = (Q, dO) (key-major), or the other way round
     const CUtensorMap* mx0 = KEYMAJOR ? &tm_k : &tm_q;
     const CUtensorMap* mx1 = KEYMAJOR ? &tm_v : &tm_do;
@@ -242,7 +284,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                                    abort_flag, dev_status)))
                 return false;
             int y_head, y_row;
-            inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
+            inner_step<KEYMAJOR, GEN>(it, o, s, G, y_head, y_row);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars->y_full[st], 2 * L::kTile);
                 uint8_t* y = smem + L::kOffY + st * 2 * L::kTile;
@@ -274,7 +316,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             if (!item_used<KEYMAJOR>(it, G)) continue;
             const int x_head = KEYMAJOR ? it.head / G : it.head;
             for (int u = 0; ok && u < it.n_qt; ++u) {
-                const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                const OuterTile o = outer_tile<KEYMAJOR, GEN>(it, u, G, p);
                 for (int s = 0; ok && reuse && s < o.n_sub; ++s) {
                     const StepFill f = ft.step(true, u, it.n_qt, s, o.n_sub);
                     if (f.first) ok = load_y(it, o, s, f.idx);
@@ -322,7 +364,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 const BandItem it = decode_band(wk.cur);
                 if (!item_used<KEYMAJOR>(it, G)) continue;
                 for (int u = 0; ok && u < it.n_qt; ++u) {
-                    const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                    const OuterTile o = outer_tile<KEYMAJOR, GEN>(it, u, G, p);
                     if (!mbar_wait(&bars->x_full, oc & 1, abort_flag, dev_status)) {
                         ok = false;
                         break;
@@ -406,7 +448,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             const BandItem it = decode_band(wk.cur);
             if (!item_used<KEYMAJOR>(it, G)) continue;
             for (int u = 0; ok && u < it.n_qt; ++u) {
-                const OuterTile o = outer_tile<KEYMAJOR>(it, u, G);
+                const OuterTile o = outer_tile<KEYMAJOR, GEN>(it, u, G, p);
                 const int slot = o.row0 + row;  // key slot (key-major) or query slot
                 const bool valid = slot < it.doc_end;
                 float lse2 = 0.f, dd = 0.f;  // query-major: this row's lse * log2(e) and D
@@ -419,10 +461,20 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     const StepFill f = ft.step(reuse, u, it.n_qt, s, o.n_sub);
                     const uint32_t st = f.idx & 1;
                     int y_head, y_row;
-                    inner_step<KEYMAJOR>(it, o, s, G, y_head, y_row);
+                    inner_step<KEYMAJOR, GEN>(it, o, s, G, y_head, y_row);
                     // visible columns [c_lo, c_hi] of this row
                     int c_lo, c_hi;
-                    if (KEYMAJOR) {  // queries slot .. slot + window - 1, inside the document
+                    if (GEN) {
+                        const int a = it.doc_start, b = it.doc_end;
+                        if (KEYMAJOR) {  // the queries that see key `slot`
+                            c_lo = (p.causal ? slot : a) - y_row;
+                            c_hi = ((p.causal && window > 0) ? min(slot + window - 1, b - 1) : b - 1) - y_row;
+                        } else {         // the keys query `slot` sees
+                            c_lo = ((window > 0) ? max(a, slot - window + 1) : a) - y_row;
+                            c_hi = (p.causal ? slot : b - 1) - y_row;
+                        }
+                        if (!valid) c_hi = c_lo - 1;
+                    } else if (KEYMAJOR) {  // queries slot .. slot + window - 1, inside the document
                         c_lo = slot - y_row;
                         c_hi = min(slot + window - 1, it.doc_end - 1) - y_row;
                     } else {         // keys slot - window + 1 .. slot
@@ -601,38 +653,44 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     if (warp == 9) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-template <int HD, bool KEYMAJOR>
+template <int HD, bool KEYMAJOR, bool GEN>
 cudaError_t launch_bwd_tc_one(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
                               const CUtensorMap& tv, const CUtensorMap& tdo,
                               const CUtensorMap& tst, const CUtensorMap& tst2, const float* dsum,
                               __nv_bfloat16* out_a, __nv_bfloat16* out_b, const int4* items,
                               WorkspaceHeader* hdr, int sms, cudaStream_t stream) {
     using L = BwdLayout<HD, KEYMAJOR>;
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<HD, KEYMAJOR>,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<HD, KEYMAJOR, GEN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attn_bwd_tc_kernel<HD, KEYMAJOR><<<sms, kBwdTcThreads, L::kSmemBytes, stream>>>(
+    attn_bwd_tc_kernel<HD, KEYMAJOR, GEN><<<sms, kBwdTcThreads, L::kSmemBytes, stream>>>(
         tq, tk, tv, tdo, tst, tst2, p, dsum, out_a, out_b, items, hdr);
     return cudaGetLastError();
 }
 
-template <int HD>
+template <int HD, bool GEN>
 cudaError_t launch_bwd_tc_hd(const AttnProblem& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, const CUtensorMap& tdo,
                              const CUtensorMap& tdq, const CUtensorMap& tdk,
                              const CUtensorMap& tdv, const float* dsum,
                              void* dq, void* dk, void* dv, const int4* items, WorkspaceHeader* hdr,
-                             cudaStream_t stream) {
+                             int which, cudaStream_t stream) {
     int dev = 0, sms = 0;
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    if ((e = launch_bwd_tc_one<HD, false>(p, tq, tk, tv, tdo, tdq, tdq, dsum, static_cast<__nv_bfloat16*>(dq),
-                                          nullptr, items, hdr, sms, stream)) != cudaSuccess)
+    if ((which & 1) &&
+        (e = launch_bwd_tc_one<HD, false, GEN>(p, tq, tk, tv, tdo, tdq, tdq, dsum,
+                                               static_cast<__nv_bfloat16*>(dq), nullptr, items, hdr,
+                                               sms, stream)) != cudaSuccess)
         return e;
-    return launch_bwd_tc_one<HD, true>(p, tq, tk, tv, tdo, tdk, tdv, dsum, static_cast<__nv_bfloat16*>(dk),
-                                       static_cast<__nv_bfloat16*>(dv), items, hdr, sms, stream);
+    if (which & 2)
+        return launch_bwd_tc_one<HD, true, GEN>(p, tq, tk, tv, tdo, tdk, tdv, dsum,
+                                                static_cast<__nv_bfloat16*>(dk),
+                                                static_cast<__nv_bfloat16*>(dv), items, hdr, sms,
+                                                stream);
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -642,14 +700,18 @@ cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
                                const CUtensorMap& tm_do, const CUtensorMap& tm_dq,
                                const CUtensorMap& tm_dk, const CUtensorMap& tm_dv,
                                const float* dsum, void* dq, void* dk, void* dv, const int4* items,
-                               WorkspaceHeader* hdr, cudaStream_t stream) {
-    if (!band_applies(p)) return cudaErrorInvalidValue;
+                               WorkspaceHeader* hdr, int which, cudaStream_t stream) {
+    const bool band = band_applies(p);
     if (p.head_dim == 128)
-        return launch_bwd_tc_hd<128>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq, dk, dv, items, hdr,
-                                     stream);
+        return band ? launch_bwd_tc_hd<128, false>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq,
+                                                   dk, dv, items, hdr, which, stream)
+                    : launch_bwd_tc_hd<128, true>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq,
+                                                  dk, dv, items, hdr, which, stream);
     if (p.head_dim == 64)
-        return launch_bwd_tc_hd<64>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq, dk, dv, items, hdr,
-                                    stream);
+        return band ? launch_bwd_tc_hd<64, false>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq,
+                                                  dk, dv, items, hdr, which, stream)
+                    : launch_bwd_tc_hd<64, true>(p, tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, dsum, dq,
+                                                 dk, dv, items, hdr, which, stream);
     return cudaErrorInvalidValue;
 }
 

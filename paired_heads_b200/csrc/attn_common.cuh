@@ -229,7 +229,7 @@ __device__ __forceinline__ void add_aux_tile(uint8_t* tile, const __nv_bfloat16*
 
 // Band work item (see kernels.cuh), decoded.
 struct BandItem {
-    int q0, n_qt, hp, head, doc_end;
+    int q0, n_qt, hp, head, doc_end, doc_start;
 };
 
 __device__ __forceinline__ BandItem decode_band(int4 w) {
@@ -239,6 +239,7 @@ __device__ __forceinline__ BandItem decode_band(int4 w) {
     it.hp = (w.y >> 15) & 1;
     it.n_qt = w.y & 0x7FFF;
     it.doc_end = w.z;
+    it.doc_start = w.w;
     return it;
 }
 

@@ -33,8 +33,15 @@ inline size_t workspace_doc_bytes(int batch) {
 //   x = first query slot, y = (head << 16) | valid query rows, z = first key slot, w = key end.
 // Keys [z, w) are streamed in tiles of kBlockN starting at z.
 // Band work item (attn_band) = a run of up to kBandTiles query tiles of one head:
-//   x = first query slot q0, y = (head << 16) | (has_prev << 15) | query tiles, z = document end.
-// Key tiles start at q0 - kBlockN (has_prev) or q0, one per step.
+//   x = first query slot q0, y = (head << 16) | (has_prev << 15) | query tiles, z = document end,
+//   w = document start. Key tiles start at q0 - kBlockN (has_prev) or q0, one per step.
+// Tile work item (the tensor-core backward outside the band case): the band item format with a
+// single tile, the 128-slot tile at q0 of one head of a document [w, z).
+
+// Work-list shapes of the scheduler: block items (attn_tc), band items (attn_band and the band
+// backward), and tile items ordered by the number of key tiles a query tile sees (dQ) or of query
+// tiles that see a key tile (dK / dV).
+enum ScheduleMode : int { kSchedBlock = 0, kSchedBand = 1, kSchedTilesQ = 2, kSchedTilesK = 3 };
 
 struct AttnProblem {
     const void* q;
@@ -94,16 +101,17 @@ cudaError_t launch_attn_bwd(const AttnProblem& p, const void* dout, const float*
 cudaError_t launch_attn_bwd_zero_outside(const AttnProblem& p, void* dq, void* dk, void* dv,
                                          cudaStream_t stream);
 
-// Backward of the band attention on the tensor cores (bf16, band_applies, head_dim 64 / 128) over
-// a band work list: the dQ kernel, then the dK / dV kernel. tm_do is a map over dout like tm_q;
-// tm_dq a map over dq like tm_q with a 64 x 32 box, tm_dk / tm_dv maps over dk / dv like tm_k
-// with a 64 x 16 box (the epilogues' TMA stores). Writes the rows inside the documents only.
+// Backward of attention on the tensor cores (bf16, head_dim 64 / 128). tm_do is a map over dout
+// like tm_q; tm_dq a map over dq like tm_q with a 64 x 32 box, tm_dk / tm_dv maps over dk / dv
+// like tm_k with a 64 x 16 box (the epilogues' TMA stores). Writes the rows inside the documents
+// only. which: 1 = the dQ kernel, 2 = the dK / dV kernel, 3 = both. Band case (band_applies):
+// band work list; otherwise tile work lists (kSchedTilesQ for dQ, kSchedTilesK for dK / dV).
 cudaError_t launch_attn_bwd_tc(const AttnProblem& p, const CUtensorMap& tm_q,
                                const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                const CUtensorMap& tm_do, const CUtensorMap& tm_dq,
                                const CUtensorMap& tm_dk, const CUtensorMap& tm_dv,
                                const float* dsum, void* dq, void* dk, void* dv, const int4* items,
-                               WorkspaceHeader* hdr, cudaStream_t stream);
+                               WorkspaceHeader* hdr, int which, cudaStream_t stream);
 
 // RoPE preceded by the QK RMS-norm of every head row (weights may be NULL = ones).
 cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const float* k_weight,
@@ -114,9 +122,9 @@ cudaError_t launch_qk_norm_rope(void* q, void* k, const float* q_weight, const f
 
 cudaError_t launch_attn_f32(const AttnProblem& p, cudaStream_t stream);
 
-// Builds the varlen work list (band items when `band`, else block items) into `items` (capacity
-// entries) and the header; doc_blocks is int32[batch + 1] scratch.
-cudaError_t launch_schedule(const AttnProblem& p, bool band, int capacity, int* doc_blocks,
+// Builds the varlen work list of the given shape into `items` (capacity entries) and the header;
+// doc_blocks is int32[batch + 1] scratch.
+cudaError_t launch_schedule(const AttnProblem& p, ScheduleMode mode, int capacity, int* doc_blocks,
                             int4* items, WorkspaceHeader* hdr, cudaStream_t stream);
 
 // tcgen05 attention over a scheduled work list. tm_q / tm_k / tm_v are 2-D bf16 tensor maps

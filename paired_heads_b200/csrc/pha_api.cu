@@ -180,14 +180,25 @@ pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* s
                : PHA_ERR_CUDA;
 }
 
+// Scheduling area of the backward: header, per-document offsets and the largest of its work
+// lists, the tile lists (one item per 128-slot tile and head), rounded up to 256 bytes.
+static size_t bwd_sched_bytes(int batch, int max_len, int n_heads, int paired) {
+    if (pha_attn_workspace_bytes(batch, max_len, n_heads, 64, paired) == 0) return 0;
+    const int64_t slots = static_cast<int64_t>(max_len) * (paired ? 2 : 1);
+    const int64_t heads = paired ? n_heads / 2 : n_heads;
+    const size_t items = static_cast<size_t>(batch) * div_up(slots, kBlockM) * heads;
+    const size_t bytes = kWorkspaceHeaderBytes + workspace_doc_bytes(batch) + items * sizeof(int4);
+    return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
 size_t pha_attn_bwd_workspace_bytes(int batch, int max_len, int total_tokens, int n_heads,
                                     int head_dim, int paired) {
+    (void)head_dim;
     if (total_tokens < 0) return 0;
-    const size_t sched = pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired);
+    const size_t sched = bwd_sched_bytes(batch, max_len, n_heads, paired);
     if (sched == 0) return 0;
-    return ((sched + 255) & ~static_cast<size_t>(255)) +
-           ((static_cast<size_t>(total_tokens) * n_heads * sizeof(float) + 255) &
-            ~static_cast<size_t>(255));
+    return sched + ((static_cast<size_t>(total_tokens) * n_heads * sizeof(float) + 255) &
+                    ~static_cast<size_t>(255));
 }
 
 pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -231,9 +242,8 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void*
     p.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(head_dim));
     p.lse = const_cast<float*>(lse);
 
-    // Workspace: the forward's scheduling area (header, document offsets, work items), then D.
-    const size_t sched = (pha_attn_workspace_bytes(batch, max_len, n_heads, head_dim, paired) + 255) &
-                         ~static_cast<size_t>(255);
+    // Workspace: the scheduling area (header, document offsets, work items), then D.
+    const size_t sched = bwd_sched_bytes(batch, max_len, n_heads, paired);
     auto* base = static_cast<uint8_t*>(workspace);
     auto* hdr = reinterpret_cast<WorkspaceHeader*>(base);
     auto* doc_blocks = reinterpret_cast<int*>(base + kWorkspaceHeaderBytes);
@@ -243,10 +253,13 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void*
     const int capacity = cap64 > 0x7FFFFFFF ? 0x7FFFFFFF : static_cast<int>(cap64);
     float* dsum = reinterpret_cast<float*>(base + sched);
 
-    // Tensor cores for the band case (bf16, causal, 1 <= window <= 128, head_dim 64 / 128);
-    // CUDA cores otherwise. The scheduler also checks cu_seqlens (pha_attn_status).
-    const bool tc = dtype == PHA_BF16 && band_applies(p) && (head_dim == 64 || head_dim == 128);
-    if (launch_schedule(p, tc, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+    // Tensor cores for bf16 with head_dim 64 / 128 (band work lists for causal windows <= 128,
+    // tile lists otherwise); CUDA cores for the rest. The scheduler also checks cu_seqlens
+    // (pha_attn_status).
+    const bool tc = dtype == PHA_BF16 && (head_dim == 64 || head_dim == 128);
+    const bool band = band_applies(p);
+    const ScheduleMode mode = !tc ? kSchedBlock : (band ? kSchedBand : kSchedTilesQ);
+    if (launch_schedule(p, mode, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
         return PHA_ERR_CUDA;
     if (launch_attn_bwd_dsum(p, o, dout, dsum, dtype == PHA_BF16, stream) != cudaSuccess)
         return PHA_ERR_CUDA;
@@ -264,10 +277,19 @@ pha_status pha_attn_bwd(const void* q, const void* k, const void* v, const void*
         !encode_slot_map(&tdk, dk, static_cast<uint64_t>(p.kv_heads) * head_dim, rows, 16) ||
         !encode_slot_map(&tdv, dv, static_cast<uint64_t>(p.kv_heads) * head_dim, rows, 16))
         return PHA_ERR_CUDA;
-    if (launch_attn_bwd_zero_outside(p, dq, dk, dv, stream) != cudaSuccess ||
-        launch_attn_bwd_tc(p, tq, tk, tv, tdo, tdq, tdk, tdv, dsum, dq, dk, dv, items, hdr,
-                           stream) !=
-            cudaSuccess)
+    if (launch_attn_bwd_zero_outside(p, dq, dk, dv, stream) != cudaSuccess) return PHA_ERR_CUDA;
+    if (band)
+        return launch_attn_bwd_tc(p, tq, tk, tv, tdo, tdq, tdk, tdv, dsum, dq, dk, dv, items, hdr, 3,
+                                  stream) == cudaSuccess
+                   ? PHA_OK
+                   : PHA_ERR_CUDA;
+    // tile lists: the dQ kernel over query tiles, then the list rebuilt over key tiles (ordered by
+    // their own cost) for the dK / dV kernel
+    if (launch_attn_bwd_tc(p, tq, tk, tv, tdo, tdq, tdk, tdv, dsum, dq, dk, dv, items, hdr, 1,
+                           stream) != cudaSuccess ||
+        launch_schedule(p, kSchedTilesK, capacity, doc_blocks, items, hdr, stream) != cudaSuccess ||
+        launch_attn_bwd_tc(p, tq, tk, tv, tdo, tdq, tdk, tdv, dsum, dq, dk, dv, items, hdr, 2,
+                           stream) != cudaSuccess)
         return PHA_ERR_CUDA;
     return PHA_OK;
 }
@@ -353,7 +375,8 @@ pha_status attn_fwd_impl(const void* q, const void* k, const void* v, const void
     // Causal windows of at most one key tile run on the band kernel, everything else on the block
     // kernel; the scheduler emits the matching item shape.
     const bool band = band_applies(p);
-    if (launch_schedule(p, band, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+    if (launch_schedule(p, band ? kSchedBand : kSchedBlock, capacity, doc_blocks, items, hdr,
+                        stream) != cudaSuccess)
         return PHA_ERR_CUDA;
     if (total_tokens == 0) return PHA_OK;
 
@@ -448,7 +471,7 @@ pha_status pha_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
     auto* doc_blocks = reinterpret_cast<int*>(base + kWorkspaceHeaderBytes);
     auto* items = reinterpret_cast<int4*>(base + fixed);
     // every window runs on the block kernel (its FP8 variant)
-    if (launch_schedule(p, false, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
+    if (launch_schedule(p, kSchedBlock, capacity, doc_blocks, items, hdr, stream) != cudaSuccess)
         return PHA_ERR_CUDA;
     if (total_tokens == 0) return PHA_OK;
     const uint64_t rows = static_cast<uint64_t>(total_tokens) * p.slot_mult;

@@ -18,6 +18,10 @@
 // and the one before it, so the run streams key tiles from q0 - 128 (q0 - 128 >= a, "has
 // previous") or q0, one per step, each shared by two consecutive query tiles.
 //
+// Tile items (the tensor-core backward outside the band case): one 128-slot tile of one document
+// and head, with the document's start; dQ lists are ordered by the key tiles the query tile sees,
+// dK / dV lists by the query tiles that see the key tile.
+//
 // Items are ordered longest first (counting sort on the number of key tiles) so that a static
 // round-robin over persistent CTAs balances; the heads of one block are adjacent so that CTAs
 // sharing a kv head (GQA) run close together in time and share K/V through L2.
@@ -68,18 +72,43 @@ struct BlockRange {
     int cost;   // key tiles streamed, clamped to the last bucket
 };
 
+__device__ __forceinline__ int mode_rows(int mode) {
+    return mode == kSchedBlock ? kItemRows : (mode == kSchedBand ? kBandRows : kBlockM);
+}
+
 __device__ __forceinline__ BlockRange block_range(const AttnProblem& p, int64_t a, int64_t b,
-                                                  int blk, int n_buckets, bool band) {
+                                                  int blk, int n_buckets, int mode) {
     BlockRange r;
-    const int rows = band ? kBandRows : kItemRows;
+    const int rows = mode_rows(mode);
     const int64_t q0 = a + static_cast<int64_t>(blk) * rows;
     const int64_t n_q = b - q0 < rows ? b - q0 : rows;
     int64_t cost;
-    if (band) {
+    if (mode == kSchedTilesQ || mode == kSchedTilesK) {
+        // tile j = blk of the document's 128-slot tiles
+        const int64_t last = (b - a - 1) / kBlockN;  // index of the document's last tile
+        int64_t lo = 0, hi = last;
+        if (mode == kSchedTilesQ) {  // key tiles this query tile sees
+            if (p.causal) {
+                hi = blk;
+                if (p.window > 0 && q0 - p.window + 1 > a) lo = (q0 - p.window + 1 - a) / kBlockN;
+            }
+        } else if (p.causal) {       // query tiles that see this key tile
+            lo = blk;
+            if (p.window > 0) {
+                // the last query that sees a key of this tile, inside the document
+                const int64_t q_last = q0 + n_q - 1 + p.window - 1;
+                hi = ((q_last < b ? q_last : b - 1) - a) / kBlockN;
+            }
+        }
+        cost = hi - lo + 1;
+        r.item = make_int4(static_cast<int>(q0), ((blk > 0 ? 1 : 0) << 15) | 1, static_cast<int>(b),
+                           static_cast<int>(a));
+    } else if (mode == kSchedBand) {
         const int n_qt = static_cast<int>((n_q + kBlockM - 1) / kBlockM);
         const int hp = blk > 0 ? 1 : 0;
         cost = n_qt + hp;
-        r.item = make_int4(static_cast<int>(q0), (hp << 15) | n_qt, static_cast<int>(b), 0);
+        r.item = make_int4(static_cast<int>(q0), (hp << 15) | n_qt, static_cast<int>(b),
+                           static_cast<int>(a));
     } else {
         int64_t lo = a, hi = b;
         if (p.causal) {
@@ -95,7 +124,7 @@ __device__ __forceinline__ BlockRange block_range(const AttnProblem& p, int64_t 
 }
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, int capacity,
-                                                                 int n_buckets, int band,
+                                                                 int n_buckets, int mode,
                                                                  int* __restrict__ doc_blocks,
                                                                  int4* __restrict__ items,
                                                                  WorkspaceHeader* hdr) {
@@ -107,7 +136,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     grid_dep_launch();
     const int tid = threadIdx.x;
     const int64_t mult = p.slot_mult;
-    const int rows = band ? kBandRows : kItemRows;
+    const int rows = mode_rows(mode);
     for (int c = tid; c < n_buckets; c += kSchedThreads) hist[c] = 0;
     if (tid == 0) bad = 0;
     __syncthreads();
@@ -165,7 +194,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     for (int g = tid; g < n_blocks; g += kSchedThreads) {
         const int d = doc_of(g);
         const BlockRange r = block_range(p, p.cu_seqlens[d] * mult, p.cu_seqlens[d + 1] * mult,
-                                         g - doc_blocks[d], n_buckets, band);
+                                         g - doc_blocks[d], n_buckets, mode);
         atomicAdd(&hist[r.cost], 1);
     }
     __syncthreads();
@@ -184,7 +213,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     for (int g = tid; g < n_blocks; g += kSchedThreads) {
         const int d = doc_of(g);
         const BlockRange r = block_range(p, p.cu_seqlens[d] * mult, p.cu_seqlens[d + 1] * mult,
-                                         g - doc_blocks[d], n_buckets, band);
+                                         g - doc_blocks[d], n_buckets, mode);
         const int slot = atomicAdd(&hist[r.cost], 1);
         int4* dst = items + static_cast<int64_t>(slot) * p.heads;
         for (int h = 0; h < p.heads; ++h)
@@ -196,17 +225,21 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     }
 }
 
-int schedule_buckets(const AttnProblem& p, bool band) {
-    if (band) return kBandTiles + 2;
+int schedule_buckets(const AttnProblem& p, int mode) {
+    if (mode == kSchedBand) return kBandTiles + 2;
+    if (mode == kSchedTilesQ || mode == kSchedTilesK) {
+        const int64_t tiles = (static_cast<int64_t>(p.max_len) * p.slot_mult + kBlockN - 1) / kBlockN + 2;
+        return static_cast<int>(tiles < kMaxCostBuckets ? tiles : kMaxCostBuckets);
+    }
     const int64_t slots = static_cast<int64_t>(p.max_len) * p.slot_mult;
     const int64_t nb = (slots + kItemRows) / kBlockN + 2;
     return static_cast<int>(nb < kMaxCostBuckets ? nb : kMaxCostBuckets);
 }
 
-cudaError_t launch_schedule(const AttnProblem& p, bool band, int capacity, int* doc_blocks,
+cudaError_t launch_schedule(const AttnProblem& p, ScheduleMode mode, int capacity, int* doc_blocks,
                             int4* items, WorkspaceHeader* hdr, cudaStream_t stream) {
-    schedule_kernel<<<1, kSchedThreads, 0, stream>>>(p, capacity, schedule_buckets(p, band),
-                                                     band ? 1 : 0, doc_blocks, items, hdr);
+    schedule_kernel<<<1, kSchedThreads, 0, stream>>>(p, capacity, schedule_buckets(p, mode),
+                                                     static_cast<int>(mode), doc_blocks, items, hdr);
     return cudaGetLastError();
 }
 

@@ -249,8 +249,8 @@ def _attn_aux(pha, **kw):
     (dict(), -3),                              # valid: only the (too small) workspace stops it
     (dict(aux=None), -1),
     (dict(aux=MIS), -1),
-    (dict(window=0), -2),                      # the band kernel only
-    (dict(window=129), -2),
+    (dict(window=0), -3),                      # the block kernel has it too: valid
+    (dict(window=129), -3),
     (dict(dtype=1), -2),
     (dict(hd=96), -2),
     (dict(H=6, Hkv=4), -1),
@@ -293,12 +293,19 @@ def test_attn_bwd_argument_errors(pha, kw, code):
 def test_attn_bwd_workspace_bytes(pha):
     def up(n):
         return (n + 255) // 256 * 256
+
+    def pad(n):
+        return (4 * (n + 1) + 15) // 16 * 16
     for batch, max_len, total, H, hd, paired in [(113, 2048, 65536, 6, 128, True),
                                                  (3, 700, 1000, 4, 64, False), (1, 0, 0, 2, 16, True)]:
         fwd = pha.pha_attn_workspace_bytes(batch, max_len, H, hd, paired)
         assert fwd > 0
+        m = 2 if paired else 1
+        tiles = -(-max_len * m // 128)                  # 128-slot tiles per document
+        sched = 256 + pad(batch) + 16 * batch * tiles * (H // m)
+        assert sched >= fwd                             # holds every work list of the forward
         assert pha.pha_attn_bwd_workspace_bytes(batch, max_len, total, H, hd, paired) == \
-            up(fwd) + up(total * H * 4)
+            up(sched) + up(total * H * 4)
     assert pha.pha_attn_bwd_workspace_bytes(1, 16, -1, 2, 16, False) == 0
     assert pha.pha_attn_bwd_workspace_bytes(0, 16, 16, 2, 16, False) == 0
     assert pha.pha_attn_bwd_workspace_bytes(1, 16, 16, 3, 16, True) == 0

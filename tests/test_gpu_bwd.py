@@ -2,10 +2,10 @@
 recompute the softmax from q and k. Needs a B200.
 
 Tolerances. Both backward paths take D_i = dO_i . O_i from the forward's stored O; the
-tensor-core path (bf16, causal, 1 <= window <= 128, head_dim 64 / 128) follows FlashAttention's
-backward arithmetic ("Training an LLM from scratch (part 2)", section "4. GQA & FlashAttention"):
-P and dS rounded to bf16 as MMA operands, float32 accumulation; the CUDA-core path (every other
-shape) keeps P and dS in float32. Near a document start a row sees few keys, P is large and dq is
+tensor-core path (bf16, head_dim 64 / 128, every window: band work lists or per-tile ones)
+follows FlashAttention's backward arithmetic ("Training an LLM from scratch (part 2)", section
+"4. GQA & FlashAttention"): P and dS rounded to bf16 as MMA operands, float32 accumulation; the
+CUDA-core path (every other shape) keeps P and dS in float32. Near a document start a row sees few keys, P is large and dq is
 a difference of large terms, so a tolerance scaled by the tensor's maximum does not describe the
 error. bf16 gradients are therefore bounded per element, from the rounding steps of the
 tensor-core path (u = 2^-8, the unit roundoff of bf16's 8 significant bits); the CUDA-core path's
@@ -125,15 +125,21 @@ def test_rope_bwd_parity(paired, stagger, dt):
 
 CASES = [
     # doc lens, H, Hkv, hd, dtype, causal, window, paired
-    # tensor-core path (bf16, causal, window <= 128, hd 64 / 128)
+    # tensor cores, band work lists (bf16, causal, window <= 128, hd 64 / 128)
     ((300, 5, 190), 6, 6, 128, "bf16", True, 128, True),
     ((257, 130), 4, 2, 64, "bf16", True, 37, False),
     ((1100, 37, 600), 6, 6, 128, "bf16", True, 128, True),   # runs split into items (has-prev)
     ((700, 129), 8, 2, 128, "bf16", True, 100, False),      # group of 4 query heads per kv head
     ((64, 1, 130), 2, 2, 64, "bf16", True, 1, True),        # window 1, a one-token document
-    # CUDA-core path
+    # tensor cores, tile work lists (bf16, hd 64 / 128, no window or one longer than a tile)
     ((200, 64), 8, 2, 128, "bf16", True, 0, False),
-    ((150, 90), 4, 4, 64, "bf16", False, 0, True),
+    ((150, 90), 4, 4, 64, "bf16", False, 0, True),          # non-causal, paired
+    ((700, 1, 1300), 4, 4, 64, "bf16", True, 0, False),     # full causal over ~10 key tiles
+    ((2000,), 4, 4, 64, "bf16", True, 1024, False),         # window 1024
+    ((900, 37), 8, 4, 128, "bf16", True, 300, True),        # window 300, paired, GQA
+    ((600,), 32, 8, 128, "bf16", True, 0, False),           # GQA 32 / 8 (groups of 4)
+    ((129, 257), 4, 2, 128, "bf16", False, 0, False),       # non-causal, GQA
+    # CUDA cores (f32; a bf16 forward exists only for head_dim 64 / 128)
     ((64,), 2, 2, 16, "f32", True, 0, True),
     ((80, 20), 4, 2, 32, "f32", True, 9, False),
 ]
