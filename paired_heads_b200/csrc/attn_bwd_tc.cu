@@ -48,7 +48,9 @@ namespace pha {
 
 namespace {
 
-constexpr int kBwdTcThreads = 320;
+// 8 elementwise warps; producer, MMA issuer and two idle warps (a whole third warpgroup for the
+// register split: the elementwise warpgroups hold 64 columns of S and of dP per thread)
+constexpr int kBwdTcThreads = 384;
 
 template <int HD, bool KEYMAJOR>
 struct BwdLayout {
@@ -264,6 +266,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 
     const int n_items = *reinterpret_cast<volatile int*>(&hdr->n_items);
     const int H = p.heads, Hkv = p.kv_heads, G = H / Hkv;
+    static_assert(8 * kTcRegsSoftmax + 4 * kTcRegsOther <= 12 * 168, "register split");
+    if (warp >= 8) regs_decrease<kTcRegsOther>();  // the whole third warpgroup, then its roles
     const bool reuse = !GEN && (!KEYMAJOR || G == 1);
     // X = (K, V) and Y = (Q, dO) (key-major), or the other way round
     const CUtensorMap* mx0 = KEYMAJOR ? &tm_k : &tm_q;
@@ -271,7 +275,9 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const CUtensorMap* my0 = KEYMAJOR ? &tm_q : &tm_k;
     const CUtensorMap* my1 = KEYMAJOR ? &tm_do : &tm_v;
 
-    if (warp == 8) {
+    if (warp >= 10) {
+        // ------------------------------------------------------------ idle (register split only)
+    } else if (warp == 8) {
         // ------------------------------------------------------------ producer
         // Per outer tile: with reuse its new Y fills, then X (the order in which their slots are
         // released); without, X and then one fill per step.
@@ -433,6 +439,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ elementwise warpgroups
+        regs_increase<kTcRegsSoftmax>();
         const int h = warp >> 2;              // the half of every step this warpgroup takes
         const int row = threadIdx.x & 127;    // TMEM lane == row of the outer tile
         const int r0 = (warp & 3) * 32;       // first row of this warp
@@ -495,41 +502,44 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                                                dev_status));
                         if (!ok) break;
                         tc_fence_after();
-#pragma unroll 1
-                        for (int c = 2 * h; c < 2 * h + 2; ++c) {
+                        // the half's 64 columns of S and dP, one wait
+                        uint32_t sv[64], dv[64];
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            tmem_ld32(tm_lane + L::kTmS + 32 * (2 * h + cc), sv + 32 * cc);
+                            tmem_ld32(tm_lane + L::kTmDP + 32 * (2 * h + cc), dv + 32 * cc);
+                        }
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            regs_after_wait(sv + 32 * cc);
+                            regs_after_wait(dv + 32 * cc);
+                        }
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int c = 2 * h + cc;
                             uint32_t pk[16], dk[16];
-                            if (32 * c > w_hi || 32 * c + 31 < w_lo) {  // no row of the warp sees it
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) pk[e] = dk[e] = 0u;
-                            } else {
-                                uint32_t sv[32], dv[32];
-                                tmem_ld32(tm_lane + L::kTmS + 32 * c, sv);
-                                tmem_ld32(tm_lane + L::kTmDP + 32 * c, dv);
-                                tmem_wait_ld();
-                                regs_after_wait(sv);
-                                regs_after_wait(dv);
+                            for (int e = 0; e < 32; e += 2) {
+                                float pr[2], dr[2];
 #pragma unroll
-                                for (int e = 0; e < 32; e += 2) {
-                                    float pr[2], dr[2];
-#pragma unroll
-                                    for (int x = 0; x < 2; ++x) {
-                                        const int col = 32 * c + e + x;
-                                        float l2 = lse2, d = dd;
-                                        if (KEYMAJOR) {
-                                            l2 = l2v[col];
-                                            d = l2v[128 + col];
-                                        }
-                                        const bool vis = col >= c_lo && col <= c_hi;
-                                        const float pe = ex2(fmaf(__uint_as_float(sv[e + x]), scale_log2, -l2));
-                                        pr[x] = vis ? pe : 0.f;
-                                        dr[x] = pr[x] * (__uint_as_float(dv[e + x]) - d);
+                                for (int x = 0; x < 2; ++x) {
+                                    const int col = 32 * c + e + x;
+                                    float l2 = lse2, d = dd;
+                                    if (KEYMAJOR) {
+                                        l2 = l2v[col];
+                                        d = l2v[128 + col];
                                     }
-                                    pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
-                                    dk[e >> 1] = pack_bf16x2(dr[0], dr[1]);
+                                    const bool vis = col >= c_lo && col <= c_hi;
+                                    const float pe = ex2(fmaf(__uint_as_float(sv[32 * cc + e + x]), scale_log2, -l2));
+                                    pr[x] = vis ? pe : 0.f;
+                                    dr[x] = pr[x] * (__uint_as_float(dv[32 * cc + e + x]) - d);
                                 }
+                                pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+                                dk[e >> 1] = pack_bf16x2(dr[0], dr[1]);
                             }
                             // packed pairs of the half's 64 columns: 32 TMEM columns from 64 h, over
-                            // columns of this half that this thread has already read
+                            // columns of this half already read
                             if (KEYMAJOR) tmem_st16(tm_lane + L::kTmS + 16 * c + 32 * h, pk);
                             tmem_st16(tm_lane + L::kTmDP + 16 * c + 32 * h, dk);
                         }
