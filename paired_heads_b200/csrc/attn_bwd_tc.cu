@@ -520,23 +520,29 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                             const int c = 2 * h + cc;
                             uint32_t pk[16], dk[16];
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
-                                float pr[2], dr[2];
+                            for (int e = 0; e < 32; e += 4) {
+                                // key-major: the four columns' lse * log2(e) and D, one broadcast
+                                // 16-byte shared load each
+                                float l2q[4] = {lse2, lse2, lse2, lse2}, dq4[4] = {dd, dd, dd, dd};
+                                if (KEYMAJOR) {
+                                    const float4 a4 = *reinterpret_cast<const float4*>(l2v + 32 * c + e);
+                                    const float4 b4 = *reinterpret_cast<const float4*>(l2v + 128 + 32 * c + e);
+                                    l2q[0] = a4.x; l2q[1] = a4.y; l2q[2] = a4.z; l2q[3] = a4.w;
+                                    dq4[0] = b4.x; dq4[1] = b4.y; dq4[2] = b4.z; dq4[3] = b4.w;
+                                }
+                                float pr[4], dr[4];
 #pragma unroll
-                                for (int x = 0; x < 2; ++x) {
+                                for (int x = 0; x < 4; ++x) {
                                     const int col = 32 * c + e + x;
-                                    float l2 = lse2, d = dd;
-                                    if (KEYMAJOR) {
-                                        l2 = l2v[col];
-                                        d = l2v[128 + col];
-                                    }
                                     const bool vis = col >= c_lo && col <= c_hi;
-                                    const float pe = ex2(fmaf(__uint_as_float(sv[32 * cc + e + x]), scale_log2, -l2));
+                                    const float pe = ex2(fmaf(__uint_as_float(sv[32 * cc + e + x]), scale_log2, -l2q[x]));
                                     pr[x] = vis ? pe : 0.f;
-                                    dr[x] = pr[x] * (__uint_as_float(dv[32 * cc + e + x]) - d);
+                                    dr[x] = pr[x] * (__uint_as_float(dv[32 * cc + e + x]) - dq4[x]);
                                 }
                                 pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+                                pk[(e >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
                                 dk[e >> 1] = pack_bf16x2(dr[0], dr[1]);
+                                dk[(e >> 1) + 1] = pack_bf16x2(dr[2], dr[3]);
                             }
                             // packed pairs of the half's 64 columns: 32 TMEM columns from 64 h, over
                             // columns of this half already read
