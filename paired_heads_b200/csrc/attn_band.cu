@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                     // below the first row's lower bound or above the last row's upper bound, wholly
                     // visible inside [last row's lower bound, first row's upper bound]. The max and
                     // the exponentials then run unmasked (2^-inf = 0).
+                    uint32_t hidden = 0;  // bit c: chunk c is hidden for every row of this warp
                     {
                         const int lo_first = q_start + r0 - window + 1 - kv0, lo_last = lo_first + 31;
                         const int hi_first = q_start + r0 - kv0, hi_last = hi_first + 31;
@@ -396,8 +397,9 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                             const int a = c_lo - lo, b = c_hi - lo;  // visible e in [a, b]
                             const uint32_t below = a <= 0 ? 0u : (a >= 32 ? ~0u : (1u << a) - 1u);
                             const uint32_t above = b >= 31 ? 0u : (b < 0 ? ~0u : ~((2u << b) - 1u));
-                            vis[c] = (hi < lo_first || lo > hi_last) ? 0u
-                                     : (lo >= lo_last && hi <= hi_first) ? ~0u : ~(below | above);
+                            const bool none = hi < lo_first || lo > hi_last;
+                            hidden |= none ? (1u << c) : 0u;
+                            vis[c] = none ? 0u : (lo >= lo_last && hi <= hi_first) ? ~0u : ~(below | above);
                         }
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
@@ -425,9 +427,20 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                     uint64_t sum_a = f32x2(0.f, 0.f), sum_b = f32x2(0.f, 0.f);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        uint32_t pk[16];
-                        chunk_exp<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
-                        tmem_st16(tm_s + 16 * c, pk);
+                        if (!((hidden >> c) & 1u)) {
+                            uint32_t pk[16];
+                            chunk_exp<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi, scale2, negm2, sum_a, sum_b, pk);
+                            tmem_st16(tm_s + 16 * c, pk);
+                        }
+                    }
+                    // chunks no row of the warp sees: P = 0, no exponentials
+                    if (hidden) {
+                        uint32_t zero[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            if ((hidden >> c) & 1u) tmem_st16(tm_s + 16 * c, zero);
                     }
                     const uint64_t sum2 = add_f32x2(sum_a, sum_b);
                     float s_lo, s_hi;
