@@ -3,6 +3,11 @@ inputs resident in HBM. Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--window W]
                     [--paired 0|1] [--qk-norm] [--aux-v] [--backward] [--impl reference]
+                    [--rope-tables factored|stored]
+
+--rope-tables picks the rotary tables of the step's RoPE: the compact float64 factor tables
+(pha_rope_factored, default) or the stored float32 cos / sin rows (pha_rope); the other form is
+timed after the step on the same inputs and reported beside it.
 
 --qk-norm replaces pha_rope with pha_qk_norm_rope (the QK RMS-norm of every head row, then RoPE,
 in one kernel). --aux-v adds a value embedding (a second v-shaped tensor) to v inside the
@@ -84,10 +89,17 @@ def attn_bytes(w) -> float:
     return float(w.total * w.head_dim * esz * (2 * w.n_heads + 2 * w.n_kv_heads) + 4 * w.total * w.n_heads)
 
 
-def rope_bytes(w, tab_width: int) -> float:
+def rope_bytes(w, tables: str = "stored", tab_rows: int = 0) -> float:
+    """Algorithmic HBM bytes of one RoPE call: q and k read and written, plus the tables: a cos
+    and a sin row per token (stored), or the factor tables read once (factored, L1 / L2-resident
+    after that)."""
     esz = 2 if w.dtype == "bf16" else 4
-    return float(2 * w.total * (w.n_heads + w.n_kv_heads) * w.head_dim * esz
-                 + 2 * 4 * w.total * tab_width)
+    qk = 2 * w.total * (w.n_heads + w.n_kv_heads) * w.head_dim * esz
+    if tables == "stored":
+        return float(qk + 2 * 4 * w.total * (2 if w.paired else 1) * w.head_dim)
+    a_width = w.head_dim if w.paired else w.head_dim // 2
+    fac = (16 * a_width + -(-tab_rows // 16) * (w.head_dim // 2)) * 16
+    return float(qk + fac)
 
 
 def load_peaks():
@@ -217,6 +229,9 @@ def main():
                     help="also time the backward (pha_attn_bwd + pha_rope_bwd)")
     ap.add_argument("--aux-v", action="store_true",
                     help="add a value embedding to v inside attention (pha_attn_fwd_aux_v)")
+    ap.add_argument("--rope-tables", default="factored", choices=["factored", "stored"],
+                    help="RoPE with the factored float64 tables (pha_rope_factored) or the stored "
+                         "float32 rows (pha_rope)")
     ap.add_argument("--oracle-tokens", type=int, default=16384)
     ap.add_argument("--no-suite", action="store_true",
                     help="skip the per-workload timings of the other page-shaped workloads")
@@ -257,7 +272,7 @@ def main():
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     cu, pos = inp["cu_seqlens"].to(dev), inp["positions"].to(dev)
     tab_rows = int(inp["positions"].max()) + 1
-    step = AttentionStep(StepShape.of(w, tab_rows), dev)
+    step = AttentionStep(StepShape.of(w, tab_rows), dev, rope_tables=args.rope_tables)
     stream = torch.cuda.current_stream(dev)
 
     def rotary(qq, kk, pp):
@@ -373,7 +388,7 @@ def main():
     for (a0, a1) in chunks:
         t0, t1 = cu_h[a0], cu_h[a1]
         sub = w.with_(doc_lens=tuple(w.doc_lens[a0:a1]))
-        st_ = AttentionStep(StepShape.of(sub, tab_rows), dev)
+        st_ = AttentionStep(StepShape.of(sub, tab_rows), dev, rope_tables=args.rope_tables)
         bufs = {n: torch.empty((t1 - t0,) + tuple(host[n].shape[1:]), dtype=host[n].dtype, device=dev)
                 for n in host if n not in ("cu_seqlens", "positions")}
         bufs["cu_seqlens"] = torch.empty(a1 - a0 + 1, dtype=torch.int32, device=dev)
@@ -421,19 +436,40 @@ def main():
     h2d = sum(host[n].numel() * host[n].element_size() for n in host)
     d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * 4
 
+    # the other RoPE table form on the same inputs, for comparison (not part of `value`)
+    alt_tables = "stored" if args.rope_tables == "factored" else "factored"
+    alt = AttentionStep(StepShape.of(w, tab_rows), dev, rope_tables=alt_tables)
+    alt_rope = alt.norm_rope if args.qk_norm else alt.rope
+    for _ in range(3):
+        alt_rope(q, k, pos)
+    alt_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+              for _ in range(max(5, min(args.steps, 50)))]
+    for e in alt_ev:
+        e[0].record(stream)
+        alt_rope(q, k, pos)
+        e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    alt_ms = sum(e[0].elapsed_time(e[1]) for e in alt_ev) / len(alt_ev)
+    del alt
+
     flops = attn_flops(w)
     peaks, peak_src = load_peaks()
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
-    tab_width = (2 if w.paired else 1) * w.head_dim
     rname = "qk_norm_rope" if args.qk_norm else "rope"
+    rb = rope_bytes(w, args.rope_tables, tab_rows)
     # the value embedding is one more v-shaped read of the attention kernel
     ab = attn_bytes(w) + (float(w.total * w.n_kv_heads * w.head_dim * 2) if args.aux_v else 0.0)
     kernels = {
-        rname: {"ms": rope_ms, "bytes": rope_bytes(w, tab_width),
-                 "gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9,
-                 "frac_of_hbm": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                 "traffic": load_traffic(w, rname)},
+        rname: {"ms": rope_ms, "tables": args.rope_tables, "bytes": rb,
+                 "gbs": rb / (rope_ms * 1e-3) / 1e9,
+                 "frac_of_hbm": rb / (rope_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                 "traffic": load_traffic(w, rname + ("_factored" if args.rope_tables == "factored"
+                                                     else ""))},
+        f"{rname}_{alt_tables}": {
+            "ms": alt_ms, "tables": alt_tables, "bytes": rope_bytes(w, alt_tables, tab_rows),
+            "gbs": rope_bytes(w, alt_tables, tab_rows) / (alt_ms * 1e-3) / 1e9,
+            "note": "the other table form, timed after the step on the same inputs; not in value"},
         "attention": {"ms": attn_ms, "flops": flops, "bytes": ab,
                       "tflops": attn_tflops,
                       "gbs": ab / (attn_ms * 1e-3) / 1e9,
@@ -455,7 +491,7 @@ def main():
                 "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"]}
     roof["kernel"] = kname
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-    roof["traffic"] = load_traffic(w, kname)
+    roof["traffic"] = kernels[kname]["traffic"]
     roof["timing"] = ("CUDA events on the launching stream around each library call in the timed "
                       "region; the attention call includes its scheduler kernel")
 
@@ -484,7 +520,8 @@ def main():
     if bwd is not None:
         line["backward"] = bwd
     if not args.no_suite and args.workload == "paired_varlen" and not (args.qk_norm or args.aux_v):
-        line["configs"] = time_suite(max(3, min(args.steps, 20)), args.warmup, dev, peaks, rank)
+        line["configs"] = time_suite(max(3, min(args.steps, 20)), args.warmup, dev, peaks, rank,
+                                     args.rope_tables)
         line["fp8"] = time_fp8(max(3, min(args.steps, 20)), args.warmup, dev, peaks, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, s, thr = time_oracle(w, args.oracle_tokens, args.qk_norm)
@@ -513,7 +550,7 @@ SUITE = (
 L2_BYTES = 126 * 1024 * 1024
 
 
-def time_suite(steps: int, warmup: int, dev, peaks, rank: int = 0):
+def time_suite(steps: int, warmup: int, dev, peaks, rank: int = 0, rope_tables: str = "factored"):
     """RoPE + attention on each workload of SUITE, timed per call with CUDA events on the launching
     stream. Workloads whose inputs fit in L2 get a 256 MiB buffer written before every step (outside
     the events). Returns {label: {...}}."""
@@ -529,9 +566,10 @@ def time_suite(steps: int, warmup: int, dev, peaks, rank: int = 0):
         inp = synth.make_inputs(w, rank=rank)
         q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
         cu, pos = inp["cu_seqlens"].to(dev), inp["positions"].to(dev)
-        step = AttentionStep(StepShape.of(w, int(inp["positions"].max()) + 1), dev)
-        tab_width = (2 if w.paired else 1) * w.head_dim
-        in_l2 = attn_bytes(w) + rope_bytes(w, tab_width) < L2_BYTES
+        rows = int(inp["positions"].max()) + 1
+        step = AttentionStep(StepShape.of(w, rows), dev, rope_tables=rope_tables)
+        rb = rope_bytes(w, rope_tables, rows)
+        in_l2 = attn_bytes(w) + rb < L2_BYTES
         for _ in range(max(warmup, 3)):
             step.rope(q, k, pos)
             step.attn(q, k, v, cu)
@@ -568,7 +606,7 @@ def time_suite(steps: int, warmup: int, dev, peaks, rank: int = 0):
             "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
             "bound": bound, "frac_of_roofline": tflops / roof_tflops,
             "attn_gbs": ab / (attn_ms * 1e-3) / 1e9,
-            "rope_ms": rope_ms, "rope_gbs": rope_bytes(w, tab_width) / (rope_ms * 1e-3) / 1e9,
+            "rope_ms": rope_ms, "rope_gbs": rb / (rope_ms * 1e-3) / 1e9,
             "step_ms": rope_ms + attn_ms,
             "tokens_per_s": w.total / ((rope_ms + attn_ms) * 1e-3),
             "l2": "flushed (256 MiB write) before each step" if in_l2 else "inputs larger than L2",

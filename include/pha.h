@@ -110,6 +110,59 @@ pha_status pha_qk_norm_rope(void* q, void* k, const float* q_weight, const float
                             int paired, int stagger_offset, pha_stream_t stream);
 
 /*
+ * pha_rope_factor_bytes -- size in bytes of the factored rotary tables (pha_rope_factor_tables)
+ *   for table rows [0, rows), head_dim and paired; 0 for invalid arguments (rows < 0, head_dim
+ *   odd or <= 0, paired not 0/1).
+ */
+size_t pha_rope_factor_bytes(int rows, int head_dim, int paired);
+
+/*
+ * pha_rope_factor_tables -- fill factored rotary tables on the device. They stand for the
+ *   pha_rope_tables of the same rows, head_dim, paired and base (same frequencies, same float64
+ *   angles), in two small float64 tables that stay in L1 / L2 instead of a float32 row per
+ *   position: table row p = 16 r + l splits each angle into a coarse part (row 16 r; for a paired
+ *   row its even position 32 r) and a fine part (row l), whose cosines and sines are stored.
+ *   The factored RoPE calls form cos(a + b) = cos a cos b - sin a sin b and
+ *   sin(a + b) = sin a cos b + cos a sin b in float64 and round each once to float32 (the
+ *   "modded-nanogpt Paired Head Attention record" page, section "2. building the paired rotary
+ *   table", keeps precomputed factor tables; this is a compact form of the same values).
+ *   Layout, pairs (cos, sin) of float64: 16 fine rows of A entries (A = head_dim/2, or head_dim
+ *   when paired), entry a of fine row l holding position l (standard) or 2l + a / (head_dim/2)
+ *   (paired) at frequency i = a % (head_dim/2); then ceil(rows/16) coarse rows of head_dim/2
+ *   entries, entry i of coarse row r holding position 16 r (standard) or 32 r (paired) at
+ *   frequency i. Frequencies f_i = base^(-2i/head_dim) as in pha_rope_tables.
+ *   factors: device buffer of `bytes` >= pha_rope_factor_bytes(rows, head_dim, paired) bytes,
+ *   16-byte aligned, written.
+ *   Errors: PHA_ERR_INVALID for a NULL or misaligned buffer, bytes too small, rows < 0, head_dim
+ *   odd or <= 0, base <= 0, paired not 0/1.
+ */
+pha_status pha_rope_factor_tables(void* factors, size_t bytes, int rows, int head_dim, int paired,
+                                  double base, pha_stream_t stream);
+
+/*
+ * pha_rope_factored -- pha_rope with factored tables (pha_rope_factor_tables) in place of
+ *   cos_tab / sin_tab: the rotation reads only q and k from HBM.
+ *   factors: as written by pha_rope_factor_tables for `rows` rows and the same head_dim and
+ *   paired, 16-byte aligned, read only. positions index rows [0, rows); a token outside is left
+ *   unchanged. Each cosine and sine equals the stored table's float32 value except in the last
+ *   bit where the float64 angle-addition result (error about 1e-11 at angles of 1e5) lies that
+ *   close to a float32 rounding midpoint; with these values the rotation is correctly rounded as
+ *   in pha_rope. Other arguments, layouts and errors: as pha_rope (there is no tab_width;
+ *   stagger_offset is 0, or head_dim when paired).
+ */
+pha_status pha_rope_factored(void* q, void* k, const void* factors, int rows,
+                             const int32_t* positions, int total_tokens, int n_heads,
+                             int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                             int stagger_offset, pha_stream_t stream);
+
+/* pha_qk_norm_rope_factored -- pha_qk_norm_rope with factored tables, as pha_rope_factored. */
+pha_status pha_qk_norm_rope_factored(void* q, void* k, const float* q_weight,
+                                     const float* k_weight, float eps, const void* factors,
+                                     int rows, const int32_t* positions, int total_tokens,
+                                     int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype,
+                                     int paired, int stagger_offset, pha_stream_t stream);
+
+/*
  * pha_attn_workspace_bytes -- device workspace that pha_attn_fwd needs: a 256-byte header,
  * int32[batch + 1] of per-document scratch (padded to 16 bytes) and the varlen work list, 16
  * bytes for each of at most batch * ceil(L/256) * H' (query block, head) items (L = max_len,
@@ -217,6 +270,12 @@ pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* s
                         int tab_rows, int tab_width, const int32_t* positions, int total_tokens,
                         int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
                         int stagger_offset, pha_stream_t stream);
+
+/* pha_rope_bwd_factored -- pha_rope_bwd with factored tables, as pha_rope_factored. */
+pha_status pha_rope_bwd_factored(void* dq, void* dk, const void* factors, int rows,
+                                 const int32_t* positions, int total_tokens, int n_heads,
+                                 int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                                 int stagger_offset, pha_stream_t stream);
 
 /*
  * pha_attn_bwd_workspace_bytes -- device scratch pha_attn_bwd needs: a scheduling area (a 256-byte

@@ -76,6 +76,27 @@ struct AttnProblem {
 cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
                                double base, cudaStream_t stream);
 
+// Factored rotary tables: kRopeLoRows fine rows and rope_hi_rows(rows) coarse rows of float64
+// (cos, sin) pairs (layout in rope.cu).
+constexpr int kRopeLoRows = 16;
+__host__ __device__ inline int rope_hi_rows(int rows) {
+    return (rows + kRopeLoRows - 1) / kRopeLoRows;
+}
+inline size_t rope_factor_bytes(int rows, int head_dim, int paired) {
+    const size_t a_width = paired ? head_dim : head_dim / 2;
+    return (static_cast<size_t>(kRopeLoRows) * a_width +
+            static_cast<size_t>(rope_hi_rows(rows)) * (head_dim / 2)) * 2 * sizeof(double);
+}
+cudaError_t launch_rope_factor_tables(double2* fac, int rows, int head_dim, int paired, double base,
+                                      cudaStream_t stream);
+
+// RoPE (norm: QK RMS-norm first; neg: the backward, rotation by -angle) with factored tables.
+cudaError_t launch_rope_factored(void* q, void* k, const double2* fac, int rows,
+                                 const int32_t* positions, int total_tokens, int n_heads,
+                                 int n_kv_heads, int head_dim, int is_bf16, int paired,
+                                 int stagger_offset, bool norm, bool neg, const float* q_weight,
+                                 const float* k_weight, float eps, cudaStream_t stream);
+
 cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,
                         int tab_width, const int32_t* positions, int total_tokens, int n_heads,
                         int n_kv_heads, int head_dim, int is_bf16, int paired, int stagger_offset,

@@ -180,6 +180,95 @@ pha_status pha_rope_bwd(void* dq, void* dk, const float* cos_tab, const float* s
                : PHA_ERR_CUDA;
 }
 
+size_t pha_rope_factor_bytes(int rows, int head_dim, int paired) {
+    if (rows < 0 || head_dim <= 0 || (head_dim & 1) || (paired != 0 && paired != 1)) return 0;
+    return rope_factor_bytes(rows, head_dim, paired);
+}
+
+pha_status pha_rope_factor_tables(void* factors, size_t bytes, int rows, int head_dim, int paired,
+                                  double base, pha_stream_t stream) {
+    if (!factors || !aligned16(factors) || rows < 0 || head_dim <= 0 || (head_dim & 1) ||
+        !(base > 0.0) || (paired != 0 && paired != 1))
+        return PHA_ERR_INVALID;
+    if (bytes < rope_factor_bytes(rows, head_dim, paired)) return PHA_ERR_INVALID;
+    return launch_rope_factor_tables(static_cast<double2*>(factors), rows, head_dim, paired, base,
+                                     stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
+// Argument checks shared by the factored RoPE calls (those of pha_rope, with the factored tables
+// in place of the stored ones).
+static pha_status rope_factored_args(const void* q, const void* k, const void* factors, int rows,
+                                     const int32_t* positions, int total_tokens, int n_heads,
+                                     int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                                     int stagger_offset) {
+    if (dtype != PHA_BF16 && dtype != PHA_F32) return PHA_ERR_INVALID;
+    const int span = dtype == PHA_BF16 ? 16 : 8;
+    if (rows < 0 || total_tokens < 0 || n_heads <= 0 || n_kv_heads < 0 || head_dim <= 0 ||
+        head_dim % span != 0 || (paired != 0 && paired != 1))
+        return PHA_ERR_INVALID;
+    if (total_tokens > 0 && (!q || !aligned16(q) || (n_kv_heads > 0 && (!k || !aligned16(k))) ||
+                             !factors || !aligned16(factors) || !positions))
+        return PHA_ERR_INVALID;
+    if (!paired && stagger_offset != 0) return PHA_ERR_INVALID;
+    if (paired && stagger_offset != 0 && stagger_offset != head_dim) return PHA_ERR_INVALID;
+    return PHA_OK;
+}
+
+pha_status pha_rope_factored(void* q, void* k, const void* factors, int rows,
+                             const int32_t* positions, int total_tokens, int n_heads,
+                             int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                             int stagger_offset, pha_stream_t stream) {
+    const pha_status st = rope_factored_args(q, k, factors, rows, positions, total_tokens, n_heads,
+                                             n_kv_heads, head_dim, dtype, paired, stagger_offset);
+    if (st != PHA_OK || total_tokens == 0) return st;
+    return launch_rope_factored(q, k, static_cast<const double2*>(factors), rows, positions,
+                                total_tokens, n_heads, n_kv_heads, head_dim, dtype == PHA_BF16,
+                                paired, stagger_offset, false, false, nullptr, nullptr, 0.f,
+                                stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
+pha_status pha_qk_norm_rope_factored(void* q, void* k, const float* q_weight,
+                                     const float* k_weight, float eps, const void* factors,
+                                     int rows, const int32_t* positions, int total_tokens,
+                                     int n_heads, int n_kv_heads, int head_dim, pha_dtype dtype,
+                                     int paired, int stagger_offset, pha_stream_t stream) {
+    const pha_status st = rope_factored_args(q, k, factors, rows, positions, total_tokens, n_heads,
+                                             n_kv_heads, head_dim, dtype, paired, stagger_offset);
+    if (st != PHA_OK) return st;
+    if (!(eps >= 0.f) || !(eps < INFINITY)) return PHA_ERR_INVALID;
+    if ((q_weight && !aligned16(q_weight)) || (k_weight && !aligned16(k_weight)))
+        return PHA_ERR_INVALID;
+    const int cph = head_dim / (dtype == PHA_BF16 ? 8 : 4);
+    if (32 % cph != 0) return PHA_ERR_UNSUPPORTED;
+    if (total_tokens == 0) return PHA_OK;
+    return launch_rope_factored(q, k, static_cast<const double2*>(factors), rows, positions,
+                                total_tokens, n_heads, n_kv_heads, head_dim, dtype == PHA_BF16,
+                                paired, stagger_offset, true, false, q_weight, k_weight, eps,
+                                stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
+pha_status pha_rope_bwd_factored(void* dq, void* dk, const void* factors, int rows,
+                                 const int32_t* positions, int total_tokens, int n_heads,
+                                 int n_kv_heads, int head_dim, pha_dtype dtype, int paired,
+                                 int stagger_offset, pha_stream_t stream) {
+    const pha_status st = rope_factored_args(dq, dk, factors, rows, positions, total_tokens,
+                                             n_heads, n_kv_heads, head_dim, dtype, paired,
+                                             stagger_offset);
+    if (st != PHA_OK || total_tokens == 0) return st;
+    return launch_rope_factored(dq, dk, static_cast<const double2*>(factors), rows, positions,
+                                total_tokens, n_heads, n_kv_heads, head_dim, dtype == PHA_BF16,
+                                paired, stagger_offset, false, true, nullptr, nullptr, 0.f,
+                                stream) == cudaSuccess
+               ? PHA_OK
+               : PHA_ERR_CUDA;
+}
+
 // Scheduling area of the backward: header, per-document offsets and the largest of its work
 // lists, the tile lists (one item per 128-slot tile and head), rounded up to 256 bytes.
 static size_t bwd_sched_bytes(int batch, int max_len, int n_heads, int paired) {

@@ -16,6 +16,17 @@
 //         midpoint, rounding y gives the same bf16 as rounding the exact value. The rare rest is
 //         recomputed in float64, where bf16 x float32 products are exact, and rounded from there.
 //   f32:  always float64 (exact products, one rounding), then rounded to float32.
+//
+// Factored tables (pha_rope_factored and its norm / backward forms): instead of a float32 row per
+// position, two small float64 tables of (cos, sin) pairs, which stay in L1 / L2, so that the
+// rotation reads only q and k from HBM. Table row p = kRopeLoRows * r + l splits each angle into
+// a coarse part (row kRopeLoRows * r; for a paired row, its even position) and a fine part (row
+// l, either half), and cos(a + b) = cos a cos b - sin a sin b, sin(a + b) = sin a cos b +
+// cos a sin b in float64, rounded once to float32, give the value that the stored table holds
+// except where that float64 result lies within its own error (~1e-11 at angles of 1e5) of a
+// float32 rounding midpoint. This path rounds bf16 results faithfully (compensated float32, see
+// rot_pair_bf16_faithful): the correctly rounded value in all but ~1e-5 of the elements, else its
+// neighbour.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -40,6 +51,39 @@ __global__ void rope_tables_kernel(float* __restrict__ cos_tab, float* __restric
         sincos(pos * freq, &s, &c);
         cos_tab[idx] = static_cast<float>(c);
         sin_tab[idx] = static_cast<float>(s);
+    }
+}
+
+// Factored tables, (cos, sin) pairs of float64: first kRopeLoRows fine rows of A entries
+// (A = head_dim / 2, or head_dim when paired: entry a = half * head_dim / 2 + i holds the angle
+// of position l (standard) or 2l + half (paired) at frequency i), then ceil(rows / kRopeLoRows)
+// coarse rows of head_dim / 2 entries (row r, entry i: position kRopeLoRows * r, or twice that
+// when paired, at frequency i). Frequencies and float64 angles as in rope_tables_kernel.
+__global__ void rope_factor_tables_kernel(double2* __restrict__ fac, int rows, int head_dim,
+                                          int paired, double base) {
+    const int half_hd = head_dim / 2;
+    const int a_width = paired ? head_dim : half_hd;
+    const int64_t n_lo = static_cast<int64_t>(kRopeLoRows) * a_width;
+    const int64_t n = n_lo + static_cast<int64_t>(rope_hi_rows(rows)) * half_hd;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        double pos;
+        int i;
+        if (idx < n_lo) {
+            const int l = static_cast<int>(idx / a_width);
+            const int a = static_cast<int>(idx % a_width);
+            const int half = a / half_hd;
+            i = a % half_hd;
+            pos = paired ? 2.0 * l + half : static_cast<double>(l);
+        } else {
+            const int64_t r = (idx - n_lo) / half_hd;
+            i = static_cast<int>((idx - n_lo) % half_hd);
+            pos = static_cast<double>(r) * kRopeLoRows * (paired ? 2.0 : 1.0);
+        }
+        const double freq = pow(base, -2.0 * static_cast<double>(i) / head_dim);
+        double sv, cv;
+        sincos(pos * freq, &sv, &cv);
+        fac[idx] = make_double2(cv, sv);
     }
 }
 
@@ -93,6 +137,22 @@ __device__ __forceinline__ uint32_t rot_pair_bf16(float x0, float x1, float c, f
     return bf16_bits_rne(e0) | (bf16_bits_rne(e1) << 16);
 }
 
+// One rotated pair, faithfully rounded with float32 arithmetic (the factored-table path): the
+// products s*x are split exactly into t = fl(s*x) and e = s*x - t (one fma each), so
+// y = fl(fl(c*x' + t) + e) is within about one float32 ulp of the exact value even under
+// cancellation, and its bf16 rounding is the correctly rounded value or, when the exact value lies
+// that close to a bf16 rounding midpoint, its neighbour (at most one bf16 ulp away).
+__device__ __forceinline__ uint32_t rot_pair_bf16_faithful(float x0, float x1, float c, float s) {
+    const uint64_t xs = f32x2(x1, x0);
+    const uint64_t t2 = mul_f32x2(f32x2(-s, s), xs);          // fl(-s*x1), fl(s*x0)
+    const uint64_t tn = mul_f32x2(f32x2(s, -s), xs);          // -t2, exactly
+    const uint64_t e2 = fma_f32x2(f32x2(-s, s), xs, tn);      // the exact rounding errors
+    const uint64_t y2 = add_f32x2(fma_f32x2(f32x2(c, c), f32x2(x0, x1), t2), e2);
+    float y0, y1;
+    f32x2_split(y2, y0, y1);
+    return pack_bf16x2(y0, y1);
+}
+
 // 16-byte chunks of a row: 8 bf16 (4 pairs) or 4 f32 (2 pairs). to_floats gives the exact values;
 // rotate_f rotates E float values with the chunk's table values c[j], s[j] (j = element within
 // the chunk) and rounds once to the buffer type; pack_f only rounds.
@@ -110,24 +170,29 @@ struct Chunk16<__nv_bfloat16> {
             x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
         }
     }
+    template <bool FAITHFUL = false>
     __device__ static uint4 rotate_f(const float (&x)[E], const float (&c)[E], const float (&s)[E]) {
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)  // both members of a pair share one angle: c[2e] == c[2e+1]
-            o[e] = rot_pair_bf16(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e]);
+            o[e] = FAITHFUL ? rot_pair_bf16_faithful(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e])
+                            : rot_pair_bf16(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e]);
         return make_uint4(o[0], o[1], o[2], o[3]);
     }
     __device__ static uint4 pack_f(const float (&x)[E]) {
         return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                           pack_bf16x2(x[6], x[7]));
     }
+    template <bool FAITHFUL = false>
     __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
         uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[e] = rot_pair_bf16(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u),
-                                 c[2 * e], s[2 * e]);
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+            o[e] = FAITHFUL ? rot_pair_bf16_faithful(x0, x1, c[2 * e], s[2 * e])
+                            : rot_pair_bf16(x0, x1, c[2 * e], s[2 * e]);
+        }
         return make_uint4(o[0], o[1], o[2], o[3]);
     }
 };
@@ -141,6 +206,7 @@ struct Chunk16<float> {
         x[2] = __uint_as_float(a.z);
         x[3] = __uint_as_float(a.w);
     }
+    template <bool FAITHFUL = false>  // float32 results are always correctly rounded
     __device__ static uint4 rotate_f(const float (&x)[E], const float (&c)[E], const float (&s)[E]) {
         float y[E];
 #pragma unroll
@@ -158,6 +224,7 @@ struct Chunk16<float> {
         return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
                           __float_as_uint(x[3]));
     }
+    template <bool FAITHFUL = false>
     __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
         float x[E];
         to_floats(a, x);
@@ -182,9 +249,45 @@ constexpr int kRopeBatch = 4;
 template <typename T, bool NORM>
 constexpr int rope_min_blocks() { return (sizeof(T) == 2 && !NORM) ? 4 : 3; }
 
+// The cosines and sines of table columns [col, col + E) of one row (E even, inside one half of a
+// paired row; both members of a pair get the pair's value). Stored tables: crow / srow point at
+// the row. Factored (FACT): lo_row / hi_row point at the row's fine and coarse factor rows.
+template <int E, bool FACT, bool NEG>
+__device__ __forceinline__ void table_cs(const float* crow, const float* srow,
+                                         const double2* lo_row, const double2* hi_row, int col,
+                                         int head_dim, float (&c)[E], float (&s)[E]) {
+    if (!FACT) {
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+            const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col + e));
+            const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col + e));
+            c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
+            s[e] = NEG ? -sv.x : sv.x; s[e + 1] = NEG ? -sv.y : sv.y;
+            s[e + 2] = NEG ? -sv.z : sv.z; s[e + 3] = NEG ? -sv.w : sv.w;
+        }
+    } else {
+        const int upper = col >= head_dim;            // paired rows: second half (position 2p+1)
+        const int i0 = ((col - (upper ? head_dim : 0)) >> 1);  // frequency of the first pair
+        const int a0 = (upper ? head_dim >> 1 : 0) + i0;
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+            const double2 f = __ldg(lo_row + a0 + e / 2);  // fine angle b
+            const double2 g = __ldg(hi_row + i0 + e / 2);  // coarse angle a
+            const float cv = __double2float_rn(fma(g.x, f.x, -(g.y * f.y)));
+            const float sv = __double2float_rn(fma(g.y, f.x, g.x * f.y));
+            c[e] = cv;
+            c[e + 1] = cv;
+            s[e] = NEG ? -sv : sv;
+            s[e + 1] = NEG ? -sv : sv;
+        }
+    }
+}
+
 // NEG: the backward of RoPE (the gradient with respect to the input is the transposed rotation,
 // i.e. the rotation by -angle): the sines enter negated, which is exact.
-template <typename T, bool NORM, bool NEG = false>
+// FACT: factored tables (fac; cos_tab / sin_tab unused, tab_rows = the rows they stand for), and
+// bf16 results faithfully rounded by rot_pair_bf16_faithful instead of correctly rounded.
+template <typename T, bool NORM, bool NEG = false, bool FACT = false>
 __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel(T* __restrict__ q, T* __restrict__ k,
                                                    const float* __restrict__ cos_tab,
                                                    const float* __restrict__ sin_tab,
@@ -194,7 +297,8 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
                                                    int n_kv_heads, int head_dim, int paired,
                                                    int stagger_offset,
                                                    const float* __restrict__ q_weight,
-                                                   const float* __restrict__ k_weight, float eps) {
+                                                   const float* __restrict__ k_weight, float eps,
+                                                   const double2* __restrict__ fac) {
     constexpr int E = Chunk16<T>::E;
     const int cph = head_dim / E;                  // chunks per head row
     const int q_chunks = n_heads * cph;
@@ -202,21 +306,31 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // the position of the warp's next token is loaded one token ahead, so that the table loads
+    // of a token go out with its q / k loads instead of after a dependent position load
+    int pos_next = warp0 < total_tokens ? __ldg(positions + warp0) : 0;
     for (int64_t t = warp0; t < total_tokens; t += n_warps) {
+        const int pos = pos_next;
+        if (t + n_warps < total_tokens) pos_next = __ldg(positions + t + n_warps);
         uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
         uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
-        // the first batch of the token's q / k chunks does not depend on its position: its loads
-        // go out before the position and table loads, so the two latencies overlap
+        // the first batch of the token's q / k chunks goes out before the table loads
         uint4 raw[kRopeBatch];
 #pragma unroll
         for (int j = 0; j < kRopeBatch; ++j) {
             const int i = 32 * j + lane;
             if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
         }
-        const int pos = __ldg(positions + t);
         const bool in_range = pos >= 0 && pos < tab_rows;
-        const float* crow = cos_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
-        const float* srow = sin_tab + static_cast<int64_t>(in_range ? pos : 0) * tab_width;
+        const int prow = in_range ? pos : 0;
+        const float* crow = FACT ? nullptr : cos_tab + static_cast<int64_t>(prow) * tab_width;
+        const float* srow = FACT ? nullptr : sin_tab + static_cast<int64_t>(prow) * tab_width;
+        const double2* lo_row =
+            FACT ? fac + (prow % kRopeLoRows) * (paired ? head_dim : head_dim >> 1) : nullptr;
+        const double2* hi_row =
+            FACT ? fac + kRopeLoRows * (paired ? head_dim : head_dim >> 1) +
+                       static_cast<int64_t>(prow / kRopeLoRows) * (head_dim >> 1)
+                 : nullptr;
         // When cph divides 32 (and, paired, 32/cph is even so the head parity is fixed too), every
         // chunk of this lane sits at the same table columns: load them once per token.
         const bool uniform_cols = (32 % cph == 0) && (!paired || ((32 / cph) % 2 == 0));
@@ -224,14 +338,7 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
         if (uniform_cols && in_range) {
             const int h0 = (lane % n_chunks) / cph;  // any chunk of this lane gives the columns
             const int col0 = ((paired && (h0 & 1)) ? stagger_offset : 0) + (lane % cph) * E;
-#pragma unroll
-            for (int e = 0; e < E; e += 4) {
-                const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col0 + e));
-                const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col0 + e));
-                cu[e] = cv.x; cu[e + 1] = cv.y; cu[e + 2] = cv.z; cu[e + 3] = cv.w;
-                su[e] = NEG ? -sv.x : sv.x; su[e + 1] = NEG ? -sv.y : sv.y;
-                su[e + 2] = NEG ? -sv.z : sv.z; su[e + 3] = NEG ? -sv.w : sv.w;
-            }
+            table_cs<E, FACT, NEG>(crow, srow, lo_row, hi_row, col0, head_dim, cu, su);
         }
         // NORM: a lane's chunks always sit at element offset (lane % cph) * E of their head row
         // (cph divides 32), so its q and k weights are the same for every chunk and token.
@@ -301,18 +408,12 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
                     const int ih = i < q_chunks ? i : i - q_chunks;  // chunk index within q or k row
                     const int h = ih / cph;
                     const int col = ((paired && (h & 1)) ? stagger_offset : 0) + (ih - h * cph) * E;
-#pragma unroll
-                    for (int e = 0; e < E; e += 4) {
-                        const float4 cv = __ldg(reinterpret_cast<const float4*>(crow + col + e));
-                        const float4 sv = __ldg(reinterpret_cast<const float4*>(srow + col + e));
-                        c[e] = cv.x; c[e + 1] = cv.y; c[e + 2] = cv.z; c[e + 3] = cv.w;
-                        s[e] = NEG ? -sv.x : sv.x; s[e + 1] = NEG ? -sv.y : sv.y;
-                        s[e + 2] = NEG ? -sv.z : sv.z; s[e + 3] = NEG ? -sv.w : sv.w;
-                    }
+                    table_cs<E, FACT, NEG>(crow, srow, lo_row, hi_row, col, head_dim, c, s);
                 }
                 // y = cos * x + sign * sin * x_flip, x_flip swapping each adjacent pair; the sign
                 // is -1 on the even member and +1 on the odd member (a rotation by +angle).
-                const uint4 y = NORM ? Chunk16<T>::rotate_f(x, c, s) : Chunk16<T>::rotate(raw[j], c, s);
+                const uint4 y = NORM ? Chunk16<T>::template rotate_f<FACT>(x, c, s)
+                                     : Chunk16<T>::template rotate<FACT>(raw[j], c, s);
                 if (i < q_chunks) qrow[i] = y; else krow[i - q_chunks] = y;
             }
         }
@@ -331,13 +432,25 @@ cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int hea
     return cudaGetLastError();
 }
 
-template <bool NORM, bool NEG = false>
+cudaError_t launch_rope_factor_tables(double2* fac, int rows, int head_dim, int paired, double base,
+                                      cudaStream_t stream) {
+    const int64_t n = static_cast<int64_t>(kRopeLoRows) * (paired ? head_dim : head_dim / 2) +
+                      static_cast<int64_t>(rope_hi_rows(rows)) * (head_dim / 2);
+    if (n == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    const int grid = static_cast<int>(blocks < 148 * 64 ? blocks : 148 * 64);
+    rope_factor_tables_kernel<<<grid, threads, 0, stream>>>(fac, rows, head_dim, paired, base);
+    return cudaGetLastError();
+}
+
+template <bool NORM, bool NEG = false, bool FACT = false>
 static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, const float* sin_tab,
                                     int tab_rows, int tab_width, const int32_t* positions,
                                     int total_tokens, int n_heads, int n_kv_heads, int head_dim,
                                     int is_bf16, int paired, int stagger_offset,
                                     const float* q_weight, const float* k_weight, float eps,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, const double2* fac = nullptr) {
     if (total_tokens == 0) return cudaSuccess;
     // Persistent grid: one wave of as many 256-thread blocks as are resident at once, each warp
     // striding over tokens, so no tail wave of partly filled SMs (at 1e5+ tokens this is ~7%
@@ -353,16 +466,38 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
                                       : rope_min_blocks<float, NORM>());
     const unsigned blocks = static_cast<unsigned>(blocks64 < resident ? blocks64 : resident);
     if (is_bf16)
-        rope_kernel<__nv_bfloat16, NORM, NEG><<<blocks, threads, 0, stream>>>(
+        rope_kernel<__nv_bfloat16, NORM, NEG, FACT><<<blocks, threads, 0, stream>>>(
             static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), cos_tab, sin_tab,
             tab_rows, tab_width, positions, total_tokens, n_heads, n_kv_heads, head_dim, paired,
-            stagger_offset, q_weight, k_weight, eps);
+            stagger_offset, q_weight, k_weight, eps, fac);
     else
-        rope_kernel<float, NORM, NEG><<<blocks, threads, 0, stream>>>(
+        rope_kernel<float, NORM, NEG, FACT><<<blocks, threads, 0, stream>>>(
             static_cast<float*>(q), static_cast<float*>(k), cos_tab, sin_tab, tab_rows, tab_width,
             positions, total_tokens, n_heads, n_kv_heads, head_dim, paired, stagger_offset,
-            q_weight, k_weight, eps);
+            q_weight, k_weight, eps, fac);
     return cudaGetLastError();
+}
+
+cudaError_t launch_rope_factored(void* q, void* k, const double2* fac, int rows,
+                                 const int32_t* positions, int total_tokens, int n_heads,
+                                 int n_kv_heads, int head_dim, int is_bf16, int paired,
+                                 int stagger_offset, bool norm, bool neg, const float* q_weight,
+                                 const float* k_weight, float eps, cudaStream_t stream) {
+    const int width = paired ? 2 * head_dim : head_dim;
+    if (norm)
+        return launch_rope_impl<true, false, true>(q, k, nullptr, nullptr, rows, width, positions,
+                                                   total_tokens, n_heads, n_kv_heads, head_dim,
+                                                   is_bf16, paired, stagger_offset, q_weight,
+                                                   k_weight, eps, stream, fac);
+    if (neg)
+        return launch_rope_impl<false, true, true>(q, k, nullptr, nullptr, rows, width, positions,
+                                                   total_tokens, n_heads, n_kv_heads, head_dim,
+                                                   is_bf16, paired, stagger_offset, nullptr,
+                                                   nullptr, 0.f, stream, fac);
+    return launch_rope_impl<false, false, true>(q, k, nullptr, nullptr, rows, width, positions,
+                                                total_tokens, n_heads, n_kv_heads, head_dim,
+                                                is_bf16, paired, stagger_offset, nullptr, nullptr,
+                                                0.f, stream, fac);
 }
 
 cudaError_t launch_rope(void* q, void* k, const float* cos_tab, const float* sin_tab, int tab_rows,

@@ -62,9 +62,17 @@ _lib.pha_attn_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i
                               _i, ctypes.c_float, _p, _p, _p, _p, _sz, _p]
 _lib.pha_qk_norm_rope.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _p, _i, _i, _p, _i, _i, _i,
                                   _i, _i, _i, _i, _p]
+_lib.pha_rope_factor_bytes.argtypes = [_i, _i, _i]
+_lib.pha_rope_factor_bytes.restype = _sz
+_lib.pha_rope_factor_tables.argtypes = [_p, _sz, _i, _i, _i, ctypes.c_double, _p]
+_lib.pha_rope_factored.argtypes = [_p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.pha_rope_bwd_factored.argtypes = [_p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.pha_qk_norm_rope_factored.argtypes = [_p, _p, _p, _p, ctypes.c_float, _p, _i, _p, _i, _i, _i,
+                                           _i, _i, _i, _i, _p]
 for _f in ("pha_rope_tables", "pha_rope", "pha_attn_fwd", "pha_attn_status",
            "pha_attn_fwd_noalloc", "pha_test_attn_fwd_stalled", "pha_attn_fwd_fp8", "pha_qk_norm_rope", "pha_attn_fwd_aux_v", "pha_rope_bwd",
-           "pha_attn_bwd"):
+           "pha_attn_bwd", "pha_rope_factor_tables", "pha_rope_factored", "pha_rope_bwd_factored",
+           "pha_qk_norm_rope_factored"):
     getattr(_lib, _f).restype = _i
 
 
@@ -171,6 +179,56 @@ def pha_rope_bwd(dq, dk, cos_tab, sin_tab, positions, paired: bool = False, stag
                                              tab_rows, tab_width, _ptr(positions), total_tokens,
                                              n_heads, n_kv_heads, head_dim, dtype, int(paired),
                                              stagger_offset, _stream(stream, dq)))
+
+
+def pha_rope_factor_bytes(rows: int, head_dim: int, paired: bool) -> int:
+    return int(_lib.pha_rope_factor_bytes(rows, head_dim, int(paired)))
+
+
+def pha_rope_factor_tables(factors, rows: int, head_dim: int, paired: bool,
+                           base: float = 10000.0, stream=None, *, nbytes=None):
+    """Factored rotary tables for table rows [0, rows) into the device buffer `factors`."""
+    if nbytes is None:
+        nbytes = factors.numel() * factors.element_size()
+    _check("pha_rope_factor_tables",
+           _lib.pha_rope_factor_tables(_ptr(factors), nbytes, rows, head_dim, int(paired),
+                                       float(base), _stream(stream, factors)))
+
+
+def _rope_shape(q, k):
+    total_tokens, n_heads, head_dim = q.shape
+    return total_tokens, n_heads, 0 if k is None else k.shape[1], head_dim, _dtype_code(q)
+
+
+def pha_rope_factored(q, k, factors, rows: int, positions, paired: bool = False,
+                      stagger_offset: int = 0, stream=None):
+    """pha_rope with factored tables (pha_rope_factor_tables for `rows` rows)."""
+    t, h, hkv, hd, dt = _rope_shape(q, k)
+    _check("pha_rope_factored",
+           _lib.pha_rope_factored(_ptr(q), _ptr(k), _ptr(factors), rows, _ptr(positions), t, h,
+                                  hkv, hd, dt, int(paired), stagger_offset, _stream(stream, q)))
+
+
+def pha_qk_norm_rope_factored(q, k, factors, rows: int, positions, q_weight=None, k_weight=None,
+                              eps: float = 1e-6, paired: bool = False, stagger_offset: int = 0,
+                              stream=None):
+    """pha_qk_norm_rope with factored tables."""
+    t, h, hkv, hd, dt = _rope_shape(q, k)
+    _check("pha_qk_norm_rope_factored",
+           _lib.pha_qk_norm_rope_factored(_ptr(q), _ptr(k), _ptr(q_weight), _ptr(k_weight),
+                                          float(eps), _ptr(factors), rows, _ptr(positions), t, h,
+                                          hkv, hd, dt, int(paired), stagger_offset,
+                                          _stream(stream, q)))
+
+
+def pha_rope_bwd_factored(dq, dk, factors, rows: int, positions, paired: bool = False,
+                          stagger_offset: int = 0, stream=None):
+    """pha_rope_bwd with factored tables."""
+    t, h, hkv, hd, dt = _rope_shape(dq, dk)
+    _check("pha_rope_bwd_factored",
+           _lib.pha_rope_bwd_factored(_ptr(dq), _ptr(dk), _ptr(factors), rows, _ptr(positions), t,
+                                      h, hkv, hd, dt, int(paired), stagger_offset,
+                                      _stream(stream, dq)))
 
 
 def pha_attn_bwd_workspace_bytes(batch: int, max_len: int, total_tokens: int, n_heads: int,

@@ -38,14 +38,27 @@ class StepShape:
 
 
 class AttentionStep:
-    def __init__(self, shape: StepShape, device="cuda"):
+    """rope_tables: "stored" -- float32 cos / sin rows per position (pha_rope_tables, pha_rope);
+    "factored" -- the compact float64 factor tables (pha_rope_factor_tables, pha_rope_factored)."""
+
+    def __init__(self, shape: StepShape, device="cuda", rope_tables: str = "stored"):
+        if rope_tables not in ("stored", "factored"):
+            raise ValueError(f"rope_tables: {rope_tables!r}")
         self.s = shape
+        self.rope_tables = rope_tables
         dev = torch.device(device)
         width = (2 if shape.paired else 1) * shape.head_dim
-        self.cos_tab = torch.empty(max(shape.tab_rows, 1), width, device=dev)
-        self.sin_tab = torch.empty_like(self.cos_tab)
-        pha.pha_rope_tables(self.cos_tab, self.sin_tab, shape.tab_rows, shape.head_dim,
-                            shape.paired, shape.rope_base)
+        self.cos_tab = self.sin_tab = self.factors = None
+        if rope_tables == "stored":
+            self.cos_tab = torch.empty(max(shape.tab_rows, 1), width, device=dev)
+            self.sin_tab = torch.empty_like(self.cos_tab)
+            pha.pha_rope_tables(self.cos_tab, self.sin_tab, shape.tab_rows, shape.head_dim,
+                                shape.paired, shape.rope_base)
+        else:
+            nbytes = pha.pha_rope_factor_bytes(shape.tab_rows, shape.head_dim, shape.paired)
+            self.factors = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+            pha.pha_rope_factor_tables(self.factors, shape.tab_rows, shape.head_dim,
+                                       shape.paired, shape.rope_base)
         dt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
         self.o = torch.empty(shape.total_tokens, shape.n_heads, shape.head_dim, dtype=dt, device=dev)
         self.lse = torch.empty(shape.total_tokens, shape.n_heads, dtype=torch.float32, device=dev)
@@ -55,11 +68,21 @@ class AttentionStep:
         self.stagger_offset = shape.head_dim if (shape.paired and shape.stagger) else 0
 
     def rope(self, q, k, positions, stream=None):
+        if self.factors is not None:
+            pha.pha_rope_factored(q, k, self.factors, self.s.tab_rows, positions,
+                                  paired=self.s.paired, stagger_offset=self.stagger_offset,
+                                  stream=stream)
+            return
         pha.pha_rope(q, k, self.cos_tab, self.sin_tab, positions, paired=self.s.paired,
                      stagger_offset=self.stagger_offset, stream=stream)
 
     def norm_rope(self, q, k, positions, q_weight=None, k_weight=None, eps=1e-6, stream=None):
         """QK RMS-norm of every head row, then RoPE, in place (one kernel)."""
+        if self.factors is not None:
+            pha.pha_qk_norm_rope_factored(q, k, self.factors, self.s.tab_rows, positions,
+                                          q_weight, k_weight, eps, paired=self.s.paired,
+                                          stagger_offset=self.stagger_offset, stream=stream)
+            return
         pha.pha_qk_norm_rope(q, k, self.cos_tab, self.sin_tab, positions, q_weight, k_weight, eps,
                              paired=self.s.paired, stagger_offset=self.stagger_offset,
                              stream=stream)
@@ -86,6 +109,11 @@ class AttentionStep:
 
     def rope_bwd(self, dq, dk, positions, stream=None):
         """In place: gradients w.r.t. the rotated q, k -> w.r.t. the unrotated q, k."""
+        if self.factors is not None:
+            pha.pha_rope_bwd_factored(dq, dk, self.factors, self.s.tab_rows, positions,
+                                      paired=self.s.paired, stagger_offset=self.stagger_offset,
+                                      stream=stream)
+            return
         pha.pha_rope_bwd(dq, dk, self.cos_tab, self.sin_tab, positions, paired=self.s.paired,
                          stagger_offset=self.stagger_offset, stream=stream)
 

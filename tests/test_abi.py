@@ -30,9 +30,11 @@ def test_header_declares_the_entry_points():
     assert _declared() == ["pha_attn_bwd", "pha_attn_bwd_workspace_bytes", "pha_attn_fwd",
                            "pha_attn_fwd_aux_v", "pha_attn_fwd_fp8", "pha_attn_fwd_noalloc",
                            "pha_attn_status",
-                           "pha_attn_workspace_bytes", "pha_qk_norm_rope", "pha_rope",
-                           "pha_rope_bwd", "pha_rope_tables", "pha_status_string",
-                           "pha_test_attn_fwd_stalled"]
+                           "pha_attn_workspace_bytes", "pha_qk_norm_rope",
+                           "pha_qk_norm_rope_factored", "pha_rope", "pha_rope_bwd",
+                           "pha_rope_bwd_factored", "pha_rope_factor_bytes",
+                           "pha_rope_factor_tables", "pha_rope_factored", "pha_rope_tables",
+                           "pha_status_string", "pha_test_attn_fwd_stalled"]
 
 
 def test_library_exports_every_declared_symbol(pha):
@@ -317,3 +319,72 @@ def test_rope_bwd_argument_errors(pha):
     assert lib.pha_rope_bwd(*args[:5], 128, *args[6:]) == -1        # table width
     assert lib.pha_rope_bwd(MIS, *args[1:]) == -1
     assert lib.pha_rope_bwd(*args[:7], 0, *args[8:]) == 0           # no tokens
+
+
+def test_rope_factor_bytes_closed_form(pha):
+    # 16 fine rows of head_dim/2 (standard) or head_dim (paired) (cos, sin) float64 pairs, then
+    # ceil(rows/16) coarse rows of head_dim/2 pairs
+    for rows, hd, paired in [(0, 64, 0), (1, 64, 1), (16, 128, 0), (17, 128, 1), (131072, 128, 1)]:
+        a = hd if paired else hd // 2
+        assert pha.pha_rope_factor_bytes(rows, hd, paired) == (16 * a + -(-rows // 16) * (hd // 2)) * 16
+    assert pha.pha_rope_factor_bytes(-1, 64, 0) == 0
+    assert pha.pha_rope_factor_bytes(4, 63, 0) == 0
+    assert pha.pha_rope_factor_bytes(4, 64, 2) == 0
+
+
+def test_rope_factor_tables_argument_errors(pha):
+    lib = pha.library()
+    need = pha.pha_rope_factor_bytes(64, 64, 1)
+    d = ctypes.c_double(1e4)
+    assert lib.pha_rope_factor_tables(None, need, 64, 64, 1, d, None) == -1
+    assert lib.pha_rope_factor_tables(MIS, need, 64, 64, 1, d, None) == -1
+    assert lib.pha_rope_factor_tables(A, need - 16, 64, 64, 1, d, None) == -1   # too small
+    assert lib.pha_rope_factor_tables(A, need, 64, 63, 1, d, None) == -1
+    assert lib.pha_rope_factor_tables(A, need, 64, 64, 1, ctypes.c_double(-1.0), None) == -1
+    assert lib.pha_rope_factor_tables(A, need, -1, 64, 1, d, None) == -1
+
+
+def _rope_factored(pha, fn="pha_rope_factored", **kw):
+    args = dict(q=A, k=A, fac=A, rows=16, pos=A, total=4, H=2, Hkv=2, hd=64,
+                dtype=pha.PHA_BF16, paired=0, stagger=0)
+    args.update(kw)
+    tail = (args["fac"], args["rows"], args["pos"], args["total"], args["H"], args["Hkv"],
+            args["hd"], args["dtype"], args["paired"], args["stagger"], None)
+    lib = pha.library()
+    if fn == "pha_qk_norm_rope_factored":
+        return lib.pha_qk_norm_rope_factored(args["q"], args["k"], None, None, ctypes.c_float(1e-6),
+                                             *tail)
+    return getattr(lib, fn)(args["q"], args["k"], *tail)
+
+
+@pytest.mark.parametrize("fn", ["pha_rope_factored", "pha_rope_bwd_factored",
+                                "pha_qk_norm_rope_factored"])
+@pytest.mark.parametrize("kw", [
+    dict(stagger=64),                          # stagger only on the paired path
+    dict(paired=1, stagger=32),                # stagger offset 0 or head_dim
+    dict(hd=40),                               # bf16 spans of 16 elements
+    dict(dtype=1, hd=12),                      # f32 spans of 8 elements
+    dict(q=MIS),
+    dict(fac=MIS),
+    dict(fac=None),
+    dict(k=None),
+    dict(pos=None),
+    dict(H=0),
+    dict(rows=-1),
+    dict(total=-2),
+])
+def test_rope_factored_argument_errors(pha, fn, kw):
+    assert _rope_factored(pha, fn, **kw) == -1
+
+
+@pytest.mark.parametrize("fn", ["pha_rope_factored", "pha_rope_bwd_factored",
+                                "pha_qk_norm_rope_factored"])
+def test_rope_factored_empty_is_a_no_op(pha, fn):
+    assert _rope_factored(pha, fn, total=0) == 0
+    assert _rope_factored(pha, fn, total=0, paired=1, stagger=64, q=None, k=None, fac=None,
+                          pos=None) == 0
+
+
+def test_norm_rope_factored_unsupported_head_dim(pha):
+    # 6 chunks per head row: not a divisor of 32
+    assert _rope_factored(pha, "pha_qk_norm_rope_factored", hd=48) == -2

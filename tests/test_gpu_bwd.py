@@ -96,9 +96,10 @@ def _ulp_bf16(x):
     return 2.0 ** (e - 7)
 
 
+@pytest.mark.parametrize("tables", ["stored", "factored"])
 @pytest.mark.parametrize("paired,stagger,dt", [(True, True, "bf16"), (False, False, "bf16"),
                                                (True, True, "f32")])
-def test_rope_bwd_parity(paired, stagger, dt):
+def test_rope_bwd_parity(paired, stagger, dt, tables):
     H, Hkv, hd, T = (6, 6, 128, 700) if dt == "bf16" else (4, 2, 16, 64)
     w = synth.Workload("rb", (T,), H, Hkv, hd, dt, paired=paired, stagger=stagger,
                        positions="global")
@@ -108,7 +109,7 @@ def test_rope_bwd_parity(paired, stagger, dt):
     pos[5] = -1                                     # outside the table: unchanged
     from paired_heads_b200.runner import AttentionStep, StepShape
 
-    step = AttentionStep(StepShape.of(w, 3000), "cuda")
+    step = AttentionStep(StepShape.of(w, 3000), "cuda", rope_tables=tables)
     gq, gk = inp["q"].cuda(), inp["k"].cuda()      # stand-ins for upstream gradients
     step.rope_bwd(gq, gk, torch.from_numpy(pos).cuda())
     for x, got in ((inp["q"], gq), (inp["k"], gk)):

@@ -39,8 +39,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("tables", ["stored", "factored"])
 @pytest.mark.parametrize("case", CASES)
-def test_norm_rope_parity(case):
+def test_norm_rope_parity(case, tables):
     dt, paired, stagger, hd, H, Hkv, T, weights, eps = case
     w = synth.Workload("norm", (T,), H, Hkv, hd, dt, paired=paired, stagger=stagger,
                        positions="global")
@@ -57,7 +58,7 @@ def test_norm_rope_parity(case):
     kw = torch.from_numpy(rng.uniform(0.5, 1.5, hd).astype(np.float32)) if weights else None
     from paired_heads_b200.runner import AttentionStep, StepShape
 
-    step = AttentionStep(StepShape.of(w, 5000), "cuda")
+    step = AttentionStep(StepShape.of(w, 5000), "cuda", rope_tables=tables)
     q, k = qh.cuda(), kh.cuda()
     step.norm_rope(q, k, torch.from_numpy(pos).cuda(), None if qw is None else qw.cuda(),
                    None if kw is None else kw.cuda(), eps)

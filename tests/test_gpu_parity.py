@@ -45,6 +45,76 @@ def test_rope_tables(paired, hd):
     np.testing.assert_allclose(st.cpu().numpy(), np.sin(ang), rtol=0, atol=6e-8)
 
 
+@pytest.mark.parametrize("paired", [False, True])
+@pytest.mark.parametrize("hd", [16, 128])
+def test_rope_factor_tables(paired, hd):
+    pha = _pha()
+    rows = 5000
+    nb = pha.pha_rope_factor_bytes(rows, hd, paired)
+    fac = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    pha.pha_rope_factor_tables(fac, rows, hd, paired, 10000.0)
+    f = fac.view(torch.float64).cpu().numpy().reshape(-1, 2)
+    half = hd // 2
+    a_width = hd if paired else half
+    n_lo = 16 * a_width
+    inv = 10000.0 ** (-2.0 * np.arange(half) / hd)
+    # the documented layout: fine rows (position l, or 2l + half) then coarse rows (16 r, or 32 r)
+    a = np.arange(a_width)
+    lo_pos = (2 * np.arange(16)[:, None] + a[None, :] // half) if paired else \
+        np.broadcast_to(np.arange(16)[:, None], (16, a_width))
+    lo_ang = lo_pos * inv[a % half][None, :]
+    n_hi = -(-rows // 16)
+    hi_ang = (np.arange(n_hi)[:, None] * 16 * (2 if paired else 1)) * inv[None, :]
+    ang = np.concatenate([lo_ang.reshape(-1), hi_ang.reshape(-1)])
+    assert f.shape[0] == n_lo + n_hi * half
+    # float64 sincos of float64 angles (up to 1e4 rad here): the C library and CUDA agree to a
+    # few units of 1e-16 per angle unit
+    np.testing.assert_allclose(f[:, 0], np.cos(ang), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(f[:, 1], np.sin(ang), rtol=0, atol=1e-12)
+    # recombined by angle addition and rounded to float32 they are the stored tables' values,
+    # except in the last bit next to float32 rounding midpoints
+    width = (2 if paired else 1) * hd
+    ct = torch.empty(rows, width, device="cuda")
+    st = torch.empty_like(ct)
+    pha.pha_rope_tables(ct, st, rows, hd, paired, 10000.0)
+    p = np.arange(rows)
+    j = np.arange(width)
+    lo_idx = (p % 16)[:, None] * a_width + ((j // hd) * half if paired else 0) + (j % hd) // 2
+    hi_idx = n_lo + (p // 16)[:, None] * half + ((j % hd) // 2)[None, :]
+    fl, fh = f[lo_idx], f[hi_idx]
+    c = (fh[..., 0] * fl[..., 0] - fh[..., 1] * fl[..., 1]).astype(np.float32)
+    s_ = (fh[..., 1] * fl[..., 0] + fh[..., 0] * fl[..., 1]).astype(np.float32)
+    for got, ref in ((c, ct.cpu().numpy()), (s_, st.cpu().numpy())):
+        d = np.abs(got.astype(np.float64) - ref)
+        assert np.all(d <= np.spacing(np.abs(ref)) * 1.0001)
+        assert np.mean(d == 0) > 0.99, float(np.mean(d == 0))
+
+
+def test_rope_factored_matches_stored():
+    # the headline shape on a slice of tokens at positions up to 131,072: the stored-table path is
+    # correctly rounded, the factored one faithfully rounded (compensated float32: the correctly
+    # rounded value except next to bf16 rounding midpoints, about 1e-5 of the elements, where it
+    # may be the neighbour); a last-bit difference of a cosine or sine moves far fewer
+    from paired_heads_b200.runner import AttentionStep, StepShape
+
+    w = synth.Workload("rope", (4096,), 6, 6, 128, "bf16", paired=True, stagger=True,
+                       positions="global")
+    inp = synth.make_inputs(w)
+    rng = np.random.default_rng(5)
+    pos = torch.from_numpy(rng.integers(0, 131072, 4096).astype(np.int32)).cuda()
+    outs = []
+    for tables in ("stored", "factored"):
+        step = AttentionStep(StepShape.of(w, 131072), "cuda", rope_tables=tables)
+        q, k = inp["q"].cuda(), inp["k"].cuda()
+        step.rope(q, k, pos)
+        outs.append((q, k))
+    for a, b in zip(outs[0], outs[1]):
+        same = (a.view(torch.int16) == b.view(torch.int16)).double().mean().item()
+        assert same > 0.9999, same
+        d = (a.double() - b.double()).abs()
+        assert torch.all(d <= a.double().abs() * 2.0 ** -7 + 1e-30)
+
+
 def _ulp_bf16(x):
     e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
     return 2.0 ** (e - 7)
@@ -62,8 +132,9 @@ ROPE_CASES = [
 ]
 
 
+@pytest.mark.parametrize("tables", ["stored", "factored"])
 @pytest.mark.parametrize("case", ROPE_CASES)
-def test_rope_parity(case):
+def test_rope_parity(case, tables):
     dt, paired, stagger, hd, H, Hkv, T = case
     w = synth.Workload("rope", (T,), H, Hkv, hd, dt, paired=paired, stagger=stagger,
                        positions="global")
@@ -75,7 +146,7 @@ def test_rope_parity(case):
     inp["positions"] = torch.from_numpy(pos)
     from paired_heads_b200.runner import AttentionStep, StepShape
 
-    step = AttentionStep(StepShape.of(w, 70000), "cuda")
+    step = AttentionStep(StepShape.of(w, 70000), "cuda", rope_tables=tables)
     q, k = inp["q"].cuda(), inp["k"].cuda()
     step.rope(q, k, inp["positions"].cuda())
     pos_ok = np.clip(pos, 0, None)
@@ -86,8 +157,10 @@ def test_rope_parity(case):
         g = got.to(torch.float64).cpu().numpy()
         # Both sides round the float64 rotation of the float32 table values once to the dtype,
         # so they agree bit for bit except where the two float32 tables differ in a last bit
-        # (CUDA's and the C library's float64 sin / cos / pow), which may move a result by one
-        # unit in the last place.
+        # (CUDA's and the C library's float64 sin / cos / pow; with factored tables also the
+        # float64 angle addition), which may move a result by one unit in the last place. The
+        # factored path rounds bf16 results faithfully (compensated float32 arithmetic): next to a
+        # rounding midpoint (about 1e-5 of the elements) it may give the other neighbour.
         diff = np.abs(g - ref)
         ulp = _ulp_bf16(ref) if dt == "bf16" else np.spacing(np.abs(ref).astype(np.float32))
         assert np.all(diff <= ulp * 1.0001), float((diff / ulp).max())
