@@ -380,13 +380,15 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 4; ++c) regs_after_wait(v + 32 * c);
-                    // Hidden scores are set to -inf in place: bit e of vis[c] says whether column
-                    // 32 c + e is visible for this row. Chunks classed uniformly over this warp's
-                    // rows (the bounds grow with the row) skip the per-row test: wholly hidden
-                    // below the first row's lower bound or above the last row's upper bound, wholly
-                    // visible inside [last row's lower bound, first row's upper bound]. The max and
-                    // the exponentials then run unmasked (2^-inf = 0).
-                    uint32_t hidden = 0;  // bit c: chunk c is hidden for every row of this warp
+                    // Chunks of 32 columns are classed over this warp's rows (the bounds grow with
+                    // the row): wholly hidden below the first row's lower bound or above the last
+                    // row's upper bound (left out of the max; P = 0 without exponentials), wholly
+                    // visible inside [last row's lower bound, first row's upper bound] (no test),
+                    // else partial: there hidden scores are set to -inf in place (bit e of vis[c]:
+                    // column 32 c + e visible for this row). The max and the exponentials then run
+                    // unmasked (2^-inf = 0).
+                    uint32_t hidden = 0;   // bit c: chunk c is hidden for every row of this warp
+                    uint32_t partial = 0;  // bit c: chunk c is neither wholly visible nor hidden
                     {
                         const int lo_first = q_start + r0 - window + 1 - kv0, lo_last = lo_first + 31;
                         const int hi_first = q_start + r0 - kv0, hi_last = hi_first + 31;
@@ -398,21 +400,29 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                             const uint32_t below = a <= 0 ? 0u : (a >= 32 ? ~0u : (1u << a) - 1u);
                             const uint32_t above = b >= 31 ? 0u : (b < 0 ? ~0u : ~((2u << b) - 1u));
                             const bool none = hi < lo_first || lo > hi_last;
+                            const bool all = lo >= lo_last && hi <= hi_first;
                             hidden |= none ? (1u << c) : 0u;
-                            vis[c] = none ? 0u : (lo >= lo_last && hi <= hi_first) ? ~0u : ~(below | above);
+                            partial |= (none || all) ? 0u : (1u << c);
+                            vis[c] = ~(below | above);
                         }
+                        // both classes are the same for every lane of the warp: the branches are
+                        // uniform, and only the partial chunks (the diagonal one for window 128)
+                        // pay the per-element test
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
+                            if ((partial >> c) & 1u) {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                v[32 * c + e] = ((vis[c] >> e) & 1u) ? v[32 * c + e]
-                                                                     : __float_as_uint(-INFINITY);
+                                for (int e = 0; e < 32; ++e)
+                                    v[32 * c + e] = ((vis[c] >> e) & 1u) ? v[32 * c + e]
+                                                                         : __float_as_uint(-INFINITY);
+                            }
                     }
-                    // row max over the visible columns
+                    // row max over the visible columns (hidden chunks hold stale scores: skipped)
                     float mx = -INFINITY;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        mx = fmaxf(mx, chunk_max<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi));
+                        if (!((hidden >> c) & 1u))
+                            mx = fmaxf(mx, chunk_max<kMaskNone>(v + 32 * c, 32 * c, c_lo, c_hi));
                     const float m_new = fmaxf(m, mx * scale_log2);
                     // Keep the reference max until the row max grows by more than 8 (a factor
                     // 256): O / l and the lse are exact for any reference value.
