@@ -191,6 +191,13 @@ size_t pha_attn_workspace_bytes(int batch, int max_len, int n_heads, int head_di
  *      its contents need not be initialised. The scheduler kernel writes the work list into it
  *      and records in its first 8 bytes the number of work items and a device-side status
  *      (see pha_attn_status). May be NULL for PHA_F32, which does not use it.
+ *      The list stays in the workspace after the call, with a copy of cu_seqlens, the shape it
+ *      was built for and a checksum of its items. A later call on the same workspace whose
+ *      cu_seqlens values, shape (batch, max_len, total_tokens, heads, causal, window, paired,
+ *      kernel) and workspace size match, and whose items are intact, keeps the list instead of
+ *      rebuilding it (the scheduler kernel then only compares; the usual case when every layer
+ *      of a model attends over the same documents). Anything else rebuilds it, so the caller may
+ *      still use the workspace as scratch between calls.
  *   total_tokens = 0: q, k, v, o, lse may be NULL; the scheduler still records 0 work items.
  *   Slots that lie outside every document (cu_seqlens[batch] < total_tokens) are not written.
  *   Supported: bf16 with head_dim in {64, 128} (tcgen05 tensor-core kernel); f32 with

@@ -17,12 +17,22 @@ constexpr int kBandRows = kBandTiles * kBlockM;
 static_assert(kBandRows >= kItemRows, "band items must not outnumber block items");
 constexpr int kMaxCostBuckets = 4096;   // scheduler cost classes (longest-first ordering)
 
-// Workspace: header (bytes [0, 256)), per-document block offsets (int32[batch + 1], padded to 16
+// Workspace: header (bytes [0, 256)), per-document scratch (int32[batch + 1], padded to 16
 // bytes), then int4 work items.
+// Work-list cache: after a build the scheduler leaves a copy of cu_seqlens in the per-document
+// scratch and records in the header what else the list depends on (key) and a checksum of the
+// items; a later call whose inputs and items match reuses the list instead of rebuilding it.
 struct WorkspaceHeader {
     int n_items;
     int status;
+    uint32_t magic;     // kScheduleMagic while the fields below describe a valid list
+    int key[10];        // mode, batch, max_len, total_tokens, slot_mult, heads, causal, window,
+                        // capacity, n_buckets
+    uint32_t checksum;  // of the items, in order
+    int reused;         // 1 when the last scheduler call kept the list (read by tests)
 };
+constexpr uint32_t kScheduleMagic = 0x50484153u;
+static_assert(sizeof(WorkspaceHeader) <= 256, "the header must fit its 256 bytes");
 constexpr size_t kWorkspaceHeaderBytes = 256;
 
 inline size_t workspace_doc_bytes(int batch) {

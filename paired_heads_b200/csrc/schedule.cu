@@ -28,7 +28,9 @@
 //
 // One CTA of 1024 threads: (1) per-document validation and block counts, (2) an exclusive scan
 // over documents, (3) a cost histogram over all blocks, (4) a scan of the histogram in descending
-// cost order, (5) emission, one thread per block.
+// cost order, (5) emission, one thread per block. Before that, (0): when the workspace holds the
+// list of an earlier call with the same inputs (header key, the copy of cu_seqlens kept in the
+// per-document scratch, and the items' checksum all match) the kernel keeps it and returns.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -65,6 +67,34 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
     __syncthreads();  // warp_sums may be reused by the caller's next scan
     *total = t;
     return before + x - v;
+}
+
+// Checksum term of work item i (a multiply-xorshift mix of its words and index); the list's
+// checksum is the XOR over its items.
+__device__ __forceinline__ uint32_t item_hash(int4 it, uint32_t i) {
+    uint32_t a = static_cast<uint32_t>(it.x) ^ (i * 0x85EBCA6Bu);
+    a = a * 0x9E3779B1u + static_cast<uint32_t>(it.y);
+    a ^= a >> 15;
+    a = a * 0xC2B2AE35u + static_cast<uint32_t>(it.z);
+    a ^= a >> 13;
+    a = a * 0x27D4EB2Fu + static_cast<uint32_t>(it.w);
+    a ^= a >> 16;
+    return a;
+}
+
+// XOR of item_hash over items [0, n), across the CTA (every thread gets it).
+__device__ uint32_t items_checksum(const int4* items, int n, uint32_t* warp_x) {
+    uint32_t x = 0;
+    for (int i = threadIdx.x; i < n; i += kSchedThreads) x ^= item_hash(items[i], static_cast<uint32_t>(i));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x ^= __shfl_xor_sync(0xffffffffu, x, o);
+    if ((threadIdx.x & 31) == 0) warp_x[threadIdx.x >> 5] = x;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll 8
+    for (int w = 0; w < kSchedThreads / 32; ++w) t ^= warp_x[w];
+    __syncthreads();
+    return t;
 }
 
 struct BlockRange {
@@ -131,12 +161,39 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
     __shared__ int hist[kMaxCostBuckets];
     __shared__ int warp_sums[kSchedThreads / 32];
     __shared__ int bad;
+    __shared__ int same;
     // the attention kernel may start its prologue (barriers, tensor memory, descriptor prefetch)
     // now; it waits for this grid's completion before it reads the work list
     grid_dep_launch();
     const int tid = threadIdx.x;
     const int64_t mult = p.slot_mult;
     const int rows = mode_rows(mode);
+    const int key[10] = {mode, p.batch, p.max_len, p.total_tokens, p.slot_mult, p.heads,
+                         p.causal, p.window, capacity, n_buckets};
+
+    // (0) the list of an earlier call with the same inputs is kept
+    if (tid == 0) {
+        int ok = hdr->magic == kScheduleMagic && hdr->status == DEV_OK && hdr->n_items >= 0 &&
+                 hdr->n_items <= capacity;
+        for (int j = 0; j < 10; ++j) ok &= hdr->key[j] == key[j];
+        same = ok;
+    }
+    __syncthreads();
+    if (same) {
+        for (int d = tid; d <= p.batch; d += kSchedThreads)
+            if (p.cu_seqlens[d] != doc_blocks[d]) same = 0;
+        const uint32_t sum = items_checksum(items, hdr->n_items, reinterpret_cast<uint32_t*>(warp_sums));
+        if (sum != hdr->checksum) same = 0;  // (every thread computes the same sum)
+        __syncthreads();
+        if (same) {
+            if (tid == 0) hdr->reused = 1;
+            return;
+        }
+    }
+    if (tid == 0) {
+        hdr->magic = 0;
+        hdr->reused = 0;
+    }
     for (int c = tid; c < n_buckets; c += kSchedThreads) hist[c] = 0;
     if (tid == 0) bad = 0;
     __syncthreads();
@@ -219,9 +276,19 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(AttnProblem p, 
         for (int h = 0; h < p.heads; ++h)
             dst[h] = make_int4(r.item.x, (h << 16) | r.item.y, r.item.z, r.item.w);
     }
+    // the cache record: the copy of cu_seqlens replaces the per-document scratch, then the key,
+    // the items' checksum and the magic
+    __syncthreads();
+    for (int d = tid; d <= p.batch; d += kSchedThreads) doc_blocks[d] = p.cu_seqlens[d];
+    const uint32_t sum = items_checksum(items, static_cast<int>(n_items),
+                                        reinterpret_cast<uint32_t*>(warp_sums));
     if (tid == 0) {
         hdr->n_items = static_cast<int>(n_items);
         hdr->status = DEV_OK;
+        for (int j = 0; j < 10; ++j) hdr->key[j] = key[j];
+        hdr->checksum = sum;
+        __threadfence_block();
+        hdr->magic = kScheduleMagic;
     }
 }
 
