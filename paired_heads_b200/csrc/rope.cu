@@ -233,21 +233,26 @@ struct Chunk16<float> {
 };
 
 // One warp per token. The token's q row (n_heads * head_dim contiguous elements) followed by its
-// k row is cut into 16-byte chunks; lane l takes chunks l, l + 32, ... in batches of kBatch, so
-// every load instruction of the warp reads 512 contiguous bytes and each lane keeps kBatch x 16
-// bytes of HBM reads in flight; the first batch is issued before the position is known. All heads
-// of the token share its table row, which is read from HBM once and then served from L1.
-constexpr int kRopeBatch = 4;
+// k row is cut into 16-byte chunks; lane l takes chunks l, l + 32, ... in batches of kRopeBatch,
+// so every load instruction of the warp reads 512 contiguous bytes and each lane keeps
+// kRopeBatch x 16 bytes of HBM reads in flight (six for the rotation: a whole token of 12 q + k
+// heads of 64, or 6 of 128, in one batch; four with the norm, whose extra pass needs the
+// registers); the first batch is issued before the table loads. All heads of the token share its
+// table row, which is read from HBM once and then served from L1.
+template <bool NORM>
+constexpr int kRopeBatch = NORM ? 4 : 6;
 
 // NORM: each head row is first RMS-normalised over head_dim in float32 ("Training an LLM from
 // scratch (part 2)", section "1. RMSNorm": x / sqrt(mean(x^2) + eps) * weight; weight NULL = 1),
 // then rotated; one rounding at the end. The chunks of one head row sit on cph consecutive lanes
 // (cph divides 32), so the row's sum of squares is a shuffle reduction over those lanes. Tokens
 // whose position lies outside the table are normalised but not rotated.
-// Resident 256-thread blocks per SM: four (64 registers) for the plain bf16 rotation, the
-// bandwidth-bound case; three (80 registers, no spills) for the others.
-template <typename T, bool NORM>
-constexpr int rope_min_blocks() { return (sizeof(T) == 2 && !NORM) ? 4 : 3; }
+// Resident 256-thread blocks per SM: four (64 registers) for the plain bf16 rotation with stored
+// tables; three (80 registers) for the others, whose factor loads, float64 arithmetic or norm
+// need the registers (measured: the factored bf16 rotation at four blocks spills and runs ~12 %
+// slower).
+template <typename T, bool NORM, bool FACT>
+constexpr int rope_min_blocks() { return (sizeof(T) == 2 && !NORM && !FACT) ? 4 : 3; }
 
 // The cosines and sines of table columns [col, col + E) of one row (E even, inside one half of a
 // paired row; both members of a pair get the pair's value). Stored tables: crow / srow point at
@@ -288,7 +293,7 @@ __device__ __forceinline__ void table_cs(const float* crow, const float* srow,
 // FACT: factored tables (fac; cos_tab / sin_tab unused, tab_rows = the rows they stand for), and
 // bf16 results faithfully rounded by rot_pair_bf16_faithful instead of correctly rounded.
 template <typename T, bool NORM, bool NEG = false, bool FACT = false>
-__global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel(T* __restrict__ q, T* __restrict__ k,
+__global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_kernel(T* __restrict__ q, T* __restrict__ k,
                                                    const float* __restrict__ cos_tab,
                                                    const float* __restrict__ sin_tab,
                                                    int tab_rows, int tab_width,
@@ -315,9 +320,9 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
         uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
         uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
         // the first batch of the token's q / k chunks goes out before the table loads
-        uint4 raw[kRopeBatch];
+        uint4 raw[kRopeBatch<NORM>];
 #pragma unroll
-        for (int j = 0; j < kRopeBatch; ++j) {
+        for (int j = 0; j < kRopeBatch<NORM>; ++j) {
             const int i = 32 * j + lane;
             if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
         }
@@ -355,19 +360,19 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
                 wk[e] = b.x; wk[e + 1] = b.y; wk[e + 2] = b.z; wk[e + 3] = b.w;
             }
         }
-        for (int base = 0; base < n_chunks; base += 32 * kRopeBatch) {
+        for (int base = 0; base < n_chunks; base += 32 * kRopeBatch<NORM>) {
             if (base > 0) {
 #pragma unroll
-                for (int j = 0; j < kRopeBatch; ++j) {
+                for (int j = 0; j < kRopeBatch<NORM>; ++j) {
                     const int i = base + 32 * j + lane;
                     if (i < n_chunks) raw[j] = i < q_chunks ? qrow[i] : krow[i - q_chunks];
                 }
             }
-            float inv[kRopeBatch];
+            float inv[kRopeBatch<NORM>];
             if (NORM) {
                 // 1 / rms of the head row of each chunk (all lanes take part in the shuffles)
 #pragma unroll
-                for (int j = 0; j < kRopeBatch; ++j) {
+                for (int j = 0; j < kRopeBatch<NORM>; ++j) {
                     float ss = 0.f;
                     if (base + 32 * j + lane < n_chunks) {
                         float x[E];
@@ -382,7 +387,7 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM>())) rope_kernel
                 continue;  // positions outside the table: leave the token unchanged
             }
 #pragma unroll
-            for (int j = 0; j < kRopeBatch; ++j) {
+            for (int j = 0; j < kRopeBatch<NORM>; ++j) {
                 const int i = base + 32 * j + lane;
                 if (i >= n_chunks) break;
                 float x[E];
@@ -462,8 +467,8 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
     if (e != cudaSuccess) return e;
     const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
     const int64_t resident = static_cast<int64_t>(sms) *
-                             (is_bf16 ? rope_min_blocks<__nv_bfloat16, NORM>()
-                                      : rope_min_blocks<float, NORM>());
+                             (is_bf16 ? rope_min_blocks<__nv_bfloat16, NORM, FACT>()
+                                      : rope_min_blocks<float, NORM, FACT>());
     const unsigned blocks = static_cast<unsigned>(blocks64 < resident ? blocks64 : resident);
     if (is_bf16)
         rope_kernel<__nv_bfloat16, NORM, NEG, FACT><<<blocks, threads, 0, stream>>>(
