@@ -501,8 +501,10 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded N(0,1) q/k/v; geometric document lengths)",
         "config": {**workload_config(w), "qk_norm": bool(args.qk_norm), "aux_v": bool(args.aux_v),
+                   "rope_tables": args.rope_tables,
                    "parallelism": f"dp{world} (independent documents per rank)",
-                   "l2": "inputs larger than L2 (q,k,v + tables > 126 MB); no flush"},
+                   "l2": (f"inputs larger than L2 (q, k, v {attn_bytes(w) / 1e6:.0f} MB > 126 MB); "
+                          "no flush")},
         "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
         "attention_only_tflops": attn_tflops,
         "tokens_per_s": w.total * world / (ms_per_step * 1e-3),
