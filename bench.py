@@ -357,7 +357,7 @@ def main():
         ab_ms = sum(e[0].elapsed_time(e[1]) for e in bev) / nb
         rb_ms = sum(e[1].elapsed_time(e[2]) for e in bev) / nb
         bwd_flops = 2.5 * attn_flops(w)
-        tc_bwd = w.dtype == "bf16" and w.causal and 1 <= w.window <= 128 and w.head_dim in (64, 128)
+        tc_bwd = w.dtype == "bf16" and w.head_dim in (64, 128)
         bwd = {"ms": b_ms, "steps": nb, "flops": bwd_flops,
                "tflops": bwd_flops * world / (b_ms * 1e-3) / 1e12,
                "attn_bwd_ms": ab_ms, "rope_bwd_ms": rb_ms,
