@@ -425,6 +425,75 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_
     }
 }
 
+// Factored-table rotation (no norm) with the tokens' q and k rows staged in shared memory: each
+// warp keeps a private ring of R token slots, and each lane copies its own 16-byte chunks of the
+// token R - 1 steps ahead into it with cp.async, so R - 1 tokens of HBM reads per warp are in
+// flight without holding registers; before a token is rotated the lane waits for its own copy
+// group (a hardware wait) and reads back only the chunks it copied (no barrier). Used when every
+// chunk of a lane sits at the same table columns (as in rope_kernel's uniform case).
+template <typename T, bool NEG, int R, int MINB>
+__global__ void __launch_bounds__(256, MINB)
+    rope_ring_kernel(T* __restrict__ q, T* __restrict__ k, const int32_t* __restrict__ positions,
+                     int64_t total_tokens, int n_heads, int n_kv_heads, int head_dim, int paired,
+                     int stagger_offset, int tab_rows, const double2* __restrict__ fac) {
+    extern __shared__ __align__(16) uint8_t ring_smem[];
+    constexpr int E = Chunk16<T>::E;
+    const int cph = head_dim / E;
+    const int q_chunks = n_heads * cph;
+    const int n_chunks = q_chunks + n_kv_heads * cph;
+    const int lane = threadIdx.x & 31;
+    const int slot_bytes = n_chunks * 16;
+    uint8_t* ring = ring_smem + (threadIdx.x >> 5) * R * slot_bytes;
+    const int64_t warp0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int h0 = (lane % n_chunks) / cph;  // any chunk of this lane gives the columns
+    const int col0 = ((paired && (h0 & 1)) ? stagger_offset : 0) + (lane % cph) * E;
+    const int a_width = paired ? head_dim : head_dim >> 1;
+    auto issue = [&](int64_t t, int slot) {
+        const uint4* qrow = reinterpret_cast<const uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
+        const uint4* krow = reinterpret_cast<const uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
+        uint8_t* dst = ring + slot * slot_bytes;
+        for (int i = lane; i < n_chunks; i += 32)
+            cp_async_16(dst + i * 16, i < q_chunks ? qrow + i : krow + (i - q_chunks));
+    };
+#pragma unroll
+    for (int r = 0; r < R - 1; ++r) {
+        const int64_t t = warp0 + r * n_warps;
+        if (t < total_tokens) issue(t, r);
+        cp_async_commit();
+    }
+    int pos_next = warp0 < total_tokens ? __ldg(positions + warp0) : 0;
+    int slot = 0;
+    for (int64_t t = warp0; t < total_tokens; t += n_warps) {
+        const int64_t ta = t + (R - 1) * n_warps;
+        if (ta < total_tokens) issue(ta, (slot + R - 1) % R);  // the slot read last step
+        cp_async_commit();
+        const int pos = pos_next;
+        if (t + n_warps < total_tokens) pos_next = __ldg(positions + t + n_warps);
+        const bool in_range = pos >= 0 && pos < tab_rows;
+        float cu[E], su[E];
+        if (in_range) {
+            const double2* lo_row = fac + (pos % kRopeLoRows) * a_width;
+            const double2* hi_row =
+                fac + kRopeLoRows * a_width + static_cast<int64_t>(pos / kRopeLoRows) * (head_dim >> 1);
+            table_cs<E, true, NEG>(nullptr, nullptr, lo_row, hi_row, col0, head_dim, cu, su);
+        }
+        cp_async_wait<R - 1>();  // this lane's chunks of token t have landed
+        if (in_range) {  // a token outside the table is left unchanged
+            uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
+            uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
+            const uint8_t* src = ring + slot * slot_bytes;
+            for (int i = lane; i < n_chunks; i += 32) {
+                const uint4 y = Chunk16<T>::template rotate<true>(
+                    *reinterpret_cast<const uint4*>(src + i * 16), cu, su);
+                if (i < q_chunks) qrow[i] = y; else krow[i - q_chunks] = y;
+            }
+        }
+        slot = slot + 1 == R ? 0 : slot + 1;
+    }
+    cp_async_wait<0>();
+}
+
 cudaError_t launch_rope_tables(float* cos_tab, float* sin_tab, int rows, int head_dim, int paired,
                                double base, cudaStream_t stream) {
     const int64_t n = static_cast<int64_t>(rows) * (paired ? 2 : 1) * head_dim;
@@ -483,12 +552,60 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
     return cudaGetLastError();
 }
 
+// Ring depth and resident blocks of rope_ring_kernel.
+constexpr int kRingDepth = 3;
+constexpr int kRingBlocks = 3;
+
+template <typename T, bool NEG>
+static cudaError_t launch_rope_ring(void* q, void* k, const double2* fac, int rows,
+                                   const int32_t* positions, int total_tokens, int n_heads,
+                                   int n_kv_heads, int head_dim, int paired, int stagger_offset,
+                                   size_t smem, int sms, cudaStream_t stream) {
+    auto kern = rope_ring_kernel<T, NEG, kRingDepth, kRingBlocks>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
+    const int64_t resident = static_cast<int64_t>(sms) * kRingBlocks;
+    const unsigned blocks = static_cast<unsigned>(blocks64 < resident ? blocks64 : resident);
+    kern<<<blocks, 256, smem, stream>>>(static_cast<T*>(q), static_cast<T*>(k), positions,
+                                        total_tokens, n_heads, n_kv_heads, head_dim, paired,
+                                        stagger_offset, rows, fac);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_rope_factored(void* q, void* k, const double2* fac, int rows,
                                  const int32_t* positions, int total_tokens, int n_heads,
                                  int n_kv_heads, int head_dim, int is_bf16, int paired,
                                  int stagger_offset, bool norm, bool neg, const float* q_weight,
                                  const float* k_weight, float eps, cudaStream_t stream) {
     const int width = paired ? 2 * head_dim : head_dim;
+    // the ring kernel when a lane's chunks share table columns and its shared memory fits
+    const int cph = head_dim / (is_bf16 ? 8 : 4);
+    const bool uniform = (32 % cph == 0) && (!paired || ((32 / cph) % 2 == 0));
+    const size_t ring_smem =
+        static_cast<size_t>(8) * kRingDepth * (n_heads + n_kv_heads) * cph * 16;
+    if (!norm && uniform && total_tokens > 0 && ring_smem * kRingBlocks <= 220 * 1024) {
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        if (is_bf16)
+            return neg ? launch_rope_ring<__nv_bfloat16, true>(q, k, fac, rows, positions,
+                                                               total_tokens, n_heads, n_kv_heads,
+                                                               head_dim, paired, stagger_offset,
+                                                               ring_smem, sms, stream)
+                       : launch_rope_ring<__nv_bfloat16, false>(q, k, fac, rows, positions,
+                                                                total_tokens, n_heads, n_kv_heads,
+                                                                head_dim, paired, stagger_offset,
+                                                                ring_smem, sms, stream);
+        return neg ? launch_rope_ring<float, true>(q, k, fac, rows, positions, total_tokens,
+                                                   n_heads, n_kv_heads, head_dim, paired,
+                                                   stagger_offset, ring_smem, sms, stream)
+                   : launch_rope_ring<float, false>(q, k, fac, rows, positions, total_tokens,
+                                                    n_heads, n_kv_heads, head_dim, paired,
+                                                    stagger_offset, ring_smem, sms, stream);
+    }
     if (norm)
         return launch_rope_impl<true, false, true>(q, k, nullptr, nullptr, rows, width, positions,
                                                    total_tokens, n_heads, n_kv_heads, head_dim,
