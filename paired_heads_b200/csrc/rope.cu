@@ -431,11 +431,15 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_
 // flight without holding registers; before a token is rotated the lane waits for its own copy
 // group (a hardware wait) and reads back only the chunks it copied (no barrier). Used when every
 // chunk of a lane sits at the same table columns (as in rope_kernel's uniform case).
-template <typename T, bool NEG, int R, int MINB>
+// NORM: the QK RMS-norm of each head row first, as in rope_kernel (the row's chunks sit on cph
+// consecutive lanes of one 32-chunk round, whose lanes all take part in the shuffles).
+template <typename T, bool NEG, bool NORM, int R, int MINB>
 __global__ void __launch_bounds__(256, MINB)
     rope_ring_kernel(T* __restrict__ q, T* __restrict__ k, const int32_t* __restrict__ positions,
                      int64_t total_tokens, int n_heads, int n_kv_heads, int head_dim, int paired,
-                     int stagger_offset, int tab_rows, const double2* __restrict__ fac) {
+                     int stagger_offset, int tab_rows, const double2* __restrict__ fac,
+                     const float* __restrict__ q_weight, const float* __restrict__ k_weight,
+                     float eps) {
     extern __shared__ __align__(16) uint8_t ring_smem[];
     constexpr int E = Chunk16<T>::E;
     const int cph = head_dim / E;
@@ -449,6 +453,19 @@ __global__ void __launch_bounds__(256, MINB)
     const int h0 = (lane % n_chunks) / cph;  // any chunk of this lane gives the columns
     const int col0 = ((paired && (h0 & 1)) ? stagger_offset : 0) + (lane % cph) * E;
     const int a_width = paired ? head_dim : head_dim >> 1;
+    float wq[E], wk[E];  // NORM: this lane's weights (the same columns for every chunk)
+    if (NORM) {
+        const int off = (lane % cph) * E;
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+            const float4 a = q_weight ? __ldg(reinterpret_cast<const float4*>(q_weight + off + e))
+                                      : make_float4(1.f, 1.f, 1.f, 1.f);
+            const float4 b = k_weight ? __ldg(reinterpret_cast<const float4*>(k_weight + off + e))
+                                      : make_float4(1.f, 1.f, 1.f, 1.f);
+            wq[e] = a.x; wq[e + 1] = a.y; wq[e + 2] = a.z; wq[e + 3] = a.w;
+            wk[e] = b.x; wk[e + 1] = b.y; wk[e + 2] = b.z; wk[e + 3] = b.w;
+        }
+    }
     auto issue = [&](int64_t t, int slot) {
         const uint4* qrow = reinterpret_cast<const uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
         const uint4* krow = reinterpret_cast<const uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
@@ -479,10 +496,30 @@ __global__ void __launch_bounds__(256, MINB)
             table_cs<E, true, NEG>(nullptr, nullptr, lo_row, hi_row, col0, head_dim, cu, su);
         }
         cp_async_wait<R - 1>();  // this lane's chunks of token t have landed
-        if (in_range) {  // a token outside the table is left unchanged
-            uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
-            uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
-            const uint8_t* src = ring + slot * slot_bytes;
+        uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
+        uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
+        const uint8_t* src = ring + slot * slot_bytes;
+        if (NORM) {  // normalised, then rotated when the position is inside the table
+            for (int base = 0; base < n_chunks; base += 32) {
+                const int i = base + lane;
+                const bool have = i < n_chunks;
+                float x[E];
+                Chunk16<T>::to_floats(have ? *reinterpret_cast<const uint4*>(src + i * 16)
+                                           : make_uint4(0u, 0u, 0u, 0u), x);
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+                for (int o = cph >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                const float inv = rsqrtf(ss / static_cast<float>(head_dim) + eps);
+                if (!have) continue;
+                const bool is_q = i < q_chunks;
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[e] = x[e] * inv * (is_q ? wq[e] : wk[e]);
+                const uint4 y = in_range ? Chunk16<T>::template rotate_f<true>(x, cu, su)
+                                         : Chunk16<T>::pack_f(x);
+                if (is_q) qrow[i] = y; else krow[i - q_chunks] = y;
+            }
+        } else if (in_range) {  // a token outside the table is left unchanged
             for (int i = lane; i < n_chunks; i += 32) {
                 const uint4 y = Chunk16<T>::template rotate<true>(
                     *reinterpret_cast<const uint4*>(src + i * 16), cu, su);
@@ -556,12 +593,13 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
 constexpr int kRingDepth = 3;
 constexpr int kRingBlocks = 3;
 
-template <typename T, bool NEG>
+template <typename T, bool NEG, bool NORM>
 static cudaError_t launch_rope_ring(void* q, void* k, const double2* fac, int rows,
                                    const int32_t* positions, int total_tokens, int n_heads,
                                    int n_kv_heads, int head_dim, int paired, int stagger_offset,
+                                   const float* q_weight, const float* k_weight, float eps,
                                    size_t smem, int sms, cudaStream_t stream) {
-    auto kern = rope_ring_kernel<T, NEG, kRingDepth, kRingBlocks>;
+    auto kern = rope_ring_kernel<T, NEG, NORM, kRingDepth, kRingBlocks>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -570,7 +608,7 @@ static cudaError_t launch_rope_ring(void* q, void* k, const double2* fac, int ro
     const unsigned blocks = static_cast<unsigned>(blocks64 < resident ? blocks64 : resident);
     kern<<<blocks, 256, smem, stream>>>(static_cast<T*>(q), static_cast<T*>(k), positions,
                                         total_tokens, n_heads, n_kv_heads, head_dim, paired,
-                                        stagger_offset, rows, fac);
+                                        stagger_offset, rows, fac, q_weight, k_weight, eps);
     return cudaGetLastError();
 }
 
@@ -585,26 +623,22 @@ cudaError_t launch_rope_factored(void* q, void* k, const double2* fac, int rows,
     const bool uniform = (32 % cph == 0) && (!paired || ((32 / cph) % 2 == 0));
     const size_t ring_smem =
         static_cast<size_t>(8) * kRingDepth * (n_heads + n_kv_heads) * cph * 16;
-    if (!norm && uniform && total_tokens > 0 && ring_smem * kRingBlocks <= 220 * 1024) {
+    if (uniform && total_tokens > 0 && ring_smem * kRingBlocks <= 220 * 1024) {
         int dev = 0, sms = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
+#define PHA_RING(T_, NEG_, NORM_)                                                                \
+    launch_rope_ring<T_, NEG_, NORM_>(q, k, fac, rows, positions, total_tokens, n_heads,        \
+                                      n_kv_heads, head_dim, paired, stagger_offset, q_weight,   \
+                                      k_weight, eps, ring_smem, sms, stream)
         if (is_bf16)
-            return neg ? launch_rope_ring<__nv_bfloat16, true>(q, k, fac, rows, positions,
-                                                               total_tokens, n_heads, n_kv_heads,
-                                                               head_dim, paired, stagger_offset,
-                                                               ring_smem, sms, stream)
-                       : launch_rope_ring<__nv_bfloat16, false>(q, k, fac, rows, positions,
-                                                                total_tokens, n_heads, n_kv_heads,
-                                                                head_dim, paired, stagger_offset,
-                                                                ring_smem, sms, stream);
-        return neg ? launch_rope_ring<float, true>(q, k, fac, rows, positions, total_tokens,
-                                                   n_heads, n_kv_heads, head_dim, paired,
-                                                   stagger_offset, ring_smem, sms, stream)
-                   : launch_rope_ring<float, false>(q, k, fac, rows, positions, total_tokens,
-                                                    n_heads, n_kv_heads, head_dim, paired,
-                                                    stagger_offset, ring_smem, sms, stream);
+            return norm ? PHA_RING(__nv_bfloat16, false, true)
+                        : (neg ? PHA_RING(__nv_bfloat16, true, false)
+                               : PHA_RING(__nv_bfloat16, false, false));
+        return norm ? PHA_RING(float, false, true)
+                    : (neg ? PHA_RING(float, true, false) : PHA_RING(float, false, false));
+#undef PHA_RING
     }
     if (norm)
         return launch_rope_impl<true, false, true>(q, k, nullptr, nullptr, rows, width, positions,
