@@ -13,7 +13,8 @@
 // both warpgroups have one tile at every step and every K / V tile is read from HBM once per run.
 //
 // CTA = 12 warps (16 with the value embedding), persistent, one per SM, items in snake order over
-// the longest-first list; the softmax warpgroups run with 200 registers per thread:
+// the longest-first list; the softmax warpgroups run with 200 registers per thread (184 with the
+// value embedding):
 //   warps 0-3, 4-7   softmax warpgroups w = 0, 1: query tiles n (CTA-wide count) with n % 2 == w.
 //                    The whole 128-column S row is loaded from TMEM with one wait; hidden scores
 //                    are set to -inf in registers (per-row bit masks, skipped for 32-column chunks
@@ -46,10 +47,14 @@ constexpr int kBandThreads = 384;
 constexpr int kBandAuxThreads = 512;
 // Register split, per thread: the softmax warpgroups hold a whole 128-column score row. Without
 // the embedding 8 x 200 + 4 x 88 = 1952 <= 12 x 168 (the launch allocation of 384 threads); with
-// it 8 x 200 + 8 x 56 = 2048 <= 16 x 128 (512 threads).
+// it 8 x 184 + 8 x 72 = 2048 <= 16 x 128 (512 threads), so that the adders keep eight 16-byte
+// aux_v loads in flight (measured: 184 / 72 with eight in flight 140 us on the paired workload,
+// 200 / 56 with four 171 us).
 constexpr int kBandRegsSoftmax = 200;
 constexpr int kBandRegsOther = 88;
-constexpr int kBandRegsOtherAux = 56;
+constexpr int kBandRegsSoftmaxAux = 184;
+constexpr int kBandRegsOtherAux = 72;
+constexpr int kBandAuxBatch = 8;  // aux_v loads in flight per adder thread
 
 struct BandBars {
     uint64_t q_full[3], q_empty[3];
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
     const int H = p.heads;
     const int G = p.heads / p.kv_heads;
     static_assert(8 * kBandRegsSoftmax + 4 * kBandRegsOther <= 12 * 168, "register split");
-    static_assert(8 * kBandRegsSoftmax + 8 * kBandRegsOtherAux <= 16 * 128, "register split");
+    static_assert(8 * kBandRegsSoftmaxAux + 8 * kBandRegsOtherAux <= 16 * 128, "register split");
 
     if (warp >= 8) {  // every warp of the third (and fourth) warpgroup, then their roles
         if (AUXV)
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[sv], (vc / S) & 1, abort_flag,
                                                        dev_status));
                 if (!ok) break;
-                add_aux_tile<HD, 128, 4>(smem + L::kOffV + sv * L::kKV, aux, kv_first + s * kBlockN,
+                add_aux_tile<HD, 128, kBandAuxBatch>(smem + L::kOffV + sv * L::kKV, aux, kv_first + s * kBlockN,
                                          gk, p.kv_heads, slots, at);
                 fence_proxy_async_smem();  // the tensor cores read the tile next
                 mbar_arrive(&bars->v_add[sv]);
@@ -323,7 +328,10 @@ __global__ void __launch_bounds__(AUXV ? kBandAuxThreads : kBandThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax of warpgroup w
-        regs_increase<kBandRegsSoftmax>();
+        if (AUXV)
+            regs_increase<kBandRegsSoftmaxAux>();
+        else
+            regs_increase<kBandRegsSoftmax>();
         const int w = warp >> 2;
         const int row = threadIdx.x & 127;  // query row in the tile == TMEM lane
         const int r0 = (warp & 3) * 32;     // first row of this warp
