@@ -16,8 +16,9 @@ F32_REL = 1e-5
 LSE_ABS = 1e-3
 
 
-def run_gpu(w, rope=True, rank=0, inputs=None):
-    """Inputs (CPU tensors) and the GPU outputs (CPU tensors) of one forward over workload w."""
+def run_gpu(w, rope=True, rank=0, inputs=None, rope_tables="stored"):
+    """Inputs (CPU tensors) and the GPU outputs (CPU tensors) of one forward over workload w
+    (RoPE with the stored float32 tables or the factored ones, as bench.py's step)."""
     from paired_heads_b200.runner import AttentionStep, StepShape
 
     inp = inputs if inputs is not None else synth.make_inputs(w, rank=rank)
@@ -25,7 +26,7 @@ def run_gpu(w, rope=True, rank=0, inputs=None):
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     cu, pos = inp["cu_seqlens"].to(dev), inp["positions"].to(dev)
     tab_rows = int(inp["positions"].max()) + 1 if w.total else 1
-    step = AttentionStep(StepShape.of(w, tab_rows), dev)
+    step = AttentionStep(StepShape.of(w, tab_rows), dev, rope_tables=rope_tables)
     if rope:
         step.rope(q, k, pos)
     o, lse = step.attn(q, k, v, cu)

@@ -262,9 +262,11 @@ SCALED = [
 
 @pytest.mark.parametrize("w", SCALED, ids=lambda w: f"{w.name}-w{w.window}-p{int(w.paired)}")
 def test_end_to_end_scaled(w):
-    inp, g = run_gpu(w)
+    inp = synth.make_inputs(w)
     o_ref, lse_ref = run_oracle(w, inp)
-    check(w, g["o"], g["lse"], o_ref, lse_ref)
+    for tables in ("stored", "factored"):  # the two RoPE table forms, then attention
+        _, g = run_gpu(w, inputs=inp, rope_tables=tables)
+        check(w, g["o"], g["lse"], o_ref, lse_ref)
 
 
 FULL = [
@@ -282,7 +284,8 @@ FULL = [
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: f"{w.name}-w{w.window}-p{int(w.paired)}")
 def test_full_size_sampled_rows(w):
-    inp, g = run_gpu(w)
+    # the launch configuration bench.py times: factored RoPE, then attention
+    inp, g = run_gpu(w, rope_tables="factored")
     rows = sample_rows(w, 400)
     o_ref, lse_ref = run_oracle(w, inp, rows=rows)
     o = g["o"].reshape(-1, w.head_dim)[torch.from_numpy(rows)]
