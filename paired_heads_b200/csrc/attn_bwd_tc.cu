@@ -159,7 +159,8 @@ __device__ __forceinline__ void inner_step(const BandItem& it, const OuterTile& 
     }
 }
 
-// Items of the key-major instance: one per kv head (the item of the group's first query head).
+// Items of the key-major instance: one per kv head (the item of the group's first query head);
+// its item walk visits only those (ItemWalk with the head group), so this always holds there.
 template <bool KEYMAJOR>
 __device__ __forceinline__ bool item_used(const BandItem& it, int G) {
     return !KEYMAJOR || it.head % G == 0;
@@ -316,7 +317,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             return true;
         };
         ItemWalk wk;
-        for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+        for (wk.start(items, n_items, KEYMAJOR ? G : 1, H); ok && !wk.done(); wk.advance()) {
             if (!wk.has()) continue;
             const BandItem it = decode_band(wk.cur);
             if (!item_used<KEYMAJOR>(it, G)) continue;
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             FillTrack<KEYMAJOR> ft;
             bool ok = true;
             ItemWalk wk;
-            for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+            for (wk.start(items, n_items, KEYMAJOR ? G : 1, H); ok && !wk.done(); wk.advance()) {
                 if (!wk.has()) continue;
                 const BandItem it = decode_band(wk.cur);
                 if (!item_used<KEYMAJOR>(it, G)) continue;
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         FillTrack<KEYMAJOR> ft;
         bool ok = true;
         ItemWalk wk;
-        for (wk.start(items, n_items); ok && !wk.done(); wk.advance()) {
+        for (wk.start(items, n_items, KEYMAJOR ? G : 1, H); ok && !wk.done(); wk.advance()) {
             if (!wk.has()) continue;
             const BandItem it = decode_band(wk.cur);
             if (!item_used<KEYMAJOR>(it, G)) continue;

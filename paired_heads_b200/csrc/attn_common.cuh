@@ -253,22 +253,33 @@ __device__ __forceinline__ int band_item_index(int k, int n_items) {
     return idx < n_items ? static_cast<int>(idx) : -2;
 }
 
-// Walks this CTA's items in order, keeping the next one's descriptor in flight.
+// Walks this CTA's items in order, keeping the next one's descriptor in flight. With a head group
+// G > 1 (H heads per block of the list, the scheduler's layout) it walks only the items of each
+// group's first head, slot * H + g * G, as one list of n / G items, so that those items, not all
+// of them, are dealt evenly to the CTAs.
 struct ItemWalk {
     const int4* items;
     int n_items, k, idx, nidx;
+    int grp = 1, heads = 1;
     int4 cur, nxt;
-    __device__ __forceinline__ void start(const int4* it, int n) {
+    __device__ __forceinline__ int real(int i) const {
+        if (grp == 1) return i;
+        const int hkv = heads / grp;
+        return (i / hkv) * heads + (i % hkv) * grp;
+    }
+    __device__ __forceinline__ void start(const int4* it, int n, int g = 1, int h = 1) {
         items = it;
-        n_items = n;
+        grp = g;
+        heads = h;
+        n_items = n / g;
         k = 0;
-        idx = band_item_index(0, n);
-        cur = idx >= 0 ? __ldg(items + idx) : make_int4(0, 0, 0, 0);
+        idx = band_item_index(0, n_items);
+        cur = idx >= 0 ? __ldg(items + real(idx)) : make_int4(0, 0, 0, 0);
         prefetch();
     }
     __device__ __forceinline__ void prefetch() {
         nidx = idx == -1 ? -1 : band_item_index(k + 1, n_items);
-        nxt = nidx >= 0 ? __ldg(items + nidx) : make_int4(0, 0, 0, 0);
+        nxt = nidx >= 0 ? __ldg(items + real(nidx)) : make_int4(0, 0, 0, 0);
     }
     __device__ __forceinline__ bool done() const { return idx == -1; }
     __device__ __forceinline__ bool has() const { return idx >= 0; }
