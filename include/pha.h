@@ -144,11 +144,14 @@ pha_status pha_rope_factor_tables(void* factors, size_t bytes, int rows, int hea
  *   cos_tab / sin_tab: the rotation reads only q and k from HBM.
  *   factors: as written by pha_rope_factor_tables for `rows` rows and the same head_dim and
  *   paired, 16-byte aligned, read only. positions index rows [0, rows); a token outside is left
- *   unchanged. Each cosine and sine equals the stored table's float32 value except in the last
- *   bit where the float64 angle-addition result (error about 1e-11 at angles of 1e5) lies that
- *   close to a float32 rounding midpoint; with these values the rotation is correctly rounded as
- *   in pha_rope. Other arguments, layouts and errors: as pha_rope (there is no tab_width;
- *   stagger_offset is 0, or head_dim when paired).
+ *   unchanged. Each cosine and sine equals the stored table's float32 value, or differs from it
+ *   by one unit in the last place next to a float32 rounding midpoint, or, for values very close
+ *   to zero, by the float64 angles' own difference (the two forms round their angles differently:
+ *   at most about 5e-11 at angles of 1.4e5). bf16 results are rounded faithfully (compensated
+ *   float32 arithmetic: the correctly rounded rotation with these values, or next to a bf16
+ *   rounding midpoint its neighbour); float32 results are correctly rounded as in pha_rope.
+ *   Other arguments, layouts and errors: as pha_rope (there is no tab_width; stagger_offset is 0,
+ *   or head_dim when paired).
  */
 pha_status pha_rope_factored(void* q, void* k, const void* factors, int rows,
                              const int32_t* positions, int total_tokens, int n_heads,

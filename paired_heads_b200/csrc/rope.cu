@@ -22,9 +22,10 @@
 // rotation reads only q and k from HBM. Table row p = kRopeLoRows * r + l splits each angle into
 // a coarse part (row kRopeLoRows * r; for a paired row, its even position) and a fine part (row
 // l, either half), and cos(a + b) = cos a cos b - sin a sin b, sin(a + b) = sin a cos b +
-// cos a sin b in float64, rounded once to float32, give the value that the stored table holds
-// except where that float64 result lies within its own error (~1e-11 at angles of 1e5) of a
-// float32 rounding midpoint. This path rounds bf16 results faithfully (compensated float32, see
+// cos a sin b in float64, rounded once to float32, give the value that the stored table holds,
+// or its neighbour next to a float32 rounding midpoint, or (values very close to zero) a value
+// off by the two forms' float64 angle difference (~5e-11 at 1.4e5 rad). This path rounds bf16
+// results faithfully (compensated float32, see
 // rot_pair_bf16_faithful): the correctly rounded value in all but ~1e-5 of the elements, else its
 // neighbour.
 #include <cuda_bf16.h>

@@ -108,3 +108,17 @@ def test_gpus_two_starts_two_ranks():
     assert len(lines) == 1, r.stdout
     d = json.loads(lines[0])
     assert d["world"] == 2 and d["ranks"] == [0, 1]
+
+
+def test_rope_bytes_by_table_form(bench):
+    # stored tables: q and k read and written, plus a cos and a sin row per token; factored tables:
+    # q and k read and written, plus the factor tables once (16 fine rows, one coarse row per 16)
+    w = synth.workload("paired_varlen")
+    qk = 2 * w.total * (w.n_heads + w.n_kv_heads) * w.head_dim * 2
+    assert bench.rope_bytes(w, "stored") == qk + 2 * 4 * w.total * 2 * w.head_dim
+    rows = 131072
+    fac = (16 * w.head_dim + (rows // 16) * (w.head_dim // 2)) * 16
+    assert bench.rope_bytes(w, "factored", rows) == qk + fac
+    g = synth.workload("gpt2")  # unpaired: fine rows hold head_dim / 2 angles
+    qk_g = 2 * g.total * (g.n_heads + g.n_kv_heads) * g.head_dim * 2
+    assert bench.rope_bytes(g, "factored", 1000) == qk_g + (16 * (g.head_dim // 2) + 63 * (g.head_dim // 2)) * 16
