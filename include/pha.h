@@ -147,9 +147,8 @@ pha_status pha_rope_factor_tables(void* factors, size_t bytes, int rows, int hea
  *   unchanged. Each cosine and sine equals the stored table's float32 value, or differs from it
  *   by one unit in the last place next to a float32 rounding midpoint, or, for values very close
  *   to zero, by the float64 angles' own difference (the two forms round their angles differently:
- *   at most about 5e-11 at angles of 1.4e5). bf16 results are rounded faithfully (compensated
- *   float32 arithmetic: the correctly rounded rotation with these values, or next to a bf16
- *   rounding midpoint its neighbour); float32 results are correctly rounded as in pha_rope.
+ *   at most about 5e-11 at angles of 1.4e5). With these values the rotation is correctly rounded
+ *   as in pha_rope (bf16: compensated float32 arithmetic, float64 next to a rounding midpoint).
  *   Other arguments, layouts and errors: as pha_rope (there is no tab_width; stagger_offset is 0,
  *   or head_dim when paired).
  */

@@ -24,10 +24,9 @@
 // l, either half), and cos(a + b) = cos a cos b - sin a sin b, sin(a + b) = sin a cos b +
 // cos a sin b in float64, rounded once to float32, give the value that the stored table holds,
 // or its neighbour next to a float32 rounding midpoint, or (values very close to zero) a value
-// off by the two forms' float64 angle difference (~5e-11 at 1.4e5 rad). This path rounds bf16
-// results faithfully (compensated float32, see
-// rot_pair_bf16_faithful): the correctly rounded value in all but ~1e-5 of the elements, else its
-// neighbour.
+// off by the two forms' float64 angle difference (~5e-11 at 1.4e5 rad). This path rotates with
+// compensated float32 arithmetic and a cheaper exactness test (rot_chunk_bf16_comp); its bf16
+// results are correctly rounded too.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -138,21 +137,52 @@ __device__ __forceinline__ uint32_t rot_pair_bf16(float x0, float x1, float c, f
     return bf16_bits_rne(e0) | (bf16_bits_rne(e1) << 16);
 }
 
-// One rotated pair, faithfully rounded with float32 arithmetic (the factored-table path): the
-// products s*x are split exactly into t = fl(s*x) and e = s*x - t (one fma each), so
-// y = fl(fl(c*x' + t) + e) is within about one float32 ulp of the exact value even under
-// cancellation, and its bf16 rounding is the correctly rounded value or, when the exact value lies
-// that close to a bf16 rounding midpoint, its neighbour (at most one bf16 ulp away).
-__device__ __forceinline__ uint32_t rot_pair_bf16_faithful(float x0, float x1, float c, float s) {
-    const uint64_t xs = f32x2(x1, x0);
-    const uint64_t t2 = mul_f32x2(f32x2(-s, s), xs);          // fl(-s*x1), fl(s*x0)
-    const uint64_t tn = mul_f32x2(f32x2(s, -s), xs);          // -t2, exactly
-    const uint64_t e2 = fma_f32x2(f32x2(-s, s), xs, tn);      // the exact rounding errors
-    const uint64_t y2 = add_f32x2(fma_f32x2(f32x2(c, c), f32x2(x0, x1), t2), e2);
-    float y0, y1;
-    f32x2_split(y2, y0, y1);
-    return pack_bf16x2(y0, y1);
+// Correctly rounded rotation from compensated float32 arithmetic (the factored-table path): the
+// products s*x are split exactly into t = fl(s*x) and e = s*x - t (one fma each), and
+// y = fl(fl(c*x' + t) + e) is within one float32 ulp of the exact value even under cancellation
+// (where fl(c*x' + t) is exact). When y lies more than eight float32 ulps from a bf16 rounding
+// midpoint, rounding y gives the bf16 of the exact value; otherwise the pair is recomputed in
+// float64 as in rot_pair_bf16 (measured: this test and its branch cost about 13 us of the 84 us
+// factored RoPE on the paired workload; testing a whole chunk at once, or rounding y +- 8 ulps
+// twice and comparing, measured slower).
+
+// The rare pair near a bf16 midpoint: float64 (exact products), one rounding. Out of line, so
+// that the fast path of the rotation loop stays small.
+__device__ __noinline__ uint32_t rot_pair_bf16_f64(float x0, float x1, float c, float s) {
+    const double e0 = fma(static_cast<double>(c), static_cast<double>(x0),
+                          -static_cast<double>(s) * static_cast<double>(x1));
+    const double e1 = fma(static_cast<double>(c), static_cast<double>(x1),
+                          static_cast<double>(s) * static_cast<double>(x0));
+    return bf16_bits_rne(e0) | (bf16_bits_rne(e1) << 16);
 }
+
+// More than eight float32 ulps from the bf16 rounding midpoint of y's binade (the low 16 bits
+// outside 0x8000 +- 8): y and anything within one ulp of it round to the same bf16.
+__device__ __forceinline__ bool far_from_bf16_midpoint(float y) {
+    return ((__float_as_uint(y) + 8u) & 0xFFF0u) != 0x8000u;
+}
+
+// Four pairs (one 16-byte bf16 chunk), each tested on its own; a pair near a bf16 rounding
+// midpoint takes the float64 path.
+__device__ __forceinline__ uint4 rot_chunk_bf16_comp(const float (&x)[8], const float (&c)[8],
+                                                     const float (&s)[8]) {
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float x0 = x[2 * e], x1 = x[2 * e + 1], cc = c[2 * e], ss = s[2 * e];
+        const uint64_t xs = f32x2(x1, x0);
+        const uint64_t t2 = mul_f32x2(f32x2(-ss, ss), xs);          // fl(-s*x1), fl(s*x0)
+        const uint64_t tn = mul_f32x2(f32x2(ss, -ss), xs);          // -t2, exactly
+        const uint64_t e2 = fma_f32x2(f32x2(-ss, ss), xs, tn);      // the exact rounding errors
+        float y0, y1;
+        f32x2_split(add_f32x2(fma_f32x2(f32x2(cc, cc), f32x2(x0, x1), t2), e2), y0, y1);
+        o[e] = (far_from_bf16_midpoint(y0) && far_from_bf16_midpoint(y1))
+                   ? pack_bf16x2(y0, y1)
+                   : rot_pair_bf16_f64(x0, x1, cc, ss);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 
 // 16-byte chunks of a row: 8 bf16 (4 pairs) or 4 f32 (2 pairs). to_floats gives the exact values;
 // rotate_f rotates E float values with the chunk's table values c[j], s[j] (j = element within
@@ -171,28 +201,32 @@ struct Chunk16<__nv_bfloat16> {
             x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
         }
     }
-    template <bool FAITHFUL = false>
+    template <bool COMP = false>
     __device__ static uint4 rotate_f(const float (&x)[E], const float (&c)[E], const float (&s)[E]) {
+        if (COMP) return rot_chunk_bf16_comp(x, c, s);
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)  // both members of a pair share one angle: c[2e] == c[2e+1]
-            o[e] = FAITHFUL ? rot_pair_bf16_faithful(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e])
-                            : rot_pair_bf16(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e]);
+            o[e] = rot_pair_bf16(x[2 * e], x[2 * e + 1], c[2 * e], s[2 * e]);
         return make_uint4(o[0], o[1], o[2], o[3]);
     }
     __device__ static uint4 pack_f(const float (&x)[E]) {
         return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                           pack_bf16x2(x[6], x[7]));
     }
-    template <bool FAITHFUL = false>
+    template <bool COMP = false>
     __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
+        if (COMP) {
+            float x[E];
+            to_floats(a, x);
+            return rot_chunk_bf16_comp(x, c, s);
+        }
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
-            o[e] = FAITHFUL ? rot_pair_bf16_faithful(x0, x1, c[2 * e], s[2 * e])
-                            : rot_pair_bf16(x0, x1, c[2 * e], s[2 * e]);
+            o[e] = rot_pair_bf16(x0, x1, c[2 * e], s[2 * e]);
         }
         return make_uint4(o[0], o[1], o[2], o[3]);
     }
@@ -207,7 +241,7 @@ struct Chunk16<float> {
         x[2] = __uint_as_float(a.z);
         x[3] = __uint_as_float(a.w);
     }
-    template <bool FAITHFUL = false>  // float32 results are always correctly rounded
+    template <bool COMP = false>  // float32 results: always float64, correctly rounded
     __device__ static uint4 rotate_f(const float (&x)[E], const float (&c)[E], const float (&s)[E]) {
         float y[E];
 #pragma unroll
@@ -225,7 +259,7 @@ struct Chunk16<float> {
         return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
                           __float_as_uint(x[3]));
     }
-    template <bool FAITHFUL = false>
+    template <bool COMP = false>
     __device__ static uint4 rotate(uint4 a, const float (&c)[E], const float (&s)[E]) {
         float x[E];
         to_floats(a, x);
@@ -292,7 +326,7 @@ __device__ __forceinline__ void table_cs(const float* crow, const float* srow,
 // NEG: the backward of RoPE (the gradient with respect to the input is the transposed rotation,
 // i.e. the rotation by -angle): the sines enter negated, which is exact.
 // FACT: factored tables (fac; cos_tab / sin_tab unused, tab_rows = the rows they stand for), and
-// bf16 results faithfully rounded by rot_pair_bf16_faithful instead of correctly rounded.
+// the bf16 rotation of rot_chunk_bf16_comp.
 template <typename T, bool NORM, bool NEG = false, bool FACT = false>
 __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_kernel(T* __restrict__ q, T* __restrict__ k,
                                                    const float* __restrict__ cos_tab,

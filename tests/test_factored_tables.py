@@ -38,10 +38,12 @@ def test_angle_addition_matches_direct_tables(paired, hd):
             assert np.mean(d == 0) > 0.9999, float(np.mean(d == 0))
 
 
-def test_compensated_rotation_is_faithful():
+def test_compensated_rotation_with_midpoint_test_is_exact():
     # the factored path's bf16 rotation: t = fl(s x1), e = s x1 - t (exact), y = fl(fl(c x0 - t) - e)
-    # rounded once to bf16 is within one bf16 ulp of the correctly rounded rotation, and equal to it
-    # in all but a small fraction of the elements; plain float32 (no e) is not within one ulp
+    # is within one float32 ulp of the exact value, so rounded once to bf16 it is within one bf16
+    # ulp of the correctly rounded rotation, and wherever y is more than eight float32 ulps from a
+    # bf16 rounding midpoint (the kernel's test; the rest goes to float64) it is that value exactly;
+    # plain float32 (no e) is not within one bf16 ulp under cancellation
     rng = np.random.default_rng(0)
     n = 400000
 
@@ -70,4 +72,8 @@ def test_compensated_rotation_is_faithful():
     ulp = np.ldexp(1.0, np.frexp(np.maximum(np.abs(exact), 1e-30))[1] - 8)
     assert np.max(np.abs(faithful - exact) / ulp) <= 1.0
     assert np.mean(faithful == exact) > 0.9999
+    yb = fl32(fl32(c * x0 - t) - e).astype(np.float32).view(np.uint32).astype(np.int64)
+    far = ((yb + 8) & 0xFFF0) != 0x8000
+    assert np.mean(far) > 0.999
+    assert np.all(faithful[far] == exact[far])          # the test never passes a wrong rounding
     assert np.max(np.abs(plain - exact) / ulp) > 1.0   # the compensation is what keeps one ulp
