@@ -624,9 +624,14 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
     return cudaGetLastError();
 }
 
-// Ring depth and resident blocks of rope_ring_kernel.
-constexpr int kRingDepth = 3;
-constexpr int kRingBlocks = 3;
+// Ring depth and resident blocks of rope_ring_kernel: two token slots per warp and four blocks per
+// SM (64 registers) for the rotation, three and three (80 registers) with the norm (measured on
+// the paired workload: depth 2 / 4 blocks 80 us, depth 3 / 3 blocks 84 us, depth 4 / 2 blocks 98
+// us).
+template <bool NORM>
+constexpr int ring_depth() { return NORM ? 3 : 2; }
+template <bool NORM>
+constexpr int ring_blocks() { return NORM ? 3 : 4; }
 
 template <typename T, bool NEG, bool NORM>
 static cudaError_t launch_rope_ring(void* q, void* k, const double2* fac, int rows,
@@ -634,12 +639,12 @@ static cudaError_t launch_rope_ring(void* q, void* k, const double2* fac, int ro
                                    int n_kv_heads, int head_dim, int paired, int stagger_offset,
                                    const float* q_weight, const float* k_weight, float eps,
                                    size_t smem, int sms, cudaStream_t stream) {
-    auto kern = rope_ring_kernel<T, NEG, NORM, kRingDepth, kRingBlocks>;
+    auto kern = rope_ring_kernel<T, NEG, NORM, ring_depth<NORM>(), ring_blocks<NORM>()>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
-    const int64_t resident = static_cast<int64_t>(sms) * kRingBlocks;
+    const int64_t resident = static_cast<int64_t>(sms) * ring_blocks<NORM>();
     const unsigned blocks = static_cast<unsigned>(blocks64 < resident ? blocks64 : resident);
     kern<<<blocks, 256, smem, stream>>>(static_cast<T*>(q), static_cast<T*>(k), positions,
                                         total_tokens, n_heads, n_kv_heads, head_dim, paired,
@@ -656,9 +661,10 @@ cudaError_t launch_rope_factored(void* q, void* k, const double2* fac, int rows,
     // the ring kernel when a lane's chunks share table columns and its shared memory fits
     const int cph = head_dim / (is_bf16 ? 8 : 4);
     const bool uniform = (32 % cph == 0) && (!paired || ((32 / cph) % 2 == 0));
-    const size_t ring_smem =
-        static_cast<size_t>(8) * kRingDepth * (n_heads + n_kv_heads) * cph * 16;
-    if (uniform && total_tokens > 0 && ring_smem * kRingBlocks <= 220 * 1024) {
+    const size_t slots = static_cast<size_t>(8) * (n_heads + n_kv_heads) * cph * 16;  // per depth
+    const size_t ring_smem = slots * (norm ? ring_depth<true>() : ring_depth<false>());
+    const int ring_bl = norm ? ring_blocks<true>() : ring_blocks<false>();
+    if (uniform && total_tokens > 0 && ring_smem * ring_bl <= 220 * 1024) {
         int dev = 0, sms = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
