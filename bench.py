@@ -373,9 +373,12 @@ def main():
                if tc_bwd else None}
 
     # ---- end to end through the public API with host buffers. Documents are independent, so the
-    # step is issued in chunks of whole documents on two streams: the host->device copy of one
-    # chunk overlaps the kernels and the device->host copy of the previous one. Every input byte
-    # is copied in and every output byte copied out within each timed step.
+    # step is issued in chunks of whole documents on three streams, one a stage: host->device
+    # copies, kernels, device->host copies, chained per chunk by events. The copy-in stream thus
+    # never waits for a kernel or a copy-out (the host->device link is the bound), and the
+    # copy-out of one chunk runs beside the copy-in of the next. Every input byte is copied in and
+    # every output byte copied out within each timed step; a step starts after the previous one's
+    # copies out.
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "cu_seqlens", "positions")}
     if args.aux_v:
         host["aux_v"] = aux.cpu().pin_memory()
@@ -383,7 +386,7 @@ def main():
     lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
     cu_h = host["cu_seqlens"].tolist()
     chunks = doc_chunks(cu_h, max(1, min(8, w.batch)))
-    streams = [torch.cuda.Stream(dev) for _ in range(2)]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     parts = []
     for (a0, a1) in chunks:
         t0, t1 = cu_h[a0], cu_h[a1]
@@ -397,13 +400,18 @@ def main():
         hsrc["cu_seqlens"] = (host["cu_seqlens"][a0:a1 + 1] - t0).pin_memory()
         parts.append((st_, bufs, hsrc, t0, t1))
 
+    ev_in = [torch.cuda.Event() for _ in parts]
+    ev_k = [torch.cuda.Event() for _ in parts]
+
     def e2e_step(first_event):
+        s_in.wait_event(first_event)
         for c, (st_, bufs, hsrc, t0, t1) in enumerate(parts):
-            sc = streams[c % 2]
-            sc.wait_event(first_event)
-            with torch.cuda.stream(sc):
+            with torch.cuda.stream(s_in):
                 for n, t in bufs.items():
                     t.copy_(hsrc[n], non_blocking=True)
+                ev_in[c].record(s_in)
+            s_comp.wait_event(ev_in[c])
+            with torch.cuda.stream(s_comp):
                 if args.qk_norm:
                     st_.norm_rope(bufs["q"], bufs["k"], bufs["positions"])
                 else:
@@ -412,9 +420,12 @@ def main():
                     o, lse = st_.attn_aux_v(bufs["q"], bufs["k"], bufs["v"], bufs["aux_v"], bufs["cu_seqlens"])
                 else:
                     o, lse = st_.attn(bufs["q"], bufs["k"], bufs["v"], bufs["cu_seqlens"])
+                ev_k[c].record(s_comp)
+            s_out.wait_event(ev_k[c])
+            with torch.cuda.stream(s_out):
                 o_host[t0:t1].copy_(o, non_blocking=True)
                 lse_host[t0:t1].copy_(lse, non_blocking=True)
-        for sc in streams:
+        for sc in (s_in, s_comp, s_out):
             stream.wait_stream(sc)
 
     for _ in range(3):
@@ -513,8 +524,9 @@ def main():
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "chunks": len(parts),
-                "how": "public API from pinned host buffers, whole-document chunks on two streams "
-                       "(host->device copies overlap the previous chunk's kernels and copy-out)"},
+                "how": "public API from pinned host buffers, whole-document chunks on three "
+                       "streams (copy-in, kernels, copy-out, chained by events: a chunk's copy-in "
+                       "overlaps the previous chunks' kernels and copy-out)"},
         "gpu_launches": 3 * args.steps,
         "work_items": n_items,
         "clocks": clk,

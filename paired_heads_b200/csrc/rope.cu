@@ -142,8 +142,8 @@ __device__ __forceinline__ uint32_t rot_pair_bf16(float x0, float x1, float c, f
 // y = fl(fl(c*x' + t) + e) is within one float32 ulp of the exact value even under cancellation
 // (where fl(c*x' + t) is exact). When y lies more than eight float32 ulps from a bf16 rounding
 // midpoint, rounding y gives the bf16 of the exact value; otherwise the pair is recomputed in
-// float64 as in rot_pair_bf16 (measured: this test and its branch cost about 13 us of the 84 us
-// factored RoPE on the paired workload; testing a whole chunk at once, or rounding y +- 8 ulps
+// float64 as in rot_pair_bf16 (measured on the paired workload: the test and its branch cost
+// about 7 us of the 78 us factored RoPE; testing a whole chunk at once, or rounding y +- 8 ulps
 // twice and comparing, measured slower).
 
 // The rare pair near a bf16 midpoint: float64 (exact products), one rounding. Out of line, so
@@ -157,28 +157,47 @@ __device__ __noinline__ uint32_t rot_pair_bf16_f64(float x0, float x1, float c, 
 }
 
 // More than eight float32 ulps from the bf16 rounding midpoint of y's binade (the low 16 bits
-// outside 0x8000 +- 8): y and anything within one ulp of it round to the same bf16.
+// outside 0x8000 +- 8): y and anything within one ulp of it round to the same bf16. Adding 0x8008
+// maps that window of the low 16 bits onto 0x0000..0x000F.
 __device__ __forceinline__ bool far_from_bf16_midpoint(float y) {
-    return ((__float_as_uint(y) + 8u) & 0xFFF0u) != 0x8000u;
+    return ((__float_as_uint(y) + 0x8008u) & 0xFFF0u) != 0u;
 }
 
-// Four pairs (one 16-byte bf16 chunk), each tested on its own; a pair near a bf16 rounding
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Four pairs (one 16-byte bf16 chunk) in two groups of two pairs a, b, each packed by member:
+// X0 = (x0 of a, x0 of b), X1 = (x1 of a, x1 of b), C and S their table values. Then
+//   y0 = c x0 - s x1:  T = fl(-S X1),  E = S X1 + T exactly (the rounding error of S X1),
+//                      Y0 = fl(fl(C X0 + T) - E)
+//   y1 = c x1 + s x0:  T' = fl(S X0), E' = -S X0 + T' exactly,  Y1 = fl(fl(C X1 + T') - E')
+// (four packed operations a pair). Each pair is tested on its own; a pair near a bf16 rounding
 // midpoint takes the float64 path.
 __device__ __forceinline__ uint4 rot_chunk_bf16_comp(const float (&x)[8], const float (&c)[8],
                                                      const float (&s)[8]) {
     uint32_t o[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float x0 = x[2 * e], x1 = x[2 * e + 1], cc = c[2 * e], ss = s[2 * e];
-        const uint64_t xs = f32x2(x1, x0);
-        const uint64_t t2 = mul_f32x2(f32x2(-ss, ss), xs);          // fl(-s*x1), fl(s*x0)
-        const uint64_t tn = mul_f32x2(f32x2(ss, -ss), xs);          // -t2, exactly
-        const uint64_t e2 = fma_f32x2(f32x2(-ss, ss), xs, tn);      // the exact rounding errors
-        float y0, y1;
-        f32x2_split(add_f32x2(fma_f32x2(f32x2(cc, cc), f32x2(x0, x1), t2), e2), y0, y1);
-        o[e] = (far_from_bf16_midpoint(y0) && far_from_bf16_midpoint(y1))
-                   ? pack_bf16x2(y0, y1)
-                   : rot_pair_bf16_f64(x0, x1, cc, ss);
+    for (int g = 0; g < 2; ++g) {
+        const int a = 2 * g, b = 2 * g + 1;  // pairs; pair p holds x[2p], x[2p + 1], angle c[2p]
+        const uint64_t x0 = f32x2(x[2 * a], x[2 * b]), x1 = f32x2(x[2 * a + 1], x[2 * b + 1]);
+        const uint64_t cc = f32x2(c[2 * a], c[2 * b]), ss = f32x2(s[2 * a], s[2 * b]);
+        const uint64_t sn = f32x2(-s[2 * a], -s[2 * b]);
+        const uint64_t t0 = mul_f32x2(sn, x1);
+        const uint64_t y0 = sub_f32x2(fma_f32x2(cc, x0, t0), fma_f32x2(ss, x1, t0));
+        const uint64_t t1 = mul_f32x2(ss, x0);
+        const uint64_t y1 = sub_f32x2(fma_f32x2(cc, x1, t1), fma_f32x2(sn, x0, t1));
+        float y0a, y0b, y1a, y1b;
+        f32x2_split(y0, y0a, y0b);
+        f32x2_split(y1, y1a, y1b);
+        o[a] = (far_from_bf16_midpoint(y0a) && far_from_bf16_midpoint(y1a))
+                   ? pack_bf16x2(y0a, y1a)
+                   : rot_pair_bf16_f64(x[2 * a], x[2 * a + 1], c[2 * a], s[2 * a]);
+        o[b] = (far_from_bf16_midpoint(y0b) && far_from_bf16_midpoint(y1b))
+                   ? pack_bf16x2(y0b, y1b)
+                   : rot_pair_bf16_f64(x[2 * b], x[2 * b + 1], c[2 * b], s[2 * b]);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -460,28 +479,33 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_
     }
 }
 
-// Factored-table rotation (no norm) with the tokens' q and k rows staged in shared memory: each
-// warp keeps a private ring of R token slots, and each lane copies its own 16-byte chunks of the
-// token R - 1 steps ahead into it with cp.async, so R - 1 tokens of HBM reads per warp are in
-// flight without holding registers; before a token is rotated the lane waits for its own copy
-// group (a hardware wait) and reads back only the chunks it copied (no barrier). Used when every
-// chunk of a lane sits at the same table columns (as in rope_kernel's uniform case).
+// Factored-table rotation with the tokens' q and k rows staged in shared memory: each warp keeps a
+// private ring of R slots, and each lane copies its own 16-byte chunks of the unit R - 1 steps
+// ahead into it with cp.async, so R - 1 units of HBM reads per warp are in flight without holding
+// registers; before a unit is rotated the lane waits for its own copy group (a hardware wait) and
+// reads back only the chunks it copied (no barrier). A unit is a token's q and k chunks, or, when
+// a token is too wide for the ring, one of its n_seg segments of seg chunks (seg a multiple of 32,
+// so that a lane's chunks keep their table columns and a head row stays inside one 32-chunk
+// round). Used when every chunk of a lane sits at the same table columns (as in rope_kernel's
+// uniform case).
 // NORM: the QK RMS-norm of each head row first, as in rope_kernel (the row's chunks sit on cph
 // consecutive lanes of one 32-chunk round, whose lanes all take part in the shuffles).
-template <typename T, bool NEG, bool NORM, int R, int MINB>
+template <typename T, bool NEG, bool NORM, bool SEG, int R, int MINB>
 __global__ void __launch_bounds__(256, MINB)
     rope_ring_kernel(T* __restrict__ q, T* __restrict__ k, const int32_t* __restrict__ positions,
                      int64_t total_tokens, int n_heads, int n_kv_heads, int head_dim, int paired,
                      int stagger_offset, int tab_rows, const double2* __restrict__ fac,
                      const float* __restrict__ q_weight, const float* __restrict__ k_weight,
-                     float eps) {
+                     float eps, int n_seg, int seg) {
     extern __shared__ __align__(16) uint8_t ring_smem[];
     constexpr int E = Chunk16<T>::E;
     const int cph = head_dim / E;
     const int q_chunks = n_heads * cph;
     const int n_chunks = q_chunks + n_kv_heads * cph;
     const int lane = threadIdx.x & 31;
-    const int slot_bytes = n_chunks * 16;
+    if (!SEG) n_seg = 1, seg = n_chunks;  // one unit a token: the index arithmetic folds away
+    const int slot_bytes = seg * 16;
+    const int64_t n_units = total_tokens * n_seg;
     uint8_t* ring = ring_smem + (threadIdx.x >> 5) * R * slot_bytes;
     const int64_t warp0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -501,27 +525,35 @@ __global__ void __launch_bounds__(256, MINB)
             wk[e] = b.x; wk[e + 1] = b.y; wk[e + 2] = b.z; wk[e + 3] = b.w;
         }
     }
-    auto issue = [&](int64_t t, int slot) {
+    // unit u: token u / n_seg, chunks [c0, c1) with c0 = (u % n_seg) * seg
+    auto token_of = [&](int64_t u) { return SEG ? u / n_seg : u; };
+    auto issue = [&](int64_t u, int slot) {
+        const int64_t t = token_of(u);
+        const int c0 = SEG ? static_cast<int>(u - t * n_seg) * seg : 0;
+        const int c1 = SEG ? min(c0 + seg, n_chunks) : n_chunks;
         const uint4* qrow = reinterpret_cast<const uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
         const uint4* krow = reinterpret_cast<const uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
         uint8_t* dst = ring + slot * slot_bytes;
-        for (int i = lane; i < n_chunks; i += 32)
-            cp_async_16(dst + i * 16, i < q_chunks ? qrow + i : krow + (i - q_chunks));
+        for (int i = c0 + lane; i < c1; i += 32)
+            cp_async_16(dst + (i - c0) * 16, i < q_chunks ? qrow + i : krow + (i - q_chunks));
     };
 #pragma unroll
     for (int r = 0; r < R - 1; ++r) {
-        const int64_t t = warp0 + r * n_warps;
-        if (t < total_tokens) issue(t, r);
+        const int64_t u = warp0 + r * n_warps;
+        if (u < n_units) issue(u, r);
         cp_async_commit();
     }
-    int pos_next = warp0 < total_tokens ? __ldg(positions + warp0) : 0;
+    int pos_next = warp0 < n_units ? __ldg(positions + token_of(warp0)) : 0;
     int slot = 0;
-    for (int64_t t = warp0; t < total_tokens; t += n_warps) {
-        const int64_t ta = t + (R - 1) * n_warps;
-        if (ta < total_tokens) issue(ta, (slot + R - 1) % R);  // the slot read last step
+    for (int64_t u = warp0; u < n_units; u += n_warps) {
+        const int64_t ua = u + (R - 1) * n_warps;
+        if (ua < n_units) issue(ua, (slot + R - 1) % R);  // the slot read last step
         cp_async_commit();
+        const int64_t t = token_of(u);
+        const int c0 = SEG ? static_cast<int>(u - t * n_seg) * seg : 0;
+        const int c1 = SEG ? min(c0 + seg, n_chunks) : n_chunks;
         const int pos = pos_next;
-        if (t + n_warps < total_tokens) pos_next = __ldg(positions + t + n_warps);
+        if (u + n_warps < n_units) pos_next = __ldg(positions + token_of(u + n_warps));
         const bool in_range = pos >= 0 && pos < tab_rows;
         float cu[E], su[E];
         if (in_range) {
@@ -530,16 +562,16 @@ __global__ void __launch_bounds__(256, MINB)
                 fac + kRopeLoRows * a_width + static_cast<int64_t>(pos / kRopeLoRows) * (head_dim >> 1);
             table_cs<E, true, NEG>(nullptr, nullptr, lo_row, hi_row, col0, head_dim, cu, su);
         }
-        cp_async_wait<R - 1>();  // this lane's chunks of token t have landed
+        cp_async_wait<R - 1>();  // this lane's chunks of unit u have landed
         uint4* qrow = reinterpret_cast<uint4*>(q + t * n_heads * static_cast<int64_t>(head_dim));
         uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
         const uint8_t* src = ring + slot * slot_bytes;
         if (NORM) {  // normalised, then rotated when the position is inside the table
-            for (int base = 0; base < n_chunks; base += 32) {
+            for (int base = c0; base < c1; base += 32) {
                 const int i = base + lane;
-                const bool have = i < n_chunks;
+                const bool have = i < c1;
                 float x[E];
-                Chunk16<T>::to_floats(have ? *reinterpret_cast<const uint4*>(src + i * 16)
+                Chunk16<T>::to_floats(have ? *reinterpret_cast<const uint4*>(src + (i - c0) * 16)
                                            : make_uint4(0u, 0u, 0u, 0u), x);
                 float ss = 0.f;
 #pragma unroll
@@ -555,9 +587,9 @@ __global__ void __launch_bounds__(256, MINB)
                 if (is_q) qrow[i] = y; else krow[i - q_chunks] = y;
             }
         } else if (in_range) {  // a token outside the table is left unchanged
-            for (int i = lane; i < n_chunks; i += 32) {
+            for (int i = c0 + lane; i < c1; i += 32) {
                 const uint4 y = Chunk16<T>::template rotate<true>(
-                    *reinterpret_cast<const uint4*>(src + i * 16), cu, su);
+                    *reinterpret_cast<const uint4*>(src + (i - c0) * 16), cu, su);
                 if (i < q_chunks) qrow[i] = y; else krow[i - q_chunks] = y;
             }
         }
@@ -624,31 +656,34 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
     return cudaGetLastError();
 }
 
-// Ring depth and resident blocks of rope_ring_kernel: two token slots per warp and four blocks per
-// SM (64 registers) for the rotation, three and three (80 registers) with the norm (measured on
-// the paired workload: depth 2 / 4 blocks 80 us, depth 3 / 3 blocks 84 us, depth 4 / 2 blocks 98
-// us).
+// Ring depth and resident blocks of rope_ring_kernel: two slots per warp and three blocks per SM
+// (85 registers) for the rotation, three and three with the norm (measured on the paired
+// workload: depth 2 at 4 blocks with 64 registers 80 us, 84 us once the packed rotation needed
+// more registers than that; depth 2 at 3 blocks 78 us; depth 3 / 3 blocks 84 us, depth 4 / 2
+// blocks 98 us with an earlier rotation).
 template <bool NORM>
 constexpr int ring_depth() { return NORM ? 3 : 2; }
 template <bool NORM>
-constexpr int ring_blocks() { return NORM ? 3 : 4; }
+constexpr int ring_blocks() { return 3; }
 
-template <typename T, bool NEG, bool NORM>
+template <typename T, bool NEG, bool NORM, bool SEG>
 static cudaError_t launch_rope_ring(void* q, void* k, const double2* fac, int rows,
                                    const int32_t* positions, int total_tokens, int n_heads,
                                    int n_kv_heads, int head_dim, int paired, int stagger_offset,
                                    const float* q_weight, const float* k_weight, float eps,
-                                   size_t smem, int sms, cudaStream_t stream) {
-    auto kern = rope_ring_kernel<T, NEG, NORM, ring_depth<NORM>(), ring_blocks<NORM>()>;
+                                   int n_seg, int seg, int sms, cudaStream_t stream) {
+    auto kern = rope_ring_kernel<T, NEG, NORM, SEG, ring_depth<NORM>(), ring_blocks<NORM>()>;
+    const size_t smem = static_cast<size_t>(8) * ring_depth<NORM>() * seg * 16;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int64_t blocks64 = (static_cast<int64_t>(total_tokens) + 7) / 8;
+    const int64_t blocks64 = (static_cast<int64_t>(total_tokens) * n_seg + 7) / 8;
     const int64_t resident = static_cast<int64_t>(sms) * ring_blocks<NORM>();
     const unsigned blocks = static_cast<unsigned>(blocks64 < resident ? blocks64 : resident);
     kern<<<blocks, 256, smem, stream>>>(static_cast<T*>(q), static_cast<T*>(k), positions,
                                         total_tokens, n_heads, n_kv_heads, head_dim, paired,
-                                        stagger_offset, rows, fac, q_weight, k_weight, eps);
+                                        stagger_offset, rows, fac, q_weight, k_weight, eps, n_seg,
+                                        seg);
     return cudaGetLastError();
 }
 
@@ -658,21 +693,32 @@ cudaError_t launch_rope_factored(void* q, void* k, const double2* fac, int rows,
                                  int stagger_offset, bool norm, bool neg, const float* q_weight,
                                  const float* k_weight, float eps, cudaStream_t stream) {
     const int width = paired ? 2 * head_dim : head_dim;
-    // the ring kernel when a lane's chunks share table columns and its shared memory fits
+    // the ring kernel when a lane's chunks share table columns; a token wider than the ring's
+    // slot (220 KB of shared memory per SM at the kernel's depth and blocks per SM) is split into
+    // segments of a multiple of 32 chunks
     const int cph = head_dim / (is_bf16 ? 8 : 4);
     const bool uniform = (32 % cph == 0) && (!paired || ((32 / cph) % 2 == 0));
-    const size_t slots = static_cast<size_t>(8) * (n_heads + n_kv_heads) * cph * 16;  // per depth
-    const size_t ring_smem = slots * (norm ? ring_depth<true>() : ring_depth<false>());
-    const int ring_bl = norm ? ring_blocks<true>() : ring_blocks<false>();
-    if (uniform && total_tokens > 0 && ring_smem * ring_bl <= 220 * 1024) {
+    if (uniform && total_tokens > 0) {
+        const int n_chunks = (n_heads + n_kv_heads) * cph;
+        const int per_chunk = 8 * 16 * (norm ? ring_depth<true>() * ring_blocks<true>()
+                                             : ring_depth<false>() * ring_blocks<false>());
+        const int seg_max = (220 * 1024 / per_chunk) / 32 * 32;
+        int n_seg = 1, seg = n_chunks;
+        if (n_chunks > seg_max) {
+            n_seg = (n_chunks + seg_max - 1) / seg_max;
+            seg = ((n_chunks + n_seg - 1) / n_seg + 31) / 32 * 32;
+        }
         int dev = 0, sms = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
 #define PHA_RING(T_, NEG_, NORM_)                                                                \
-    launch_rope_ring<T_, NEG_, NORM_>(q, k, fac, rows, positions, total_tokens, n_heads,        \
-                                      n_kv_heads, head_dim, paired, stagger_offset, q_weight,   \
-                                      k_weight, eps, ring_smem, sms, stream)
+    (n_seg > 1 ? launch_rope_ring<T_, NEG_, NORM_, true>(                                       \
+                     q, k, fac, rows, positions, total_tokens, n_heads, n_kv_heads, head_dim,   \
+                     paired, stagger_offset, q_weight, k_weight, eps, n_seg, seg, sms, stream)  \
+               : launch_rope_ring<T_, NEG_, NORM_, false>(                                      \
+                     q, k, fac, rows, positions, total_tokens, n_heads, n_kv_heads, head_dim,   \
+                     paired, stagger_offset, q_weight, k_weight, eps, n_seg, seg, sms, stream))
         if (is_bf16)
             return norm ? PHA_RING(__nv_bfloat16, false, true)
                         : (neg ? PHA_RING(__nv_bfloat16, true, false)

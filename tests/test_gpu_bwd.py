@@ -97,10 +97,12 @@ def _ulp_bf16(x):
 
 
 @pytest.mark.parametrize("tables", ["stored", "factored"])
-@pytest.mark.parametrize("paired,stagger,dt", [(True, True, "bf16"), (False, False, "bf16"),
-                                               (True, True, "f32")])
-def test_rope_bwd_parity(paired, stagger, dt, tables):
-    H, Hkv, hd, T = (6, 6, 128, 700) if dt == "bf16" else (4, 2, 16, 64)
+@pytest.mark.parametrize("paired,stagger,dt,H,Hkv", [
+    (True, True, "bf16", 6, 6), (False, False, "bf16", 6, 6), (True, True, "f32", 4, 2),
+    (False, False, "bf16", 32, 8),   # 640 chunks a token: the factored kernel splits tokens
+])
+def test_rope_bwd_parity(paired, stagger, dt, H, Hkv, tables):
+    hd, T = (128, 700) if dt == "bf16" else (16, 64)
     w = synth.Workload("rb", (T,), H, Hkv, hd, dt, paired=paired, stagger=stagger,
                        positions="global")
     inp = synth.make_inputs(w)

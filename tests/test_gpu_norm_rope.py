@@ -36,6 +36,11 @@ CASES = [
     ("bf16", False, False, 256, 4, 2, 200, True, 1e-6),
     ("f32", False, False, 16, 2, 2, 64, True, 1e-6),
     ("f32", True, True, 128, 4, 2, 100, False, 1e-6),
+    # wider tokens than one ring slot of the factored kernel with the norm (192 chunks of 16
+    # bytes): 640, 416 and 384 chunks, split into segments of 4 x 160, 160 + 160 + 96 and 2 x 192
+    ("bf16", False, False, 128, 32, 8, 300, True, 1e-6),
+    ("bf16", True, True, 128, 20, 6, 200, True, 1e-6),
+    ("f32", True, True, 128, 6, 6, 100, True, 1e-6),
 ]
 
 

@@ -130,6 +130,11 @@ ROPE_CASES = [
     ("f32", False, False, 16, 2, 2, 64),
     ("f32", True, True, 16, 2, 2, 64),
     ("f32", True, True, 128, 4, 2, 100),
+    # wider tokens than one ring slot of the factored kernel (288 chunks of 16 bytes): 640, 416
+    # and 384 chunks, split into segments of 224 + 224 + 192, 224 + 192 and 2 x 192 chunks
+    ("bf16", False, False, 128, 32, 8, 500),
+    ("bf16", True, True, 128, 20, 6, 300),
+    ("f32", True, True, 128, 6, 6, 200),
 ]
 
 
