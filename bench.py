@@ -377,8 +377,9 @@ def main():
     # copies, kernels, device->host copies, chained per chunk by events. The copy-in stream thus
     # never waits for a kernel or a copy-out (the host->device link is the bound), and the
     # copy-out of one chunk runs beside the copy-in of the next. Every input byte is copied in and
-    # every output byte copied out within each timed step; a step starts after the previous one's
-    # copies out.
+    # every output byte copied out within each timed step. Steps follow each other as a stream of
+    # batches would: a chunk's buffers are refilled once the previous step's kernels on that chunk
+    # are done, and its outputs rewritten once the previous step's copy-out of them is done.
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "cu_seqlens", "positions")}
     if args.aux_v:
         host["aux_v"] = aux.cpu().pin_memory()
@@ -402,15 +403,17 @@ def main():
 
     ev_in = [torch.cuda.Event() for _ in parts]
     ev_k = [torch.cuda.Event() for _ in parts]
+    ev_out = [torch.cuda.Event() for _ in parts]
 
-    def e2e_step(first_event):
-        s_in.wait_event(first_event)
+    def e2e_step():
         for c, (st_, bufs, hsrc, t0, t1) in enumerate(parts):
+            s_in.wait_event(ev_k[c])  # the previous step's kernels on this chunk are done
             with torch.cuda.stream(s_in):
                 for n, t in bufs.items():
                     t.copy_(hsrc[n], non_blocking=True)
                 ev_in[c].record(s_in)
             s_comp.wait_event(ev_in[c])
+            s_comp.wait_event(ev_out[c])  # the previous step's outputs of this chunk are out
             with torch.cuda.stream(s_comp):
                 if args.qk_norm:
                     st_.norm_rope(bufs["q"], bufs["k"], bufs["positions"])
@@ -425,22 +428,25 @@ def main():
             with torch.cuda.stream(s_out):
                 o_host[t0:t1].copy_(o, non_blocking=True)
                 lse_host[t0:t1].copy_(lse, non_blocking=True)
+                ev_out[c].record(s_out)
+
+    def e2e_run(n_steps, start_event):
+        for sc in (s_in, s_comp, s_out):
+            sc.wait_event(start_event)
+        for _ in range(n_steps):
+            e2e_step()
         for sc in (s_in, s_comp, s_out):
             stream.wait_stream(sc)
 
-    for _ in range(3):
-        ev0 = torch.cuda.Event()
-        ev0.record(stream)
-        e2e_step(ev0)
+    ev0 = torch.cuda.Event()
+    ev0.record(stream)
+    e2e_run(3, ev0)
     torch.cuda.synchronize(dev)
     e_steps = max(5, min(args.steps, 20))
     pdist.barrier(dist)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(e_steps):
-        ev0 = torch.cuda.Event()
-        ev0.record(stream)
-        e2e_step(ev0)
+    e2e_run(e_steps, a)
     b.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = pdist.max_over_ranks(dist, a.elapsed_time(b) / e_steps, dev)
@@ -526,7 +532,8 @@ def main():
                 "chunks": len(parts),
                 "how": "public API from pinned host buffers, whole-document chunks on three "
                        "streams (copy-in, kernels, copy-out, chained by events: a chunk's copy-in "
-                       "overlaps the previous chunks' kernels and copy-out)"},
+                       "overlaps the previous chunks' kernels and copy-out, and the next step's "
+                       "copy-in the end of this one)"},
         "gpu_launches": 3 * args.steps,
         "work_items": n_items,
         "clocks": clk,
