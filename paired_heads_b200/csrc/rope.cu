@@ -360,6 +360,9 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_
                                                    const double2* __restrict__ fac) {
     constexpr int E = Chunk16<T>::E;
     const int cph = head_dim / E;                  // chunks per head row
+    // NORM: 1 / head_dim is exact (head_dim is a power of two here), so ss * inv_hd + eps rounds
+    // once, as ss / head_dim + eps does
+    const float inv_hd = 1.0f / static_cast<float>(head_dim);
     const int q_chunks = n_heads * cph;
     const int n_chunks = q_chunks + n_kv_heads * cph;
     const int lane = threadIdx.x & 31;
@@ -435,7 +438,7 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_
                         for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
                     }
                     for (int o = cph >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                    inv[j] = rsqrtf(ss / static_cast<float>(head_dim) + eps);
+                    inv[j] = rsqrtf(fmaf(ss, inv_hd, eps));
                 }
             } else if (!in_range) {
                 continue;  // positions outside the table: leave the token unchanged
@@ -525,6 +528,9 @@ __global__ void __launch_bounds__(256, MINB)
             wk[e] = b.x; wk[e + 1] = b.y; wk[e + 2] = b.z; wk[e + 3] = b.w;
         }
     }
+    // NORM: 1 / head_dim is exact (head_dim is a power of two here), so ss * inv_hd + eps rounds
+    // once, as ss / head_dim + eps does
+    const float inv_hd = 1.0f / static_cast<float>(head_dim);
     // unit u: token u / n_seg, chunks [c0, c1) with c0 = (u % n_seg) * seg
     auto token_of = [&](int64_t u) { return SEG ? u / n_seg : u; };
     auto issue = [&](int64_t u, int slot) {
@@ -577,7 +583,7 @@ __global__ void __launch_bounds__(256, MINB)
 #pragma unroll
                 for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
                 for (int o = cph >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                const float inv = rsqrtf(ss / static_cast<float>(head_dim) + eps);
+                const float inv = rsqrtf(fmaf(ss, inv_hd, eps));
                 if (!have) continue;
                 const bool is_q = i < q_chunks;
 #pragma unroll
