@@ -437,7 +437,9 @@ __global__ void __launch_bounds__(256, (rope_min_blocks<T, NORM, FACT>())) rope_
 #pragma unroll
                         for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
                     }
-                    for (int o = cph >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)  // offsets cph / 2 .. 1 (cph divides 32)
+                        if (o < cph) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                     inv[j] = rsqrtf(fmaf(ss, inv_hd, eps));
                 }
             } else if (!in_range) {
@@ -582,7 +584,9 @@ __global__ void __launch_bounds__(256, MINB)
                 float ss = 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
-                for (int o = cph >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)  // offsets cph / 2 .. 1 (cph divides 32)
+                    if (o < cph) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                 const float inv = rsqrtf(fmaf(ss, inv_hd, eps));
                 if (!have) continue;
                 const bool is_q = i < q_chunks;
