@@ -575,6 +575,7 @@ __global__ void __launch_bounds__(256, MINB)
         uint4* krow = reinterpret_cast<uint4*>(k + t * n_kv_heads * static_cast<int64_t>(head_dim));
         const uint8_t* src = ring + slot * slot_bytes;
         if (NORM) {  // normalised, then rotated when the position is inside the table
+#pragma unroll 2  // two rounds in flight (115.9 -> 114.3 us on the paired workload)
             for (int base = c0; base < c1; base += 32) {
                 const int i = base + lane;
                 const bool have = i < c1;
