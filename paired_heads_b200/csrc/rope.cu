@@ -671,10 +671,11 @@ static cudaError_t launch_rope_impl(void* q, void* k, const float* cos_tab, cons
 }
 
 // Ring depth and resident blocks of rope_ring_kernel: two slots per warp and three blocks per SM
-// (85 registers) for the rotation, three and three with the norm (measured on the paired
-// workload: depth 2 at 4 blocks with 64 registers 80 us, 84 us once the packed rotation needed
-// more registers than that; depth 2 at 3 blocks 78 us; depth 3 / 3 blocks 84 us, depth 4 / 2
-// blocks 98 us with an earlier rotation).
+// (up to 85 registers, which the rotation loop's unroll by two uses) for the rotation, three and
+// three with the norm (measured on the paired workload: depth 2 at 4 blocks with 64 registers
+// 80 us, 84 us once the packed rotation needed more registers than that; depth 2 at 3 blocks
+// 78 us, 76.4 us unrolled; depth 3 at 3 blocks 78.2 us unrolled, 84 us with an earlier rotation;
+// depth 4 at 2 blocks 98 us).
 template <bool NORM>
 constexpr int ring_depth() { return NORM ? 3 : 2; }
 template <bool NORM>
