@@ -97,12 +97,13 @@ def _ulp_bf16(x):
 
 
 @pytest.mark.parametrize("tables", ["stored", "factored"])
-@pytest.mark.parametrize("paired,stagger,dt,H,Hkv", [
-    (True, True, "bf16", 6, 6), (False, False, "bf16", 6, 6), (True, True, "f32", 4, 2),
-    (False, False, "bf16", 32, 8),   # 640 chunks a token: the factored kernel splits tokens
+@pytest.mark.parametrize("paired,stagger,dt,H,Hkv,T", [
+    (True, True, "bf16", 6, 6, 700), (False, False, "bf16", 6, 6, 700), (True, True, "f32", 4, 2, 64),
+    (False, False, "bf16", 32, 8, 700),  # 640 chunks a token: the factored kernel splits tokens
+    (True, True, "bf16", 6, 6, 5000),    # more tokens than the factored kernel's warps
 ])
-def test_rope_bwd_parity(paired, stagger, dt, H, Hkv, tables):
-    hd, T = (128, 700) if dt == "bf16" else (16, 64)
+def test_rope_bwd_parity(paired, stagger, dt, H, Hkv, T, tables):
+    hd = 128 if dt == "bf16" else 16
     w = synth.Workload("rb", (T,), H, Hkv, hd, dt, paired=paired, stagger=stagger,
                        positions="global")
     inp = synth.make_inputs(w)

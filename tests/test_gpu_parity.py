@@ -135,6 +135,10 @@ ROPE_CASES = [
     ("bf16", False, False, 128, 32, 8, 500),
     ("bf16", True, True, 128, 20, 6, 300),
     ("f32", True, True, 128, 6, 6, 200),
+    # more tokens than the factored kernel's warps (148 SMs x 24): several rounds, the last one
+    # partly filled
+    ("bf16", True, True, 128, 6, 6, 5000),
+    ("bf16", False, False, 64, 12, 4, 4001),
 ]
 
 
